@@ -1,0 +1,12 @@
+"""B200 (sm_100a) kernels for the MiniMax Sparse Attention hot path.
+
+The compute lives in ``libmsa.so`` (built from ``csrc/`` by ``build.py``);
+``msa`` is its ctypes binding.
+"""
+from . import msa  # noqa: F401
+from .msa import (  # noqa: F401
+    Shape, MsaError, lib, workspace_size, alloc_workspace, index_scores, block_topk,
+    sparse_attn_prefill, sparse_attn_decode, forward, dense_attn_prefill, dense_attn_decode,
+    device_status, OP_INDEX_SCORES, OP_BLOCK_TOPK, OP_SPARSE_PREFILL, OP_SPARSE_DECODE,
+    OP_FORWARD, OP_DENSE_PREFILL, OP_DENSE_DECODE,
+)

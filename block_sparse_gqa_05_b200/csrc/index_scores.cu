@@ -1,0 +1,439 @@
+// Index branch scoring with the block max-pool fused in (yhxrc.cn article on
+// the MSA figure, section 第一步: one index query per GQA group, one index key
+// shared by all heads, score Q_idx . K_idx, block max-pooling).
+//
+// Prefill: persistent tcgen05 GEMM.  A = 128 (token, group) rows of q_idx,
+// B = one 128-key block of k_idx, D = 128 x 128 fp32 scores in TMEM.  The
+// epilogue masks keys past each row's position and reduces the 128 columns to
+// one pooled value, so token scores never leave the SM.
+// Decode (T*G < 128): a bandwidth-bound scan of k_idx with mma.sync.
+#include <math.h>
+
+#include "internal.h"
+#include "ptx.cuh"
+
+namespace msa {
+namespace {
+
+constexpr int kStages = 6;
+constexpr int kAcc = 4;          // TMEM accumulator buffers of 128 columns
+constexpr int kThreads = 320;    // warp 0: TMA, warp 1: MMA, warps 2..9: epilogue
+constexpr int kChunkBlocks = 32; // key blocks per work item
+
+struct IdxParams {
+  float* pooled;
+  uint32_t* err;
+  int T, N, G, q_off, nb;
+  int M;         // row tiles per sequence = ceil(T*G / 128)
+  int tpt;       // tokens per row tile = 128 / G
+  int kc;        // key blocks per chunk
+  int C;         // chunks per sequence
+  long long items_per_seq;
+  long long items_total;
+};
+
+// First row tile whose causal key range reaches chunk c (tiles >= it are valid).
+__host__ __device__ inline int chunk_mmin(const IdxParams& p, int c) {
+  const long long need = static_cast<long long>(c) * p.kc * 128 - p.q_off + 1;
+  long long m = need <= 0 ? 0 : (need + p.tpt - 1) / p.tpt - 1;
+  if (m < 0) m = 0;
+  if (m > p.M - 1) m = p.M - 1;
+  return static_cast<int>(m);
+}
+
+// Number of causal key blocks of row tile m (blocks 0 .. ncb-1).
+__host__ __device__ inline int tile_causal_blocks(const IdxParams& p, int m) {
+  long long t_last = static_cast<long long>(p.tpt) * (m + 1) - 1;
+  if (t_last > p.T - 1) t_last = p.T - 1;
+  return static_cast<int>((p.q_off + t_last) / 128 + 1);
+}
+
+struct ItemCursor {
+  int seq = -1, c = 0, cnt = 0;
+  long long base = 0;
+};
+
+// Work items are ordered (sequence, chunk, row tile); each CTA walks its items
+// in increasing order, so the chunk cursor only moves forward.
+__device__ inline void item_decode(const IdxParams& p, long long w, ItemCursor& cur, int& seq,
+                                   int& m, int& b0, int& b1) {
+  const int s = static_cast<int>(w / p.items_per_seq);
+  const long long r = w - static_cast<long long>(s) * p.items_per_seq;
+  if (s != cur.seq) {
+    cur.seq = s;
+    cur.c = 0;
+    cur.base = 0;
+    cur.cnt = p.M - chunk_mmin(p, 0);
+  }
+  while (r >= cur.base + cur.cnt) {
+    cur.base += cur.cnt;
+    cur.c += 1;
+    cur.cnt = p.M - chunk_mmin(p, cur.c);
+  }
+  seq = s;
+  m = chunk_mmin(p, cur.c) + static_cast<int>(r - cur.base);
+  b0 = cur.c * p.kc;
+  const int ncb = tile_causal_blocks(p, m);
+  b1 = min(b0 + p.kc, ncb);
+}
+
+template <int DI>
+__global__ void __launch_bounds__(kThreads, 1)
+    index_scores_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
+                           const __grid_constant__ CUtensorMap tm_k, const IdxParams p) {
+  constexpr uint32_t kTile = 128u * DI * 2u;        // bytes of one 128-row operand tile
+  constexpr uint32_t kLayout = DI == 64 ? 2u : 4u;  // 128-byte / 64-byte swizzle
+  constexpr uint32_t kSbo = 8u * DI * 2u;           // 8-row swizzle atom
+  constexpr uint32_t kIdesc = idesc_bf16(128, 128, 0, 0);
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint8_t* qbuf = smem;
+  uint8_t* kbuf = smem + 2 * kTile;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(kbuf + kStages * kTile);
+  uint64_t* kfull = bars;
+  uint64_t* kempty = bars + kStages;
+  uint64_t* qfull = bars + 2 * kStages;
+  uint64_t* qempty = qfull + 2;
+  uint64_t* accfull = qempty + 2;
+  uint64_t* accempty = accfull + kAcc;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accempty + kAcc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kStages; ++i) {
+      mbar_init(&kfull[i], 1);
+      mbar_init(&kempty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&qfull[i], 1);
+      mbar_init(&qempty[i], 1);
+    }
+    for (int i = 0; i < kAcc; ++i) {
+      mbar_init(&accfull[i], 1);
+      mbar_init(&accempty[i], 128);
+    }
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) tmem_alloc(tmem_slot, 512);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      tma_prefetch_desc(&tm_q);
+      tma_prefetch_desc(&tm_k);
+      ItemCursor cur;
+      long long j = 0, q = 0;
+      bool ok = true;
+      for (long long w = blockIdx.x; ok && w < p.items_total; w += gridDim.x, ++q) {
+        int seq, m, b0, b1;
+        item_decode(p, w, cur, seq, m, b0, b1);
+        const int qb = static_cast<int>(q & 1);
+        if (!(ok = mbar_wait(&qempty[qb], ((q >> 1) & 1) ^ 1, abort_flag, p.err))) break;
+        mbar_arrive_expect_tx(&qfull[qb], kTile);
+        tma_load_2d(qbuf + qb * kTile, &tm_q, &qfull[qb], 0, seq * p.T * p.G + m * 128);
+        for (int b = b0; b < b1; ++b, ++j) {
+          const int s = static_cast<int>(j % kStages);
+          if (!(ok = mbar_wait(&kempty[s], ((j / kStages) & 1) ^ 1, abort_flag, p.err))) break;
+          mbar_arrive_expect_tx(&kfull[s], kTile);
+          tma_load_2d(kbuf + s * kTile, &tm_k, &kfull[s], 0, seq * p.N + b * 128);
+        }
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      ItemCursor cur;
+      long long j = 0, i = 0, q = 0;
+      bool ok = true;
+      for (long long w = blockIdx.x; ok && w < p.items_total; w += gridDim.x, ++q) {
+        int seq, m, b0, b1;
+        item_decode(p, w, cur, seq, m, b0, b1);
+        const int qb = static_cast<int>(q & 1);
+        if (!(ok = mbar_wait(&qfull[qb], (q >> 1) & 1, abort_flag, p.err))) break;
+        const uint32_t qaddr = smem_u32(qbuf + qb * kTile);
+        for (int b = b0; b < b1; ++b, ++j, ++i) {
+          const int s = static_cast<int>(j % kStages);
+          const int a = static_cast<int>(i % kAcc);
+          if (!(ok = mbar_wait(&kfull[s], (j / kStages) & 1, abort_flag, p.err))) break;
+          if (!(ok = mbar_wait(&accempty[a], ((i / kAcc) & 1) ^ 1, abort_flag, p.err))) break;
+          tc_fence_after();
+          const uint32_t kaddr = smem_u32(kbuf + s * kTile);
+#pragma unroll
+          for (int ks = 0; ks < DI / 16; ++ks) {
+            const uint64_t ad = smem_desc(qaddr + ks * 32, 16, kSbo, kLayout);
+            const uint64_t bd = smem_desc(kaddr + ks * 32, 16, kSbo, kLayout);
+            tc_mma_ss(tmem + a * 128, ad, bd, kIdesc, ks > 0 ? 1u : 0u);
+          }
+          tc_commit(&kempty[s]);
+          tc_commit(&accfull[a]);
+        }
+        if (ok) tc_commit(&qempty[qb]);
+      }
+    }
+    __syncwarp();
+  } else {
+    // --------------------------------------------- epilogue: mask + block max
+    const int wg = (warp - 2) >> 2;          // which accumulator buffers (parity)
+    const int quarter = warp & 3;            // TMEM lanes 32*quarter .. +31
+    const int row = quarter * 32 + lane;
+    const uint32_t taddr_row = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
+    ItemCursor cur;
+    long long i = 0;
+    bool ok = true;
+    const int rows_per_seq = p.T * p.G;
+    for (long long w = blockIdx.x; ok && w < p.items_total; w += gridDim.x) {
+      int seq, m, b0, b1;
+      item_decode(p, w, cur, seq, m, b0, b1);
+      const int trow = m * 128 + row;
+      const bool valid = trow < rows_per_seq;
+      const int t = trow / p.G;
+      const int pos = p.q_off + t;
+      const int bt = pos >> 7;
+      float* out = p.pooled + (static_cast<long long>(seq) * rows_per_seq + trow) *
+                                  static_cast<long long>(p.nb);
+      for (int b = b0; b < b1; ++b, ++i) {
+        if ((i & 1) != wg) continue;
+        const int a = static_cast<int>(i % kAcc);
+        if (!(ok = mbar_wait(&accfull[a], (i / kAcc) & 1, abort_flag, p.err))) break;
+        tc_fence_after();
+        float v[128];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) tmem_ld32(taddr_row + a * 128 + c * 32, v + c * 32);
+        tc_wait_ld();
+        tc_fence_before();
+        mbar_arrive(&accempty[a]);
+        if (valid && b <= bt) {
+          const int lim = (b == bt) ? (pos & 127) : 127;
+          float mx = -INFINITY;
+          if (lim == 127) {
+            float m4[4] = {v[0], v[1], v[2], v[3]};
+#pragma unroll
+            for (int c = 4; c < 128; c += 4) {
+              m4[0] = fmaxf(m4[0], v[c]);
+              m4[1] = fmaxf(m4[1], v[c + 1]);
+              m4[2] = fmaxf(m4[2], v[c + 2]);
+              m4[3] = fmaxf(m4[3], v[c + 3]);
+            }
+            mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
+          } else {
+#pragma unroll
+            for (int c = 0; c < 128; ++c) mx = fmaxf(mx, c <= lim ? v[c] : -INFINITY);
+          }
+          out[b] = mx;
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// pooled[row, b] = -inf for every b > b_t (rows are (seq, t, g)); one warp per row.
+__global__ void fill_upper_kernel(float* pooled, long long rows, int T, int G, int q_off,
+                                  int nb) {
+  const long long warps = static_cast<long long>(gridDim.x) * (blockDim.x >> 5);
+  for (long long r = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); r < rows; r += warps) {
+    const int t = static_cast<int>((r / G) % T);
+    const int bt = (q_off + t) >> 7;
+    float* out = pooled + r * nb;
+    for (int b = bt + 1 + (threadIdx.x & 31); b < nb; b += 32) out[b] = -INFINITY;
+  }
+}
+
+// --------------------------------------------------------------- decode scan
+// One CTA per (sequence*T + t, chunk of 8 blocks); warp w owns block 8*chunk+w.
+// S[key, group] = k_idx[key, :] . q_idx[t, group, :] on mma.sync m16n8k16 with
+// the 16 keys of a tile as rows and 8 groups as columns.  The K dimension is
+// permuted identically for both operands so that each thread reads contiguous
+// bytes: thread quad q holds index dims [q*4*KS, (q+1)*4*KS), and k-step ks
+// uses dims 4*ks .. 4*ks+3 of that range.
+__device__ __forceinline__ void mma_bf16_16816(float* d, const uint32_t* a, const uint32_t* b) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 "
+      "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
+}
+
+template <int DI>
+__global__ void __launch_bounds__(256) index_scores_scan_kernel(const uint16_t* __restrict__ q_idx,
+                                                                const uint16_t* __restrict__ k_idx,
+                                                                float* __restrict__ pooled, int T,
+                                                                int N, int G, int q_off, int nb) {
+  constexpr int KS = DI / 16;          // k-steps
+  constexpr int W = KS * 2;            // 32-bit words per thread per row
+  const int row_bt = blockIdx.y;       // seq * T + t
+  const int seq = row_bt / T;
+  const int t = row_bt - seq * T;
+  const int pos = q_off + t;
+  const int bt = pos >> 7;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int blk = blockIdx.x * 8 + warp;
+  if (blk > bt) return;
+  const int gq = lane >> 2, qd = lane & 3;
+  const uint16_t* kbase = k_idx + static_cast<long long>(seq) * N * DI;
+  for (int g0 = 0; g0 < G; g0 += 8) {
+    // B operand: index query of group g0 + gq, this thread's dim range
+    uint32_t bw[W];
+    const int grp = g0 + gq;
+    if (grp < G) {
+      const uint32_t* src = reinterpret_cast<const uint32_t*>(
+          q_idx + (static_cast<long long>(row_bt) * G + grp) * DI + qd * 4 * KS);
+#pragma unroll
+      for (int x = 0; x < W; ++x) bw[x] = src[x];
+    } else {
+#pragma unroll
+      for (int x = 0; x < W; ++x) bw[x] = 0u;
+    }
+    float mx0 = -INFINITY, mx1 = -INFINITY;
+#pragma unroll 2
+    for (int tile = 0; tile < 8; ++tile) {
+      const int key0 = blk * 128 + tile * 16 + gq;
+      const int key1 = key0 + 8;
+      uint32_t r0[W], r1[W];
+      if (key0 < N) {
+        const uint4* s0 = reinterpret_cast<const uint4*>(kbase + static_cast<long long>(key0) * DI +
+                                                         qd * 4 * KS);
+#pragma unroll
+        for (int x = 0; x < W / 4; ++x) {
+          uint4 u = __ldg(s0 + x);
+          r0[4 * x] = u.x; r0[4 * x + 1] = u.y; r0[4 * x + 2] = u.z; r0[4 * x + 3] = u.w;
+        }
+      } else {
+#pragma unroll
+        for (int x = 0; x < W; ++x) r0[x] = 0u;
+      }
+      if (key1 < N) {
+        const uint4* s1 = reinterpret_cast<const uint4*>(kbase + static_cast<long long>(key1) * DI +
+                                                         qd * 4 * KS);
+#pragma unroll
+        for (int x = 0; x < W / 4; ++x) {
+          uint4 u = __ldg(s1 + x);
+          r1[4 * x] = u.x; r1[4 * x + 1] = u.y; r1[4 * x + 2] = u.z; r1[4 * x + 3] = u.w;
+        }
+      } else {
+#pragma unroll
+        for (int x = 0; x < W; ++x) r1[x] = 0u;
+      }
+      float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int ks = 0; ks < KS; ++ks) {
+        const uint32_t a[4] = {r0[2 * ks], r1[2 * ks], r0[2 * ks + 1], r1[2 * ks + 1]};
+        const uint32_t b[2] = {bw[2 * ks], bw[2 * ks + 1]};
+        mma_bf16_16816(acc, a, b);
+      }
+      if (key0 <= pos) {
+        mx0 = fmaxf(mx0, acc[0]);
+        mx1 = fmaxf(mx1, acc[1]);
+      }
+      if (key1 <= pos) {
+        mx0 = fmaxf(mx0, acc[2]);
+        mx1 = fmaxf(mx1, acc[3]);
+      }
+    }
+#pragma unroll
+    for (int off = 4; off < 32; off <<= 1) {
+      mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, off));
+      mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, off));
+    }
+    if (gq == 0) {
+      const int ga = g0 + 2 * qd, gb = ga + 1;
+      float* out = pooled + static_cast<long long>(row_bt) * G * nb;
+      if (ga < G) out[static_cast<long long>(ga) * nb + blk] = mx0;
+      if (gb < G) out[static_cast<long long>(gb) * nb + blk] = mx1;
+    }
+  }
+}
+
+template <int DI>
+cudaError_t launch_tc(const msa_shape& s, const uint16_t* q_idx, const uint16_t* k_idx,
+                      float* pooled, const DevCtx* ctx, cudaStream_t st) {
+  IdxParams p{};
+  p.pooled = pooled;
+  p.err = ctx->err;
+  p.T = s.seq_q;
+  p.N = s.seq_kv;
+  p.G = s.n_kv_heads;
+  p.q_off = s.q_offset;
+  p.nb = static_cast<int>(ceil_div(s.seq_kv, 128));
+  p.tpt = 128 / p.G;
+  p.M = static_cast<int>(ceil_div(static_cast<int64_t>(p.T) * p.G, 128));
+  p.kc = kChunkBlocks;
+  p.C = static_cast<int>(ceil_div(static_cast<int64_t>(p.q_off) + p.T, p.kc * 128));
+  long long per = 0;
+  for (int c = 0; c < p.C; ++c) per += p.M - chunk_mmin(p, c);
+  p.items_per_seq = per;
+  p.items_total = per * s.batch;
+
+  CUtensorMap tq, tk;
+  const uint64_t dq[2] = {static_cast<uint64_t>(DI),
+                          static_cast<uint64_t>(s.batch) * s.seq_q * s.n_kv_heads};
+  const uint64_t dk[2] = {static_cast<uint64_t>(DI), static_cast<uint64_t>(s.batch) * s.seq_kv};
+  const uint64_t stride[1] = {static_cast<uint64_t>(DI) * 2};
+  const uint32_t box[2] = {static_cast<uint32_t>(DI), 128};
+  const CUtensorMapSwizzle sw =
+      DI == 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
+  if (!encode_tmap(&tq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, q_idx, dq, stride, box, sw) ||
+      !encode_tmap(&tk, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, k_idx, dk, stride, box, sw))
+    return cudaErrorInvalidValue;
+
+  const size_t smem = 1024 + (2 + kStages) * 128 * DI * 2 + 256;
+  cudaError_t e = cudaFuncSetAttribute(index_scores_tc_kernel<DI>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  const long long grid = p.items_total < ctx->num_sms ? p.items_total : ctx->num_sms;
+  index_scores_tc_kernel<DI><<<static_cast<unsigned>(grid), kThreads, smem, st>>>(tq, tk, p);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_index_scores(const msa_shape& s, const uint16_t* q_idx, const uint16_t* k_idx,
+                                float* pooled, bool fill_upper, cudaStream_t st) {
+  const DevCtx* ctx = device_ctx();
+  if (!ctx) return cudaErrorInitializationError;
+  const int nb = static_cast<int>(ceil_div(s.seq_kv, 128));
+  const long long rows = static_cast<long long>(s.batch) * s.seq_q * s.n_kv_heads;
+  cudaError_t e;
+  if (static_cast<long long>(s.seq_q) * s.n_kv_heads < 128) {
+    const int last_bt = (s.q_offset + s.seq_q - 1) / 128;
+    dim3 grid(static_cast<unsigned>(ceil_div(last_bt + 1, 8)),
+              static_cast<unsigned>(s.batch * s.seq_q));
+    if (s.index_dim == 64)
+      index_scores_scan_kernel<64><<<grid, 256, 0, st>>>(q_idx, k_idx, pooled, s.seq_q, s.seq_kv,
+                                                         s.n_kv_heads, s.q_offset, nb);
+    else
+      index_scores_scan_kernel<32><<<grid, 256, 0, st>>>(q_idx, k_idx, pooled, s.seq_q, s.seq_kv,
+                                                         s.n_kv_heads, s.q_offset, nb);
+    e = cudaGetLastError();
+  } else {
+    e = s.index_dim == 64 ? launch_tc<64>(s, q_idx, k_idx, pooled, ctx, st)
+                          : launch_tc<32>(s, q_idx, k_idx, pooled, ctx, st);
+  }
+  if (e != cudaSuccess || !fill_upper) return e;
+  const long long warps_needed = rows;
+  long long blocks = (warps_needed + 7) / 8;
+  if (blocks > 65535LL * 8) blocks = 65535LL * 8;
+  fill_upper_kernel<<<static_cast<unsigned>(blocks), 256, 0, st>>>(pooled, rows, s.seq_q,
+                                                                   s.n_kv_heads, s.q_offset, nb);
+  return cudaGetLastError();
+}
+
+}  // namespace msa

@@ -1,0 +1,49 @@
+// Host-side declarations shared by the translation units of libmsa.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "msa.h"
+
+namespace msa {
+
+// Per-device context: the device error word (a __device__ symbol) and SM count.
+struct DevCtx {
+  uint32_t* err = nullptr;
+  int num_sms = 0;
+  int device = -1;
+};
+
+// Returns nullptr if the CUDA runtime cannot be queried.
+const DevCtx* device_ctx();
+
+// TMA descriptor encoding through the driver entry point (no -lcuda link).
+bool encode_tmap(CUtensorMap* map, CUtensorMapDataType dtype, int rank, const void* base,
+                 const uint64_t* dims, const uint64_t* strides_bytes, const uint32_t* box,
+                 CUtensorMapSwizzle swizzle);
+
+inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// ---------------------------------------------------------------- launchers
+// Each returns cudaSuccess or the launch error.  Shapes are already validated.
+cudaError_t launch_index_scores(const msa_shape& s, const uint16_t* q_idx,
+                                const uint16_t* k_idx, float* pooled, bool fill_upper,
+                                cudaStream_t st);
+cudaError_t launch_block_topk(const msa_shape& s, const float* pooled, int32_t* sel,
+                              cudaStream_t st);
+size_t prefill_workspace_bytes(const msa_shape& s);
+cudaError_t launch_sparse_prefill(const msa_shape& s, const uint16_t* q, const uint16_t* k,
+                                  const uint16_t* v, const int32_t* sel, uint16_t* o,
+                                  float* lse, void* ws, cudaStream_t st);
+size_t decode_workspace_bytes(const msa_shape& s, bool dense);
+cudaError_t launch_decode(const msa_shape& s, const uint16_t* q, const uint16_t* k,
+                          const uint16_t* v, const int32_t* sel, uint16_t* o, float* lse,
+                          void* ws, bool dense, cudaStream_t st);
+cudaError_t launch_dense_prefill(const msa_shape& s, const uint16_t* q, const uint16_t* k,
+                                 const uint16_t* v, uint16_t* o, float* lse, cudaStream_t st);
+
+}  // namespace msa

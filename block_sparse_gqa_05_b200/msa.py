@@ -1,0 +1,211 @@
+"""Thin ctypes binding of libmsa (argument marshalling only).
+
+Every function takes CUDA torch tensors in the C-ABI layouts (see
+``include/msa.h``), passes their device pointers and the current CUDA stream
+to the library, and raises ``MsaError`` on a non-zero status.  Nothing here
+computes any part of the method: when the shared library is missing the
+import-time loader raises instead of falling back to anything else.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libmsa.so")
+HEADER_PATH = os.path.join(os.path.dirname(_PKG), "include", "msa.h")
+
+OP_INDEX_SCORES, OP_BLOCK_TOPK, OP_SPARSE_PREFILL, OP_SPARSE_DECODE, OP_FORWARD, \
+    OP_DENSE_PREFILL, OP_DENSE_DECODE = range(7)
+
+STATUS = {0: "MSA_OK", 1: "MSA_ERR_INVALID_SHAPE", 2: "MSA_ERR_NULL_PTR", 3: "MSA_ERR_MISALIGNED",
+          4: "MSA_ERR_WORKSPACE_TOO_SMALL", 5: "MSA_ERR_UNSUPPORTED", 6: "MSA_ERR_CUDA",
+          7: "MSA_ERR_DEVICE_TIMEOUT"}
+
+
+class MsaError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {STATUS.get(status, status)}")
+
+
+class Shape(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int) for n in (
+        "batch", "seq_q", "seq_kv", "q_offset", "n_q_heads", "n_kv_heads",
+        "head_dim", "index_dim", "block", "topk")]
+
+    @classmethod
+    def of(cls, spec) -> "Shape":
+        """From any object with the same attribute names (e.g. a WorkloadSpec)."""
+        return cls(*[int(getattr(spec, n)) for n, _ in cls._fields_])
+
+    @property
+    def nb(self) -> int:
+        return (self.seq_kv + self.block - 1) // self.block
+
+
+_vp = ctypes.c_void_p
+_SIGS = {
+    "msa_status_string": ([ctypes.c_int], ctypes.c_char_p),
+    "msa_workspace_size": ([ctypes.POINTER(Shape), ctypes.c_int, ctypes.POINTER(ctypes.c_size_t)],
+                           ctypes.c_int),
+    "msa_index_scores": ([ctypes.POINTER(Shape), _vp, _vp, _vp, _vp], ctypes.c_int),
+    "msa_block_topk": ([ctypes.POINTER(Shape), _vp, _vp, _vp], ctypes.c_int),
+    "msa_sparse_attn_prefill": ([ctypes.POINTER(Shape), _vp, _vp, _vp, _vp, _vp, _vp, _vp,
+                                 ctypes.c_size_t, _vp], ctypes.c_int),
+    "msa_sparse_attn_decode": ([ctypes.POINTER(Shape), _vp, _vp, _vp, _vp, _vp, _vp, _vp,
+                                ctypes.c_size_t, _vp], ctypes.c_int),
+    "msa_forward": ([ctypes.POINTER(Shape), _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
+                     ctypes.c_size_t, _vp], ctypes.c_int),
+    "msa_dense_attn_prefill": ([ctypes.POINTER(Shape), _vp, _vp, _vp, _vp, _vp, _vp,
+                                ctypes.c_size_t, _vp], ctypes.c_int),
+    "msa_dense_attn_decode": ([ctypes.POINTER(Shape), _vp, _vp, _vp, _vp, _vp, _vp,
+                               ctypes.c_size_t, _vp], ctypes.c_int),
+    "msa_device_status": ([ctypes.POINTER(ctypes.c_uint32)], ctypes.c_int),
+}
+
+_lib = None
+
+
+def lib():
+    """The loaded libmsa (raises if it was not built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"libmsa is not built ({LIB_PATH} missing); run "
+                              "python -m block_sparse_gqa_05_b200.build")
+        L = ctypes.CDLL(LIB_PATH)
+        for name, (args, res) in _SIGS.items():
+            fn = getattr(L, name)
+            fn.argtypes = args
+            fn.restype = res
+        _lib = L
+    return _lib
+
+
+def header_functions() -> list:
+    """Names of the functions ``include/msa.h`` declares."""
+    src = open(HEADER_PATH).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(msa_[a-z_]+)\s*\(", src)))
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("libmsa takes CUDA tensors")
+    if not t.is_contiguous():
+        raise ValueError("libmsa takes contiguous tensors")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _check(status: int, what: str):
+    if status != 0:
+        raise MsaError(status, what)
+
+
+def workspace_size(shape: Shape, op: int) -> int:
+    n = ctypes.c_size_t(0)
+    _check(lib().msa_workspace_size(ctypes.byref(shape), op, ctypes.byref(n)), "msa_workspace_size")
+    return int(n.value)
+
+
+def alloc_workspace(shape: Shape, op: int, device=None) -> torch.Tensor:
+    n = workspace_size(shape, op)
+    return torch.empty(max(n, 16), dtype=torch.uint8, device=device or "cuda")
+
+
+def index_scores(shape: Shape, q_idx, k_idx, pooled=None, stream=None):
+    if pooled is None:
+        pooled = torch.empty((shape.batch, shape.seq_q, shape.n_kv_heads, shape.nb),
+                             dtype=torch.float32, device=q_idx.device)
+    _check(lib().msa_index_scores(ctypes.byref(shape), _ptr(q_idx), _ptr(k_idx), _ptr(pooled),
+                                  _stream(stream)), "msa_index_scores")
+    return pooled
+
+
+def block_topk(shape: Shape, pooled, sel=None, stream=None):
+    if sel is None:
+        sel = torch.empty((shape.batch, shape.seq_q, shape.n_kv_heads, shape.topk),
+                          dtype=torch.int32, device=pooled.device)
+    _check(lib().msa_block_topk(ctypes.byref(shape), _ptr(pooled), _ptr(sel), _stream(stream)),
+           "msa_block_topk")
+    return sel
+
+
+def _attn_out(shape, q, o, lse, want_lse):
+    if o is None:
+        o = torch.empty_like(q)
+    if lse is None and want_lse:
+        lse = torch.empty((shape.batch, shape.seq_q, shape.n_q_heads), dtype=torch.float32,
+                          device=q.device)
+    return o, lse
+
+
+def sparse_attn_prefill(shape: Shape, q, k, v, sel, o=None, lse=None, ws=None, want_lse=True,
+                        stream=None):
+    o, lse = _attn_out(shape, q, o, lse, want_lse)
+    ws = alloc_workspace(shape, OP_SPARSE_PREFILL, q.device) if ws is None else ws
+    _check(lib().msa_sparse_attn_prefill(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(sel),
+                                         _ptr(o), _ptr(lse), _ptr(ws), ws.numel(), _stream(stream)),
+           "msa_sparse_attn_prefill")
+    return o, lse
+
+
+def sparse_attn_decode(shape: Shape, q, k, v, sel, o=None, lse=None, ws=None, want_lse=True,
+                       stream=None):
+    o, lse = _attn_out(shape, q, o, lse, want_lse)
+    ws = alloc_workspace(shape, OP_SPARSE_DECODE, q.device) if ws is None else ws
+    _check(lib().msa_sparse_attn_decode(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(sel),
+                                        _ptr(o), _ptr(lse), _ptr(ws), ws.numel(), _stream(stream)),
+           "msa_sparse_attn_decode")
+    return o, lse
+
+
+def forward(shape: Shape, q, k, v, q_idx, k_idx, o=None, lse=None, sel=None, ws=None,
+            want_lse=True, want_sel=True, stream=None):
+    o, lse = _attn_out(shape, q, o, lse, want_lse)
+    if sel is None and want_sel:
+        sel = torch.empty((shape.batch, shape.seq_q, shape.n_kv_heads, shape.topk),
+                          dtype=torch.int32, device=q.device)
+    ws = alloc_workspace(shape, OP_FORWARD, q.device) if ws is None else ws
+    _check(lib().msa_forward(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(q_idx),
+                             _ptr(k_idx), _ptr(o), _ptr(lse), _ptr(sel), _ptr(ws), ws.numel(),
+                             _stream(stream)), "msa_forward")
+    return o, lse, sel
+
+
+def dense_attn_prefill(shape: Shape, q, k, v, o=None, lse=None, want_lse=True, stream=None):
+    o, lse = _attn_out(shape, q, o, lse, want_lse)
+    _check(lib().msa_dense_attn_prefill(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(o),
+                                        _ptr(lse), None, 0, _stream(stream)),
+           "msa_dense_attn_prefill")
+    return o, lse
+
+
+def dense_attn_decode(shape: Shape, q, k, v, o=None, lse=None, ws=None, want_lse=True,
+                      stream=None):
+    o, lse = _attn_out(shape, q, o, lse, want_lse)
+    ws = alloc_workspace(shape, OP_DENSE_DECODE, q.device) if ws is None else ws
+    _check(lib().msa_dense_attn_decode(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(o),
+                                       _ptr(lse), _ptr(ws), ws.numel(), _stream(stream)),
+           "msa_dense_attn_decode")
+    return o, lse
+
+
+def device_status() -> int:
+    """Raw device error word (0 = no bounded wait expired); clears it."""
+    f = ctypes.c_uint32(0)
+    st = lib().msa_device_status(ctypes.byref(f))
+    if st not in (0, 7):
+        raise MsaError(st, "msa_device_status")
+    return int(f.value)

@@ -1,0 +1,177 @@
+/*
+ * libmsa -- B200 (sm_100a) kernels for the hot path of MiniMax Sparse Attention
+ * (MSA): index branch (block-pooled index scores -> per-group top-k blocks with
+ * the local block forced in) and main branch (exact softmax attention over the
+ * real K/V of the selected blocks, shared by every query head of a group).
+ *
+ * Sources of the definitions (web pages on the method):
+ *   [P2] hamidun.com, "MiniMax lança MSA: atenção esparsa acelera em 28 vezes…",
+ *        section "Como o MSA funciona" (index branch picks top-k KV blocks per
+ *        query and per GQA group; main branch runs exact attention on them).
+ *   [P3] yhxrc.cn article on the MSA figure, section 第一步 (index branch: one
+ *        index query per GQA group, one index key shared by all heads, score
+ *        Q_idx.K_idx, block max-pooling, TopK -> block index sets) and section
+ *        第二步 (sparse branch on the real K/V; Q1/Q2/Q3 share I1).
+ *   [P4] lumi-systems AI news on MSA (per-group independent top-k; exact
+ *        block-sparse attention; exponential-free top-k; KV-outer kernel).
+ *   [P5] lefilia.fr, "MiniMax Sparse Attention (MSA) : attention block-sparse à
+ *        deux branches…" (16 blocks of 128 tokens = 2,048-token budget; a local
+ *        block is always included).
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ * Shapes: B = batch, T = seq_q, N = seq_kv, H = n_q_heads, G = n_kv_heads
+ * (= index groups), r = H/G, d = head_dim, d_i = index_dim, Bk = block (128),
+ * k = topk (counts the local block), nb = ceil(N / Bk).
+ * Query row t of a sequence sits at absolute position p_t = q_offset + t; its
+ * local block is b_t = floor(p_t / Bk); its causal keys are 0..p_t.
+ * Blocks are aligned at position 0.  Head h belongs to group floor(h / r).
+ *
+ * Layouts (row-major, contiguous; bf16 values are passed as uint16_t bit
+ * patterns):
+ *   q, o     [B, T, H, d]   bf16        k, v   [B, G, N, d]  bf16
+ *   q_idx    [B, T, G, d_i] bf16        k_idx  [B, N, d_i]   bf16
+ *   pooled   [B, T, G, nb]  float32     sel    [B, T, G, k]  int32
+ *   lse      [B, T, H]      float32 (natural-log softmax normaliser; optional)
+ *
+ * Ownership: the caller allocates every buffer (device memory unless stated)
+ * and the optional workspace.  The library never allocates or frees device
+ * memory, never synchronises the stream, and all calls are asynchronous on
+ * ``stream`` (a cudaStream_t passed as void*; NULL = legacy default stream).
+ *
+ * Errors: shape, pointer and alignment checks run before any launch and return
+ * a status without touching the device.  Device pointers must be 16-byte
+ * aligned (TMA).  A failed launch returns MSA_ERR_CUDA.  Kernels never spin
+ * without a bound: a wait that exceeds its limit records a device error word
+ * read by msa_device_status() and the kernel returns early.
+ *
+ * Limits: Bk == 128; d in {64, 128}; d_i in {32, 64}; 1 <= k <= 64;
+ * r = H/G in {1, 2, 4, 8, 16}; G divides 128; q_offset + T <= N.
+ */
+#ifndef MSA_H_
+#define MSA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum msa_status {
+  MSA_OK = 0,
+  MSA_ERR_INVALID_SHAPE = 1,
+  MSA_ERR_NULL_PTR = 2,
+  MSA_ERR_MISALIGNED = 3,
+  MSA_ERR_WORKSPACE_TOO_SMALL = 4,
+  MSA_ERR_UNSUPPORTED = 5,
+  MSA_ERR_CUDA = 6,
+  MSA_ERR_DEVICE_TIMEOUT = 7
+} msa_status;
+
+typedef struct msa_shape {
+  int batch;       /* B  */
+  int seq_q;       /* T  */
+  int seq_kv;      /* N  */
+  int q_offset;    /* absolute position of query row 0 */
+  int n_q_heads;   /* H  */
+  int n_kv_heads;  /* G  (= index groups) */
+  int head_dim;    /* d  */
+  int index_dim;   /* d_i */
+  int block;       /* Bk (128) */
+  int topk;        /* k, including the local block */
+} msa_shape;
+
+/* Operations whose workspace size can be queried. */
+typedef enum msa_op {
+  MSA_OP_INDEX_SCORES = 0,
+  MSA_OP_BLOCK_TOPK = 1,
+  MSA_OP_SPARSE_PREFILL = 2,
+  MSA_OP_SPARSE_DECODE = 3,
+  MSA_OP_FORWARD = 4,
+  MSA_OP_DENSE_PREFILL = 5,
+  MSA_OP_DENSE_DECODE = 6
+} msa_op;
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char* msa_status_string(msa_status s);
+
+/* Bytes of device workspace ``op`` needs for ``shape`` (0 if none).
+ * Errors: MSA_ERR_NULL_PTR, MSA_ERR_INVALID_SHAPE, MSA_ERR_UNSUPPORTED. */
+msa_status msa_workspace_size(const msa_shape* shape, msa_op op, size_t* bytes);
+
+/* Index branch scoring, [P3] section 第一步 (and [P2] "Como o MSA funciona"):
+ *   pooled[b,t,g,j] = max over keys x of block j with x <= p_t of
+ *                     sum_c q_idx[b,t,g,c] * k_idx[b,x,c]      (fp32 accumulate)
+ *   pooled[b,t,g,j] = -inf for j > b_t.
+ * Token-level scores never reach memory (the block max is taken on chip).
+ * Prefill shapes run on tcgen05 tensor cores; T*G < 128 (decode) runs a
+ * bandwidth-bound scan of k_idx. */
+msa_status msa_index_scores(const msa_shape* shape, const uint16_t* q_idx,
+                            const uint16_t* k_idx, float* pooled, void* stream);
+
+/* Block top-k with the local block forced in, [P3] 第一步 (TopK), [P4]
+ * (per-group independent top-k, exponential-free), [P5] (local block always
+ * included; k blocks of Bk tokens):
+ *   sel[b,t,g,:] = {b_t} + the (k-1) best blocks of 0..b_t-1 under the order
+ *   (pooled descending, block index ascending), written in ascending block
+ *   order; when b_t + 1 <= k every causal block 0..b_t is taken and the
+ *   remaining slots are -1.  Reads pooled[..., 0..b_t] only. */
+msa_status msa_block_topk(const msa_shape* shape, const float* pooled, int32_t* sel,
+                          void* stream);
+
+/* Main branch, prefill, [P3] section 第二步, [P2], [P4] (exact block-sparse
+ * attention), [P5]:  for head h of group g = floor(h/r),
+ *   o[b,t,h,:] = sum_x softmax_x(q[b,t,h,:] . k[b,g,x,:] / sqrt(d)) v[b,g,x,:]
+ * over keys x in the blocks listed in sel[b,t,g,:] (entries -1 ignored) with
+ * x <= p_t.  Blocks listed must satisfy 0 <= block <= b_t.  lse may be NULL.
+ * ws/ws_bytes: workspace of at least msa_workspace_size(MSA_OP_SPARSE_PREFILL).
+ * KV-outer schedule ([P4]): each selected 128-row K/V block of a group is
+ * loaded once and reused by every (token, head) row that selected it. */
+msa_status msa_sparse_attn_prefill(const msa_shape* shape, const uint16_t* q,
+                                   const uint16_t* k, const uint16_t* v,
+                                   const int32_t* sel, uint16_t* o, float* lse,
+                                   void* ws, size_t ws_bytes, void* stream);
+
+/* Main branch, decode: same formula with T == 1 and q_offset == N - 1 (the new
+ * token is already the last cache row).  Split-K over the selected blocks
+ * with an in-kernel combine.  ws >= msa_workspace_size(MSA_OP_SPARSE_DECODE). */
+msa_status msa_sparse_attn_decode(const msa_shape* shape, const uint16_t* q,
+                                  const uint16_t* k, const uint16_t* v,
+                                  const int32_t* sel, uint16_t* o, float* lse,
+                                  void* ws, size_t ws_bytes, void* stream);
+
+/* Whole layer: index scores -> top-k -> sparse attention (prefill path when
+ * T > 1, decode path when T == 1), one stream, no host synchronisation.
+ * sel_out (may be NULL) receives the selection.  ws >= msa_workspace_size(
+ * MSA_OP_FORWARD); the pooled scores live in the workspace and entries with
+ * j > b_t are left unwritten there. */
+msa_status msa_forward(const msa_shape* shape, const uint16_t* q, const uint16_t* k,
+                       const uint16_t* v, const uint16_t* q_idx, const uint16_t* k_idx,
+                       uint16_t* o, float* lse, int32_t* sel_out, void* ws,
+                       size_t ws_bytes, void* stream);
+
+/* Dense causal GQA attention (every key x <= p_t), the baseline the pages
+ * compare MSA against ([P1] GQA definition; [P2], [P4] speed-ups vs GQA).
+ * Prefill: q-outer flash attention, no workspace needed (pass NULL/0). */
+msa_status msa_dense_attn_prefill(const msa_shape* shape, const uint16_t* q,
+                                  const uint16_t* k, const uint16_t* v, uint16_t* o,
+                                  float* lse, void* ws, size_t ws_bytes, void* stream);
+
+/* Dense causal GQA decode (T == 1): split-K over all causal blocks.
+ * ws >= msa_workspace_size(MSA_OP_DENSE_DECODE). */
+msa_status msa_dense_attn_decode(const msa_shape* shape, const uint16_t* q,
+                                 const uint16_t* k, const uint16_t* v, uint16_t* o,
+                                 float* lse, void* ws, size_t ws_bytes, void* stream);
+
+/* Reads and clears the device error word of the current device (bit 0: a
+ * bounded wait timed out).  Synchronises the current device.  Returns
+ * MSA_ERR_DEVICE_TIMEOUT if any bit was set, MSA_OK otherwise; *flags (may be
+ * NULL) receives the raw word. */
+msa_status msa_device_status(uint32_t* flags);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MSA_H_ */

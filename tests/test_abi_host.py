@@ -1,0 +1,94 @@
+"""C-ABI checks that need no GPU: the library loads, exports every symbol the
+header declares, and rejects bad arguments before touching the device."""
+import ctypes
+
+import pytest
+
+import block_sparse_gqa_05_b200 as M
+from block_sparse_gqa_05_b200 import msa as B
+
+
+@pytest.fixture(scope="module")
+def L():
+    return B.lib()
+
+
+def tiny(**kw):
+    d = dict(batch=1, seq_q=2048, seq_kv=2048, q_offset=0, n_q_heads=8, n_kv_heads=2,
+             head_dim=64, index_dim=32, block=128, topk=4)
+    d.update(kw)
+    return M.Shape(**d)
+
+
+def test_exports_every_header_symbol(L):
+    names = B.header_functions()
+    assert len(names) >= 10
+    for n in names:
+        assert hasattr(L, n), n
+
+
+def test_status_strings(L):
+    for code in range(8):
+        s = L.msa_status_string(code).decode()
+        assert s.startswith(B.STATUS[code])
+
+
+def ws(shape, op):
+    n = ctypes.c_size_t(123)
+    st = B.lib().msa_workspace_size(ctypes.byref(shape), op, ctypes.byref(n))
+    return st, n.value
+
+
+def test_workspace_sizes_and_validation():
+    st, n = ws(tiny(), M.OP_INDEX_SCORES)
+    assert st == 0 and n == 0
+    st, pre = ws(tiny(), M.OP_SPARSE_PREFILL)
+    assert st == 0
+    # partial outputs alone: B*T*H*k*d bf16 + B*T*H*k lse
+    assert pre >= 2048 * 8 * 4 * 64 * 2 + 2048 * 8 * 4 * 4
+    st, fwd = ws(tiny(), M.OP_FORWARD)
+    assert st == 0 and fwd >= pre + 2048 * 2 * 16 * 4 + 2048 * 2 * 4 * 4
+    dec = tiny(batch=3, seq_q=1, seq_kv=5000, q_offset=4999)
+    st, n = ws(dec, M.OP_SPARSE_DECODE)
+    assert st == 0 and n >= 3 * 8 * 4 * 64 * 4
+    st, nd = ws(dec, M.OP_DENSE_DECODE)
+    assert st == 0 and nd > 0
+    # decode needs T == 1 and q_offset == N - 1
+    assert ws(tiny(batch=3, seq_q=1, seq_kv=5000, q_offset=10), M.OP_SPARSE_DECODE)[0] == 1
+    assert ws(tiny(), M.OP_SPARSE_DECODE)[0] == 1
+
+
+@pytest.mark.parametrize("bad,code", [
+    (dict(block=64), 5), (dict(topk=0), 1), (dict(topk=65), 5), (dict(head_dim=96), 5),
+    (dict(index_dim=48), 5), (dict(n_q_heads=7), 1), (dict(n_q_heads=6), 5), (dict(n_kv_heads=3, n_q_heads=6), 5),
+    (dict(n_q_heads=64, n_kv_heads=2), 5), (dict(q_offset=1), 1), (dict(seq_q=0), 1),
+    (dict(batch=0), 1),
+])
+def test_shape_validation(bad, code):
+    assert ws(tiny(**bad), M.OP_FORWARD)[0] == code
+
+
+def test_pointer_checks_precede_device_use(L):
+    s = tiny()
+    ok = ctypes.c_void_p(1 << 20)           # never dereferenced: validation fails first
+    mis = ctypes.c_void_p((1 << 20) + 8)
+    assert L.msa_index_scores(ctypes.byref(s), None, ok, ok, None) == 2
+    assert L.msa_index_scores(ctypes.byref(s), mis, ok, ok, None) == 3
+    assert L.msa_block_topk(ctypes.byref(s), ok, None, None) == 2
+    assert L.msa_sparse_attn_prefill(ctypes.byref(s), ok, ok, ok, ok, ok, None, None, 0, None) == 2
+    assert L.msa_sparse_attn_prefill(ctypes.byref(s), ok, ok, ok, ok, ok, None, ok, 16, None) == 4
+    bad = tiny(block=256)
+    assert L.msa_forward(ctypes.byref(bad), ok, ok, ok, ok, ok, ok, None, None, ok, 1 << 40,
+                         None) == 5
+    dec = tiny(seq_q=1, seq_kv=4096, q_offset=4095)
+    assert L.msa_sparse_attn_decode(ctypes.byref(dec), ok, ok, ok, ok, ok, None, ok, 8, None) == 4
+    assert L.msa_dense_attn_decode(ctypes.byref(s), ok, ok, ok, ok, None, ok, 1 << 30, None) == 1
+
+
+def test_binding_rejects_cpu_tensors():
+    import torch
+    s = tiny()
+    with pytest.raises(ValueError):
+        M.index_scores(s, torch.zeros(1, 2048, 2, 32, dtype=torch.bfloat16),
+                       torch.zeros(1, 2048, 32, dtype=torch.bfloat16),
+                       pooled=torch.zeros(1, 2048, 2, 16))

@@ -1,0 +1,194 @@
+"""GPU parity of every libmsa entry point against the CPU oracle (through the C ABI).
+
+Index scores and selections are compared bit for bit (integer-valued index
+inputs make every score exact in fp32); attention outputs, fed the same
+selection on both sides, within max-abs 1e-2 / mean-abs 1e-3 of the fp64
+oracle.  Shapes span several tiles and ragged tails.
+"""
+import numpy as np
+import pytest
+import torch
+
+import block_sparse_gqa_05_b200 as M
+import oracle as O
+import synth
+from tests.gpu_helpers import (spec, inputs_cpu, positions, oracle_pooled, oracle_sel,
+                               check_pooled, check_attn, oracle_attention, cuda, LSE_ABS)
+
+pytestmark = pytest.mark.gpu
+
+TINY = synth.workload("tiny_prefill_2k")
+# batch 2, rows T*G not a multiple of 128, q_offset > 0, N not a multiple of 128
+RAGGED = spec(2, 300, 1000, 700, 16, 4, 64, 64, 5, seed=11)
+RAGGED_R8 = spec(2, 300, 1000, 700, 16, 2, 128, 64, 5, seed=12)
+
+
+@pytest.fixture(scope="module")
+def tiny_inputs():
+    return inputs_cpu(TINY)
+
+
+@pytest.fixture(scope="module")
+def tiny_oracle(tiny_inputs):
+    pooled = oracle_pooled(TINY, tiny_inputs, 0)
+    sel = oracle_sel(TINY, pooled)
+    return pooled, sel
+
+
+# ------------------------------------------------------------ index scores
+def test_index_scores_tiny(tiny_inputs, tiny_oracle):
+    sh = M.Shape.of(TINY)
+    pooled = M.index_scores(sh, cuda(tiny_inputs.q_idx), cuda(tiny_inputs.k_idx))
+    torch.cuda.synchronize()
+    check_pooled(pooled[0], tiny_oracle[0], TINY)
+
+
+@pytest.mark.parametrize("sp", [RAGGED, spec(1, 640, 9000, 8000, 8, 8, 64, 64, 16, seed=3),
+                                spec(1, 513, 513, 0, 8, 1, 64, 32, 4, seed=4)])
+def test_index_scores_ragged(sp):
+    inp = inputs_cpu(sp, ("q_idx", "k_idx"))
+    pooled = M.index_scores(M.Shape.of(sp), cuda(inp.q_idx), cuda(inp.k_idx))
+    torch.cuda.synchronize()
+    for b in range(sp.batch):
+        check_pooled(pooled[b], oracle_pooled(sp, inp, b), sp)
+
+
+@pytest.mark.parametrize("sp", [spec(3, 1, 3000, 2999, 16, 8, 128, 64, 16, seed=5),
+                                spec(2, 1, 1100, 1099, 8, 2, 64, 32, 4, seed=6),
+                                spec(2, 3, 700, 690, 8, 4, 64, 64, 4, seed=8)])
+def test_index_scores_decode_scan(sp):
+    inp = inputs_cpu(sp, ("q_idx", "k_idx"))
+    pooled = M.index_scores(M.Shape.of(sp), cuda(inp.q_idx), cuda(inp.k_idx))
+    torch.cuda.synchronize()
+    for b in range(sp.batch):
+        check_pooled(pooled[b], oracle_pooled(sp, inp, b), sp)
+
+
+# ------------------------------------------------------------------ top-k
+def test_topk_on_oracle_pooled(tiny_oracle):
+    pooled, sel_ref = tiny_oracle
+    sh = M.Shape.of(TINY)
+    pl = torch.from_numpy(pooled.astype(np.float32))[None]
+    sel = M.block_topk(sh, cuda(pl))
+    torch.cuda.synchronize()
+    assert np.array_equal(sel[0].cpu().numpy(), sel_ref)
+
+
+def _random_pooled(sp, gen, lo, hi, integer=True):
+    nb = sp.nb
+    if integer:
+        x = torch.randint(lo, hi + 1, (sp.batch, sp.seq_q, sp.n_kv_heads, nb), generator=gen).float()
+    else:
+        x = torch.randn((sp.batch, sp.seq_q, sp.n_kv_heads, nb), generator=gen)
+    return x
+
+
+@pytest.mark.parametrize("sp,lo,hi", [
+    (spec(1, 4096, 4096 + 9000, 9000, 8, 8, 64, 64, 16), -3, 3),        # heavy ties
+    (spec(1, 2000, 2000 + 1100, 1100, 8, 4, 64, 64, 16), -200, 200),    # nb % 4 != 0
+    (spec(2, 300, 5000, 4700, 16, 8, 64, 64, 64), -5, 5),               # k = 64: general merge
+    (spec(1, 500, 6000, 5500, 16, 8, 64, 64, 33), -1000, 1000),         # k-1 = 32
+    (spec(64, 1, 300000, 299999, 64, 8, 64, 64, 16), -50, 50),          # 2344 blocks: 3 chunks
+    (spec(16, 1, 300000, 299999, 64, 8, 64, 64, 16), 0, 0),             # all equal, long rows
+    (spec(1, 1500, 1500, 0, 8, 8, 64, 64, 1), -3, 3),                   # k = 1: local only
+])
+def test_topk_random_scores(sp, lo, hi):
+    gen = torch.Generator().manual_seed(sp.seq_q + sp.topk)
+    pl = _random_pooled(sp, gen, lo, hi)
+    sel = M.block_topk(M.Shape.of(sp), cuda(pl))
+    torch.cuda.synchronize()
+    got = sel.cpu().numpy()
+    for b in range(sp.batch):
+        ref = O.block_topk(pl[b].double().numpy(), positions(sp), sp.block, sp.topk)
+        assert np.array_equal(got[b], ref), np.argwhere(got[b] != ref)[:5]
+
+
+def test_topk_real_valued_scores():
+    sp = spec(1, 3000, 3000 + 20000, 20000, 8, 8, 64, 64, 16)
+    gen = torch.Generator().manual_seed(99)
+    pl = _random_pooled(sp, gen, 0, 0, integer=False)
+    sel = M.block_topk(M.Shape.of(sp), cuda(pl))
+    torch.cuda.synchronize()
+    ref = O.block_topk(pl[0].double().numpy(), positions(sp), sp.block, sp.topk)
+    assert np.array_equal(sel[0].cpu().numpy(), ref)
+
+
+# ------------------------------------------------------- sparse attention
+def test_sparse_prefill_tiny(tiny_inputs, tiny_oracle):
+    _, sel_ref = tiny_oracle
+    sh = M.Shape.of(TINY)
+    sel = cuda(torch.from_numpy(sel_ref)[None])
+    o, lse = M.sparse_attn_prefill(sh, cuda(tiny_inputs.q), cuda(tiny_inputs.k),
+                                   cuda(tiny_inputs.v), sel)
+    torch.cuda.synchronize()
+    O_ref, L_ref = oracle_attention(TINY, tiny_inputs, sel_ref, 0)
+    check_attn(o[0], O_ref, "tiny prefill")
+    assert np.abs(lse[0].double().cpu().numpy() - L_ref).max() < LSE_ABS
+
+
+@pytest.mark.parametrize("sp", [RAGGED, RAGGED_R8])
+def test_sparse_prefill_ragged(sp):
+    inp = inputs_cpu(sp)
+    sels = [oracle_sel(sp, oracle_pooled(sp, inp, b)) for b in range(sp.batch)]
+    sel = cuda(torch.from_numpy(np.stack(sels)))
+    o, lse = M.sparse_attn_prefill(M.Shape.of(sp), cuda(inp.q), cuda(inp.k), cuda(inp.v), sel)
+    torch.cuda.synchronize()
+    for b in range(sp.batch):
+        O_ref, L_ref = oracle_attention(sp, inp, sels[b], b)
+        check_attn(o[b], O_ref, f"ragged prefill b={b}")
+        assert np.abs(lse[b].double().cpu().numpy() - L_ref).max() < LSE_ABS
+
+
+@pytest.mark.parametrize("sp", [spec(3, 1, 3000, 2999, 16, 2, 128, 64, 4, seed=21),
+                                spec(2, 1, 5000, 4999, 8, 2, 64, 32, 16, seed=22),
+                                spec(2, 1, 129, 128, 16, 1, 128, 64, 16, seed=23)])
+def test_sparse_decode(sp):
+    inp = inputs_cpu(sp)
+    sels = [oracle_sel(sp, oracle_pooled(sp, inp, b)) for b in range(sp.batch)]
+    sel = cuda(torch.from_numpy(np.stack(sels)))
+    o, lse = M.sparse_attn_decode(M.Shape.of(sp), cuda(inp.q), cuda(inp.k), cuda(inp.v), sel)
+    torch.cuda.synchronize()
+    for b in range(sp.batch):
+        O_ref, L_ref = oracle_attention(sp, inp, sels[b], b)
+        check_attn(o[b], O_ref, f"decode b={b}")
+        assert np.abs(lse[b].double().cpu().numpy() - L_ref).max() < LSE_ABS
+
+
+def test_dense_decode():
+    sp = spec(2, 1, 4000, 3999, 16, 2, 128, 64, 4, seed=31)
+    inp = inputs_cpu(sp)
+    o, lse = M.dense_attn_decode(M.Shape.of(sp), cuda(inp.q), cuda(inp.k), cuda(inp.v))
+    torch.cuda.synchronize()
+    for b in range(sp.batch):
+        O_ref, L_ref = O.dense_attention(inp.q[b], inp.k[b], inp.v[b], positions(sp))
+        check_attn(o[b], O_ref, f"dense decode b={b}")
+        assert np.abs(lse[b].double().cpu().numpy() - L_ref).max() < LSE_ABS
+
+
+# ------------------------------------------------------------- whole layer
+def test_forward_tiny(tiny_inputs, tiny_oracle):
+    pooled_ref, sel_ref = tiny_oracle
+    sh = M.Shape.of(TINY)
+    o, lse, sel = M.forward(sh, cuda(tiny_inputs.q), cuda(tiny_inputs.k), cuda(tiny_inputs.v),
+                            cuda(tiny_inputs.q_idx), cuda(tiny_inputs.k_idx))
+    torch.cuda.synchronize()
+    assert np.array_equal(sel[0].cpu().numpy(), sel_ref)
+    O_ref, _ = oracle_attention(TINY, tiny_inputs, sel_ref, 0)
+    check_attn(o[0], O_ref, "forward tiny")
+
+
+def test_forward_decode():
+    sp = spec(4, 1, 20000, 19999, 16, 2, 128, 64, 16, seed=41, planted=4)
+    inp = inputs_cpu(sp)
+    o, lse, sel = M.forward(M.Shape.of(sp), cuda(inp.q), cuda(inp.k), cuda(inp.v),
+                            cuda(inp.q_idx), cuda(inp.k_idx))
+    torch.cuda.synchronize()
+    for b in range(sp.batch):
+        sref = oracle_sel(sp, oracle_pooled(sp, inp, b))
+        assert np.array_equal(sel[b].cpu().numpy(), sref)
+        O_ref, _ = oracle_attention(sp, inp, sref, b)
+        check_attn(o[b], O_ref, f"forward decode b={b}")
+
+
+def test_device_status_clean():
+    assert M.device_status() == 0
