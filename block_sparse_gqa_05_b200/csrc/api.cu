@@ -1,5 +1,8 @@
 // C ABI of libmsa: validation, workspace sizing and dispatch (see include/msa.h).
+#include <atomic>
+#include <cstring>
 #include <mutex>
+#include <vector>
 
 #include "internal.h"
 
@@ -75,7 +78,72 @@ bool forward_is_decode(const msa_shape& s) {
 
 msa_status from_cuda(cudaError_t e) { return e == cudaSuccess ? MSA_OK : MSA_ERR_CUDA; }
 
+// ------------------------------------------------------------- profiling
+struct ProfRecord {
+  const char* name;
+  cudaEvent_t a, b;
+};
+struct ProfEntry {
+  const char* name;
+  double ms;
+  long long launches;
+};
+std::atomic<bool> g_prof_on{false};
+std::mutex g_prof_mu;
+std::vector<ProfRecord> g_prof_pending;
+std::vector<cudaEvent_t> g_prof_free;
+std::vector<ProfEntry> g_prof_table;
+
+cudaEvent_t prof_event() {
+  if (!g_prof_free.empty()) {
+    cudaEvent_t e = g_prof_free.back();
+    g_prof_free.pop_back();
+    return e;
+  }
+  cudaEvent_t e = nullptr;
+  if (cudaEventCreate(&e) != cudaSuccess) return nullptr;
+  return e;
+}
+
+bool prof_drain() {
+  bool ok = true;
+  for (const ProfRecord& r : g_prof_pending) {
+    float ms = 0.f;
+    if (cudaEventSynchronize(r.b) != cudaSuccess || cudaEventElapsedTime(&ms, r.a, r.b) != cudaSuccess)
+      ok = false;
+    ProfEntry* e = nullptr;
+    for (ProfEntry& x : g_prof_table)
+      if (std::strcmp(x.name, r.name) == 0) e = &x;
+    if (!e) {
+      g_prof_table.push_back(ProfEntry{r.name, 0.0, 0});
+      e = &g_prof_table.back();
+    }
+    e->ms += ms;
+    e->launches += 1;
+    g_prof_free.push_back(r.a);
+    g_prof_free.push_back(r.b);
+  }
+  g_prof_pending.clear();
+  return ok;
+}
+
 }  // namespace
+
+ProfScope::ProfScope(const char* name, cudaStream_t st) : st_(st) {
+  if (!g_prof_on.load(std::memory_order_relaxed)) return;
+  std::lock_guard<std::mutex> lk(g_prof_mu);
+  cudaEvent_t a = prof_event(), b = prof_event();
+  if (!a || !b || cudaEventRecord(a, st) != cudaSuccess) return;
+  g_prof_pending.push_back(ProfRecord{name, a, b});
+  slot_ = static_cast<int>(g_prof_pending.size()) - 1;
+}
+
+ProfScope::~ProfScope() {
+  if (slot_ < 0) return;
+  std::lock_guard<std::mutex> lk(g_prof_mu);
+  if (slot_ < static_cast<int>(g_prof_pending.size()))
+    cudaEventRecord(g_prof_pending[slot_].b, st_);
+}
 
 const DevCtx* device_ctx() {
   int dev = -1;
@@ -292,6 +360,27 @@ msa_status msa_dense_attn_decode(const msa_shape* s, const uint16_t* q, const ui
   if (!device_ctx()) return MSA_ERR_CUDA;
   return from_cuda(launch_decode(*s, q, k, v, nullptr, o, lse, ws, true,
                                  static_cast<cudaStream_t>(stream)));
+}
+
+msa_status msa_profile_enable(int on) {
+  std::lock_guard<std::mutex> lk(g_prof_mu);
+  if (on) {
+    prof_drain();
+    g_prof_table.clear();
+  }
+  g_prof_on.store(on != 0);
+  return MSA_OK;
+}
+
+msa_status msa_profile_read(int index, const char** name, double* total_ms, long long* launches) {
+  std::lock_guard<std::mutex> lk(g_prof_mu);
+  if (!prof_drain()) return MSA_ERR_CUDA;
+  if (index < 0 || index >= static_cast<int>(g_prof_table.size())) return MSA_ERR_INVALID_SHAPE;
+  const ProfEntry& e = g_prof_table[index];
+  if (name) *name = e.name;
+  if (total_ms) *total_ms = e.ms;
+  if (launches) *launches = e.launches;
+  return MSA_OK;
 }
 
 msa_status msa_device_status(uint32_t* flags) {

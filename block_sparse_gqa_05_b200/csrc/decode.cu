@@ -373,12 +373,18 @@ cudaError_t launch_decode(const msa_shape& s, const uint16_t* q, const uint16_t*
     e = cudaFuncSetAttribute(decode_attn_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(smem));
     if (e != cudaSuccess) return e;
+    {
+    ProfScope ps_("decode_attn", st);
     decode_attn_kernel<128><<<grid, kThreads, smem, st>>>(tk, tv, p);
+  }
   } else {
     e = cudaFuncSetAttribute(decode_attn_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(smem));
     if (e != cudaSuccess) return e;
+    {
+    ProfScope ps_("decode_attn", st);
     decode_attn_kernel<64><<<grid, kThreads, smem, st>>>(tk, tv, p);
+  }
   }
   return cudaGetLastError();
 }

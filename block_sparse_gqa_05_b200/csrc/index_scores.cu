@@ -399,7 +399,10 @@ cudaError_t launch_tc(const msa_shape& s, const uint16_t* q_idx, const uint16_t*
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   const long long grid = p.items_total < ctx->num_sms ? p.items_total : ctx->num_sms;
-  index_scores_tc_kernel<DI><<<static_cast<unsigned>(grid), kThreads, smem, st>>>(tq, tk, p);
+  {
+    ProfScope ps_("index_scores_tc", st);
+    index_scores_tc_kernel<DI><<<static_cast<unsigned>(grid), kThreads, smem, st>>>(tq, tk, p);
+  }
   return cudaGetLastError();
 }
 
@@ -417,11 +420,17 @@ cudaError_t launch_index_scores(const msa_shape& s, const uint16_t* q_idx, const
     dim3 grid(static_cast<unsigned>(ceil_div(last_bt + 1, 8)),
               static_cast<unsigned>(s.batch * s.seq_q));
     if (s.index_dim == 64)
-      index_scores_scan_kernel<64><<<grid, 256, 0, st>>>(q_idx, k_idx, pooled, s.seq_q, s.seq_kv,
+      {
+    ProfScope ps_("index_scores_scan", st);
+    index_scores_scan_kernel<64><<<grid, 256, 0, st>>>(q_idx, k_idx, pooled, s.seq_q, s.seq_kv,
                                                          s.n_kv_heads, s.q_offset, nb);
+  }
     else
-      index_scores_scan_kernel<32><<<grid, 256, 0, st>>>(q_idx, k_idx, pooled, s.seq_q, s.seq_kv,
+      {
+    ProfScope ps_("index_scores_scan", st);
+    index_scores_scan_kernel<32><<<grid, 256, 0, st>>>(q_idx, k_idx, pooled, s.seq_q, s.seq_kv,
                                                          s.n_kv_heads, s.q_offset, nb);
+  }
     e = cudaGetLastError();
   } else {
     e = s.index_dim == 64 ? launch_tc<64>(s, q_idx, k_idx, pooled, ctx, st)
@@ -431,8 +440,11 @@ cudaError_t launch_index_scores(const msa_shape& s, const uint16_t* q_idx, const
   const long long warps_needed = rows;
   long long blocks = (warps_needed + 7) / 8;
   if (blocks > 65535LL * 8) blocks = 65535LL * 8;
-  fill_upper_kernel<<<static_cast<unsigned>(blocks), 256, 0, st>>>(pooled, rows, s.seq_q,
+  {
+    ProfScope ps_("fill_upper", st);
+    fill_upper_kernel<<<static_cast<unsigned>(blocks), 256, 0, st>>>(pooled, rows, s.seq_q,
                                                                    s.n_kv_heads, s.q_offset, nb);
+  }
   return cudaGetLastError();
 }
 

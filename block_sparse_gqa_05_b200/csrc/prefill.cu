@@ -33,8 +33,8 @@ struct PrefillWs {
   uint32_t* tile_off;    // [ncol + 1]
   uint32_t* entries;     // [B*T*G*k]   (t << 6) | slot
   int4* tiles;           // [max_tiles] (column, entry start, count, 0)
-  uint16_t* part_o;      // [B, T, H, k, d] bf16
-  float* part_lse;       // [B, T, H, k]   log2 units
+  uint16_t* part_o;      // [B, T, k, H, d] bf16, normalised partial outputs
+  float* part_lse;       // [B, T, k, H]    log-sum-exp of each partial, log2 units
   long long ncol, max_tiles;
 };
 
@@ -62,7 +62,6 @@ PrefillWs carve(const msa_shape& s, void* base) {
   w.part_o = reinterpret_cast<uint16_t*>(take(2ull * s.batch * s.seq_q * s.n_q_heads *
                                               s.topk * s.head_dim));
   w.part_lse = reinterpret_cast<float*>(take(4ull * s.batch * s.seq_q * s.n_q_heads * s.topk));
-  // total bytes are returned through max_tiles' neighbour: recomputed by the caller
   return w;
 }
 
@@ -275,46 +274,81 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 
   if (warp == 0) {
     // ----------------------------------------------------------------- TMA
-    if (lane == 0 && t_begin < t_end) {
-      tma_prefetch_desc(&tm_q);
-      tma_prefetch_desc(&tm_k);
-      tma_prefetch_desc(&tm_v);
+    // The whole warp walks the tiles: lane j gathers tokens j, j+32, ... of a
+    // tile, so the entry loads and the per-token Q copies proceed in parallel.
+    // Tile descriptors are read two tiles ahead, entries one tile ahead.
+    if (t_begin < t_end) {
+      if (lane == 0) {
+        tma_prefetch_desc(&tm_q);
+        tma_prefetch_desc(&tm_k);
+        tma_prefetch_desc(&tm_v);
+      }
+      const int4 zero4 = make_int4(-1, 0, 0, 0);
+      int4 td_cur = p.w.tiles[t_begin];
+      int4 td_nx = t_begin + 1 < t_end ? p.w.tiles[t_begin + 1] : zero4;
+      uint32_t ent_cur[4];
+#pragma unroll
+      for (int x = 0; x < 4; ++x)
+        ent_cur[x] = lane + 32 * x < td_cur.z ? p.w.entries[td_cur.y + lane + 32 * x] : 0u;
       int prev_col = -1;
       long long u = -1;   // column ordinal
       for (long long ti = t_begin; ti < t_end; ++ti) {
         const long long i = ti - t_begin;
-        const int4 td = p.w.tiles[ti];
+        const int4 td = td_cur;
+        uint32_t ent[4];
+#pragma unroll
+        for (int x = 0; x < 4; ++x) ent[x] = ent_cur[x];
+        const int4 td_nn = ti + 2 < t_end ? p.w.tiles[ti + 2] : zero4;
+#pragma unroll
+        for (int x = 0; x < 4; ++x)
+          ent_cur[x] = lane + 32 * x < td_nx.z ? p.w.entries[td_nx.y + lane + 32 * x] : 0u;
+        td_cur = td_nx;
+        td_nx = td_nn;
+
         const int col = td.x;
+        const int bg = static_cast<int>(col / p.nb);
+        const int blk = static_cast<int>(col - static_cast<long long>(bg) * p.nb);
+        int ok = 1;
         if (col != prev_col) {
           prev_col = col;
           ++u;
           const int st = static_cast<int>(u & 1);
-          if (!mbar_wait(&kvempty[st], ((u >> 1) & 1) ^ 1, abort_flag, p.err)) break;
-          const int bg = static_cast<int>(col / p.nb);
-          const int blk = static_cast<int>(col - static_cast<long long>(bg) * p.nb);
-          mbar_arrive_expect_tx(&kvfull[st], 2 * L::kKV);
+          if (lane == 0) {
+            ok = mbar_wait(&kvempty[st], ((u >> 1) & 1) ^ 1, abort_flag, p.err) ? 1 : 0;
+            if (ok) {
+              mbar_arrive_expect_tx(&kvfull[st], 2 * L::kKV);
 #pragma unroll
-          for (int c = 0; c < D / 64; ++c) {
-            tma_load_3d(smem + L::kOffK + st * L::kKV + c * 16384, &tm_k, &kvfull[st], c * 64,
-                        blk * 128, bg);
-            tma_load_3d(smem + L::kOffV + st * L::kKV + c * 16384, &tm_v, &kvfull[st], c * 64,
-                        blk * 128, bg);
+              for (int c = 0; c < D / 64; ++c) {
+                tma_load_3d(smem + L::kOffK + st * L::kKV + c * 16384, &tm_k, &kvfull[st], c * 64,
+                            blk * 128, bg);
+                tma_load_3d(smem + L::kOffV + st * L::kKV + c * 16384, &tm_v, &kvfull[st], c * 64,
+                            blk * 128, bg);
+              }
+            }
           }
+          ok = __shfl_sync(0xffffffffu, ok, 0);
+          if (!ok) break;
         }
         const int qb = static_cast<int>(i & 1);
-        if (!mbar_wait(&qempty[qb], ((i >> 1) & 1) ^ 1, abort_flag, p.err)) break;
-        const int bg = static_cast<int>(col / p.nb);
-        const int b = bg / p.G, g = bg % p.G;
         const int cnt = td.z;
-        mbar_arrive_expect_tx(&qfull[qb], static_cast<uint32_t>(cnt * p.r * D * 2));
-        for (int j = 0; j < cnt; ++j) {
-          const uint32_t e = p.w.entries[td.y + j];
-          const int t = static_cast<int>(e >> 6);
-          const int row = (b * p.T + t) * p.H + g * p.r;
+        if (lane == 0) {
+          ok = mbar_wait(&qempty[qb], ((i >> 1) & 1) ^ 1, abort_flag, p.err) ? 1 : 0;
+          if (ok) mbar_arrive_expect_tx(&qfull[qb], static_cast<uint32_t>(cnt * p.r * D * 2));
+        }
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        if (!ok) break;
+        const int b = bg / p.G, g = bg % p.G;
 #pragma unroll
-          for (int c = 0; c < D / 64; ++c)
-            tma_load_2d(smem + L::kOffQ + qb * L::kQ + c * 16384 + j * p.r * 128, &tm_q,
-                        &qfull[qb], c * 64, row);
+        for (int x = 0; x < 4; ++x) {
+          const int j = lane + 32 * x;
+          if (j < cnt) {
+            const int t = static_cast<int>(ent[x] >> 6);
+            const int row = (b * p.T + t) * p.H + g * p.r;
+#pragma unroll
+            for (int c = 0; c < D / 64; ++c)
+              tma_load_2d(smem + L::kOffQ + qb * L::kQ + c * 16384 + j * p.r * 128, &tm_q,
+                          &qfull[qb], c * 64, row);
+          }
         }
       }
     }
@@ -327,12 +361,17 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       int prev_col = -1;
       long long u = -1;
       int cur_stage = 0;
-      // per-tile KV stage, recorded when S is issued (PV of the same tile reuses it)
+      // columns of the next two tiles, read ahead of use
+      int col_cur = p.w.tiles[t_begin].x;
+      int col_nx = n > 1 ? p.w.tiles[t_begin + 1].x : -1;
       int stage_of[2] = {0, 0};
       bool last_of_col[2] = {false, false};
       auto issue_s = [&](long long i) -> bool {
         const long long ti = t_begin + i;
-        const int col = p.w.tiles[ti].x;
+        const int col = col_cur;
+        const int col_next = col_nx;
+        col_cur = col_nx;
+        col_nx = i + 2 < n ? p.w.tiles[ti + 2].x : -1;
         if (col != prev_col) {
           prev_col = col;
           ++u;
@@ -341,7 +380,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         }
         const int qb = static_cast<int>(i & 1);
         stage_of[qb] = cur_stage;
-        last_of_col[qb] = (ti + 1 >= t_end) || (p.w.tiles[ti + 1].x != col);
+        last_of_col[qb] = col_next != col;
         if (!mbar_wait(&qfull[qb], (i >> 1) & 1, abort_flag, p.err)) return false;
         if (!mbar_wait(&sempty[qb], ((i >> 1) & 1) ^ 1, abort_flag, p.err)) return false;
         tc_fence_after();
@@ -350,8 +389,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 #pragma unroll
         for (int ks = 0; ks < D / 16; ++ks) {
           const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
-          tc_mma_ss(tS + qb * 128, smem_desc(qa + off, 16, 1024, 2), smem_desc(ka + off, 16, 1024, 2),
-                    kIdescS, ks > 0 ? 1u : 0u);
+          tc_mma_ss(tS + qb * 128, smem_desc(qa + off, 16, 1024, 2),
+                    smem_desc(ka + off, 16, 1024, 2), kIdescS, ks > 0 ? 1u : 0u);
         }
         tc_commit(&sfull[qb]);
         tc_commit(&qempty[qb]);
@@ -387,19 +426,29 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     const int tok = row / p.r, head = row % p.r;
     const long long n = t_end - t_begin;
     uint8_t* prow = smem + L::kOffP + row * 128;
+    // descriptors two tiles ahead, this row's entry one tile ahead
+    const int4 zero4 = make_int4(-1, 0, 0, 0);
+    int4 td_cur = n > 0 ? p.w.tiles[t_begin] : zero4;
+    int4 td_nx = n > 1 ? p.w.tiles[t_begin + 1] : zero4;
+    uint32_t ent_cur = tok < td_cur.z ? p.w.entries[td_cur.y + tok] : 0u;
     // state of the tile whose output is pending
     bool pend_valid = false;
-    long long pend_base = 0;    // index of (b, t, h, slot) for part arrays
+    long long pend_row = 0;     // row of the part arrays: ((b*T + t)*k + slot)*H + h
     float pend_inv_l = 0.f;
     bool ok = true;
     for (long long i = 0; i <= n && ok; ++i) {
       bool cur_valid = false;
-      long long cur_base = 0;
-      float cur_inv_l = 0.f, cur_lse = 0.f;
+      long long cur_row = 0;
+      float cur_inv_l = 0.f;
       uint32_t pk[64];
       if (i < n) {
         const int qb = static_cast<int>(i & 1);
-        const int4 td = p.w.tiles[t_begin + i];
+        const int4 td = td_cur;
+        const uint32_t e = ent_cur;
+        const int4 td_nn = i + 2 < n ? p.w.tiles[t_begin + i + 2] : zero4;
+        ent_cur = tok < td_nx.z ? p.w.entries[td_nx.y + tok] : 0u;
+        td_cur = td_nx;
+        td_nx = td_nn;
         const int col = td.x;
         const int bg = static_cast<int>(col / p.nb);
         const int blk = static_cast<int>(col - static_cast<long long>(bg) * p.nb);
@@ -407,11 +456,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         cur_valid = tok < td.z;
         int lim = 127;
         if (cur_valid) {
-          const uint32_t e = p.w.entries[td.y + tok];
           const int t = static_cast<int>(e >> 6), slot = static_cast<int>(e & 63u);
           const int pos = p.q_off + t;
           if ((pos >> 7) == blk) lim = pos & 127;
-          cur_base = ((static_cast<long long>(b) * p.T + t) * p.H + g * p.r + head) * p.k + slot;
+          cur_row = ((static_cast<long long>(b) * p.T + t) * p.k + slot) * p.H + g * p.r + head;
         }
         if (!(ok = mbar_wait(&sfull[qb], (i >> 1) & 1, abort_flag, p.err))) break;
         tc_fence_after();
@@ -439,8 +487,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           l += back.x + back.y;
         }
         cur_inv_l = 1.f / l;
-        cur_lse = mxs + log2f(l);
-        if (cur_valid) p.w.part_lse[cur_base] = cur_lse;
+        if (cur_valid) p.w.part_lse[cur_row] = mxs + log2f(l);
       }
       // epilogue of the previous tile (its PV also frees the P buffer)
       if (i > 0) {
@@ -454,7 +501,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           tmem_ld32(tO + ob * D + lane_off + c * 32, ov);
           tc_wait_ld();
           if (pend_valid) {
-            uint4* dst = reinterpret_cast<uint4*>(p.w.part_o + pend_base * D + c * 32);
+            uint4* dst = reinterpret_cast<uint4*>(p.w.part_o + pend_row * D + c * 32);
 #pragma unroll
             for (int x = 0; x < 4; ++x) {
               __nv_bfloat162 h0 = __floats2bfloat162_rn(ov[8 * x] * pend_inv_l, ov[8 * x + 1] * pend_inv_l);
@@ -480,7 +527,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         fence_proxy_async_smem();
         mbar_arrive(pfull);
         pend_valid = cur_valid;
-        pend_base = cur_base;
+        pend_row = cur_row;
         pend_inv_l = cur_inv_l;
       }
     }
@@ -495,62 +542,57 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 }
 
 // ------------------------------------------------------------- 4. combine
-// One warp per (sequence, token, head): merge the k normalised partials by
-// their log-sum-exp.
+// One CTA per (sequence, token): merge the k normalised partials of each of
+// the H heads by their log-sum-exp.  Partials of one token are laid out
+// [slot][head][d], so each slot is one contiguous H*d run.
 template <int D>
 __global__ void __launch_bounds__(256) combine_kernel(const int32_t* __restrict__ sel,
                                                       const PrefillWs w, uint16_t* __restrict__ o,
-                                                      float* __restrict__ lse, long long rows,
-                                                      int H, int G, int r, int k) {
-  constexpr int V = D / 32;   // bf16 elements per lane (2 or 4)
-  const long long nwarps = static_cast<long long>(gridDim.x) * (blockDim.x >> 5);
-  const int lane = threadIdx.x & 31;
-  for (long long row = static_cast<long long>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
-       row < rows; row += nwarps) {
-    const long long bt = row / H;
-    const int h = static_cast<int>(row % H);
-    const int g = h / r;
-    const int32_t* srow = sel + (bt * G + g) * k;
+                                                      float* __restrict__ lse, int H, int G,
+                                                      int r, int k) {
+  constexpr int CH = D / 8;                  // 16-byte chunks per head row
+  extern __shared__ float sm_lse[];          // [k][H] log2 units, -inf for unused slots
+  const long long bt = blockIdx.x;           // b*T + t
+  const float* lsrc = w.part_lse + bt * k * H;
+  const int32_t* srow = sel + bt * G * k;
+  for (int x = threadIdx.x; x < k * H; x += blockDim.x) {
+    const int s = x / H, h = x % H;
+    sm_lse[x] = srow[(h / r) * k + s] >= 0 ? lsrc[x] : -INFINITY;
+  }
+  __syncthreads();
+  const uint16_t* osrc = w.part_o + bt * k * H * D;
+  for (int item = threadIdx.x; item < H * CH; item += blockDim.x) {
+    const int h = item / CH, c = item % CH;
     float M = -INFINITY;
-    for (int s = 0; s < k; ++s)
-      if (srow[s] >= 0) M = fmaxf(M, w.part_lse[row * k + s]);
-    float acc[V];
+    for (int s = 0; s < k; ++s) M = fmaxf(M, sm_lse[s * H + h]);
+    float acc[8];
 #pragma unroll
-    for (int e = 0; e < V; ++e) acc[e] = 0.f;
+    for (int e = 0; e < 8; ++e) acc[e] = 0.f;
     float den = 0.f;
+#pragma unroll 4
     for (int s = 0; s < k; ++s) {
-      if (srow[s] < 0) continue;
-      const float ws = exp2f(w.part_lse[row * k + s] - M);
+      const float ls = sm_lse[s * H + h];
+      if (ls == -INFINITY) continue;
+      const float ws = exp2f(ls - M);
       den += ws;
-      const uint16_t* src = w.part_o + (row * k + s) * D + lane * V;
-      uint32_t u[V / 2];
-      if constexpr (V == 4) {
-        const uint2 x = *reinterpret_cast<const uint2*>(src);
-        u[0] = x.x;
-        u[1] = x.y;
-      } else {
-        u[0] = *reinterpret_cast<const uint32_t*>(src);
-      }
+      const uint4 u = __ldcs(reinterpret_cast<const uint4*>(osrc + (static_cast<long long>(s) * H + h) * D) + c);
+      const uint32_t wds[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
-      for (int e = 0; e < V / 2; ++e) {
-        const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u[e]));
+      for (int e = 0; e < 4; ++e) {
+        const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&wds[e]));
         acc[2 * e] += ws * f.x;
         acc[2 * e + 1] += ws * f.y;
       }
     }
     const float inv = 1.f / den;
-    uint32_t out[V / 2];
+    uint32_t out[4];
 #pragma unroll
-    for (int e = 0; e < V / 2; ++e) {
+    for (int e = 0; e < 4; ++e) {
       __nv_bfloat162 x = __floats2bfloat162_rn(acc[2 * e] * inv, acc[2 * e + 1] * inv);
       out[e] = *reinterpret_cast<uint32_t*>(&x);
     }
-    uint16_t* dst = o + row * D + lane * V;
-    if constexpr (V == 4)
-      *reinterpret_cast<uint2*>(dst) = make_uint2(out[0], out[1]);
-    else
-      *reinterpret_cast<uint32_t*>(dst) = out[0];
-    if (lse && lane == 0) lse[row] = (M + log2f(den)) / kLog2e;
+    *(reinterpret_cast<uint4*>(o + (bt * H + h) * D) + c) = make_uint4(out[0], out[1], out[2], out[3]);
+    if (lse && c == 0) lse[bt * H + h] = (M + log2f(den)) / kLog2e;
   }
 }
 
@@ -580,7 +622,10 @@ cudaError_t launch_attn(const msa_shape& s, const uint16_t* q, const uint16_t* k
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  kvouter_attn_kernel<D><<<ctx->num_sms, kAttnThreads, smem, st>>>(tq, tk, tv, p);
+  {
+    ProfScope ps_("kvouter_attn", st);
+    kvouter_attn_kernel<D><<<ctx->num_sms, kAttnThreads, smem, st>>>(tq, tk, tv, p);
+  }
   return cudaGetLastError();
 }
 
@@ -607,10 +652,22 @@ cudaError_t launch_sparse_prefill(const msa_shape& s, const uint16_t* q, const u
   e = cudaFuncSetAttribute(sel_invert_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(hsmem));
   if (e != cudaSuccess) return e;
-  sel_invert_kernel<<<hgrid, 256, hsmem, st>>>(sel, w, s.seq_q, s.n_kv_heads, s.topk, nb, 0);
-  scan_columns_kernel<<<1, 1024, 0, st>>>(w, tpt);
-  sel_invert_kernel<<<hgrid, 256, hsmem, st>>>(sel, w, s.seq_q, s.n_kv_heads, s.topk, nb, 1);
-  make_tiles_kernel<<<static_cast<unsigned>(ceil_div(w.ncol, 256)), 256, 0, st>>>(w, tpt);
+  {
+    ProfScope ps_("sel_count", st);
+    sel_invert_kernel<<<hgrid, 256, hsmem, st>>>(sel, w, s.seq_q, s.n_kv_heads, s.topk, nb, 0);
+  }
+  {
+    ProfScope ps_("scan_columns", st);
+    scan_columns_kernel<<<1, 1024, 0, st>>>(w, tpt);
+  }
+  {
+    ProfScope ps_("sel_scatter", st);
+    sel_invert_kernel<<<hgrid, 256, hsmem, st>>>(sel, w, s.seq_q, s.n_kv_heads, s.topk, nb, 1);
+  }
+  {
+    ProfScope ps_("make_tiles", st);
+    make_tiles_kernel<<<static_cast<unsigned>(ceil_div(w.ncol, 256)), 256, 0, st>>>(w, tpt);
+  }
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
 
   AttnParams p{};
@@ -629,17 +686,17 @@ cudaError_t launch_sparse_prefill(const msa_shape& s, const uint16_t* q, const u
   e = s.head_dim == 128 ? launch_attn<128>(s, q, k, v, p, ctx, st)
                         : launch_attn<64>(s, q, k, v, p, ctx, st);
   if (e != cudaSuccess) return e;
-  const long long rows = static_cast<long long>(s.batch) * s.seq_q * s.n_q_heads;
-  long long blocks = ceil_div(rows, 8);
-  if (blocks > static_cast<long long>(ctx->num_sms) * 64) blocks = ctx->num_sms * 64ll;
-  if (s.head_dim == 128)
-    combine_kernel<128><<<static_cast<unsigned>(blocks), 256, 0, st>>>(sel, w, o, lse, rows,
-                                                                       s.n_q_heads, s.n_kv_heads,
-                                                                       r, s.topk);
-  else
-    combine_kernel<64><<<static_cast<unsigned>(blocks), 256, 0, st>>>(sel, w, o, lse, rows,
-                                                                      s.n_q_heads, s.n_kv_heads,
-                                                                      r, s.topk);
+  const unsigned ntok = static_cast<unsigned>(static_cast<long long>(s.batch) * s.seq_q);
+  const size_t csmem = sizeof(float) * s.topk * s.n_q_heads;
+  {
+    ProfScope ps_("combine", st);
+    if (s.head_dim == 128)
+      combine_kernel<128><<<ntok, 256, csmem, st>>>(sel, w, o, lse, s.n_q_heads, s.n_kv_heads, r,
+                                                    s.topk);
+    else
+      combine_kernel<64><<<ntok, 256, csmem, st>>>(sel, w, o, lse, s.n_q_heads, s.n_kv_heads, r,
+                                                   s.topk);
+  }
   return cudaGetLastError();
 }
 

@@ -9,7 +9,8 @@
 // scores is filtered against a threshold that provably keeps the (k-1) best
 // (the (k-1)-th largest of the 32 per-lane maxima, or the running (k-1)-th
 // best), and the survivors are merged into the running list with a warp
-// bitonic sort.  No exponentials, no full sort of the row.
+// bitonic sort.  No exponentials, no full sort of the row.  Thresholds are
+// compared on the 32-bit score keys; only the survivors get 64-bit keys.
 #include <math.h>
 
 #include "internal.h"
@@ -19,7 +20,9 @@ namespace msa {
 namespace {
 
 constexpr int kWarps = 8;
-constexpr int kChunk = 1024;   // scores held per warp at a time (32 per lane)
+constexpr int kPer = 16;             // scores per lane per chunk
+constexpr int kChunk = 32 * kPer;    // scores per warp per chunk
+constexpr int kScratch = 128;        // per-warp merge buffer (64-bit keys)
 
 MSA_DEV uint64_t shfl_xor64(uint64_t x, int m) {
   uint32_t lo = static_cast<uint32_t>(x), hi = static_cast<uint32_t>(x >> 32);
@@ -35,15 +38,16 @@ MSA_DEV uint64_t shfl64(uint64_t x, int src) {
   return (static_cast<uint64_t>(hi) << 32) | lo;
 }
 
-MSA_DEV uint64_t make_key(float score, int idx) {
-  return (static_cast<uint64_t>(float_order_key(score)) << 32) |
+// Composite key: larger = better; ties in score resolved by the lower index.
+MSA_DEV uint64_t make_key(uint32_t ord_score, int idx) {
+  return (static_cast<uint64_t>(ord_score) << 32) |
          static_cast<uint64_t>(0xFFFFFFFFu - static_cast<uint32_t>(idx));
 }
 MSA_DEV int key_index(uint64_t key) {
   return static_cast<int>(0xFFFFFFFFu - static_cast<uint32_t>(key));
 }
 
-// Descending bitonic sort of 32*S keys; element e = s*32 + lane lives in x[s].
+// Descending bitonic sort of 32*S 64-bit keys; element e = s*32 + lane in x[s].
 template <int S>
 MSA_DEV void warp_sort_desc(uint64_t (&x)[S]) {
   const int lane = threadIdx.x & 31;
@@ -68,14 +72,42 @@ MSA_DEV void warp_sort_desc(uint64_t (&x)[S]) {
         for (int s = 0; s < S; ++s) {
           const uint64_t y = shfl_xor64(x[s], j);
           const bool desc = ((s * 32 + lane) & k) == 0;
-          const bool lower = (lane & j) == 0;
-          const bool take_max = (desc == lower);
+          const bool take_max = desc == ((lane & j) == 0);
           const uint64_t mx = x[s] > y ? x[s] : y, mn = x[s] > y ? y : x[s];
           x[s] = take_max ? mx : mn;
         }
       }
     }
   }
+}
+
+// Descending bitonic sort of 32 32-bit values, one per lane.
+MSA_DEV uint32_t warp_sort_desc32(uint32_t x) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int k = 2; k <= 32; k <<= 1) {
+#pragma unroll
+    for (int j = k >> 1; j > 0; j >>= 1) {
+      const uint32_t y = __shfl_xor_sync(0xffffffffu, x, j);
+      const bool take_max = ((lane & k) == 0) == ((lane & j) == 0);
+      x = take_max ? max(x, y) : min(x, y);
+    }
+  }
+  return x;
+}
+
+// Sorts the first m (<= 32*S) keys of buf descending into best (elements
+// lane and 32+lane); slots past m count as empty (key 0).
+template <int S>
+__device__ __noinline__ void sort_buffer(const uint64_t* buf, int m, uint64_t& best0,
+                                         uint64_t& best1) {
+  const int lane = threadIdx.x & 31;
+  uint64_t x[S];
+#pragma unroll
+  for (int s = 0; s < S; ++s) x[s] = s * 32 + lane < m ? buf[s * 32 + lane] : 0ull;
+  warp_sort_desc<S>(x);
+  best0 = x[0];
+  best1 = S > 1 ? x[1 % S] : 0ull;
 }
 
 // best0/best1: running list (elements lane, 32+lane, descending); nk: one new
@@ -87,11 +119,12 @@ __device__ __noinline__ void merge128(uint64_t& best0, uint64_t& best1, uint64_t
   best1 = xk[1];
 }
 
-__global__ void __launch_bounds__(kWarps * 32)
+__global__ void __launch_bounds__(kWarps * 32, 3)
     block_topk_kernel(const float* __restrict__ pooled, int32_t* __restrict__ sel,
                       long long rows, int T, int G, int q_off, int nb, int k) {
-  __shared__ uint64_t scratch[kWarps][32];
+  __shared__ uint64_t scratch[kWarps][kScratch];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  uint64_t* buf = scratch[warp];
   const long long nwarps = static_cast<long long>(gridDim.x) * kWarps;
   const bool vec = (nb & 3) == 0;
   for (long long r = static_cast<long long>(blockIdx.x) * kWarps + warp; r < rows; r += nwarps) {
@@ -110,60 +143,47 @@ __global__ void __launch_bounds__(kWarps * 32)
     }
     const float* src = pooled + r * nb;
     uint64_t best[2] = {0ull, 0ull};          // sorted descending: element lane / lane+32
-    int have = 0;                             // valid entries in best
+    int have = 0;                             // valid entries in best (<= kk after a chunk)
     for (int base = 0; base < n; base += kChunk) {
-      float v[32];
-      if (vec) {
+      // this lane's scores: block base + x*128 + lane*4 + e, as order-preserving keys
+      uint32_t uk[kPer];
 #pragma unroll
-        for (int x = 0; x < 8; ++x) {
-          const int i0 = base + x * 128 + lane * 4;
-          if (i0 + 3 < n) {
-            const float4 f = __ldg(reinterpret_cast<const float4*>(src + i0));
-            v[4 * x] = f.x; v[4 * x + 1] = f.y; v[4 * x + 2] = f.z; v[4 * x + 3] = f.w;
-          } else {
-#pragma unroll
-            for (int e = 0; e < 4; ++e) v[4 * x + e] = i0 + e < n ? __ldg(src + i0 + e) : 0.f;
-          }
+      for (int x = 0; x < kPer / 4; ++x) {
+        const int i0 = base + x * 128 + lane * 4;
+        float4 f;
+        if (vec && i0 + 3 < n) {
+          f = __ldg(reinterpret_cast<const float4*>(src + i0));
+        } else {
+          f.x = i0 < n ? __ldg(src + i0) : 0.f;
+          f.y = i0 + 1 < n ? __ldg(src + i0 + 1) : 0.f;
+          f.z = i0 + 2 < n ? __ldg(src + i0 + 2) : 0.f;
+          f.w = i0 + 3 < n ? __ldg(src + i0 + 3) : 0.f;
         }
-      } else {
-#pragma unroll
-        for (int x = 0; x < 8; ++x)
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int i = base + x * 128 + lane * 4 + e;
-            v[4 * x + e] = i < n ? __ldg(src + i) : 0.f;
-          }
+        uk[4 * x] = i0 < n ? float_order_key(f.x) : 0u;
+        uk[4 * x + 1] = i0 + 1 < n ? float_order_key(f.y) : 0u;
+        uk[4 * x + 2] = i0 + 2 < n ? float_order_key(f.z) : 0u;
+        uk[4 * x + 3] = i0 + 3 < n ? float_order_key(f.w) : 0u;
       }
-      // element (x, e) of this lane has block index base + x*128 + lane*4 + e
-      uint64_t lmax = 0ull;
-#pragma unroll
-      for (int x = 0; x < 8; ++x)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int i = base + x * 128 + lane * 4 + e;
-          const uint64_t key = i < n ? make_key(v[4 * x + e], i) : 0ull;
-          lmax = key > lmax ? key : lmax;
-        }
-      uint64_t tau = 0ull;
-      if (kk <= 32) {
-        uint64_t m1[1] = {lmax};
-        warp_sort_desc<1>(m1);
-        tau = shfl64(m1[0], kk - 1);
-      }
+      // score threshold that keeps every member of the new top-kk
+      uint32_t tau;
       if (have >= kk) {
-        const uint64_t run = shfl64(best[(kk - 1) >> 5], (kk - 1) & 31);
-        tau = run > tau ? run : tau;
+        // every later block has a larger index than the list's members, so a
+        // score equal to the current kk-th best can no longer enter: strict >
+        const uint32_t kth = static_cast<uint32_t>(shfl64(best[(kk - 1) >> 5], (kk - 1) & 31) >> 32);
+        if (kth == 0xFFFFFFFFu) continue;
+        tau = kth + 1u;
+      } else if (kk <= 32) {
+        uint32_t lmax = 0u;
+#pragma unroll
+        for (int x = 0; x < kPer; ++x) lmax = max(lmax, uk[x]);
+        tau = __shfl_sync(0xffffffffu, warp_sort_desc32(lmax), kk - 1);
+      } else {
+        tau = 0u;
       }
-      // count survivors (key >= tau, key > 0)
+      tau = max(tau, 1u);
       int cnt = 0;
 #pragma unroll
-      for (int x = 0; x < 8; ++x)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int i = base + x * 128 + lane * 4 + e;
-          const uint64_t key = i < n ? make_key(v[4 * x + e], i) : 0ull;
-          cnt += (key != 0ull && key >= tau) ? 1 : 0;
-        }
+      for (int x = 0; x < kPer; ++x) cnt += uk[x] >= tau ? 1 : 0;
       int incl = cnt;
 #pragma unroll
       for (int off = 1; off < 32; off <<= 1) {
@@ -172,65 +192,61 @@ __global__ void __launch_bounds__(kWarps * 32)
       }
       const int total = __shfl_sync(0xffffffffu, incl, 31);
       if (total == 0) continue;
-      const int keep_have = have < kk ? have : kk;
-      if (kk <= 32 && keep_have + total <= 32) {
-        // fast path: one 32-wide sort of (running list + survivors)
-        int slot = incl - cnt;
+      const int keep = have < kk ? have : kk;
+      const int m = keep + total;
+      if (m <= kScratch) {
+        // running list and survivors into the warp buffer, one sort of <= 128
+        if (lane < keep) buf[lane] = best[0];
+        if (lane + 32 < keep) buf[32 + lane] = best[1];
+        int slot = keep + incl - cnt;
 #pragma unroll
-        for (int x = 0; x < 8; ++x)
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int i = base + x * 128 + lane * 4 + e;
-            const uint64_t key = i < n ? make_key(v[4 * x + e], i) : 0ull;
-            if (key != 0ull && key >= tau) scratch[warp][slot++] = key;
-          }
-        __syncwarp();
-        uint64_t xk[1];
-        xk[0] = lane < keep_have ? best[0]
-                                 : (lane - keep_have < total ? scratch[warp][lane - keep_have] : 0ull);
-        __syncwarp();
-        warp_sort_desc<1>(xk);
-        best[0] = xk[0];
-        best[1] = 0ull;
-        have = keep_have + total;
-      } else {
-        // general path: merge survivors one register slot at a time into the
-        // list with a 128-wide sort (list in elements 0..63, new in 64..95)
-#pragma unroll
-        for (int x = 0; x < 8; ++x) {
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int i = base + x * 128 + lane * 4 + e;
-            const uint64_t key = i < n ? make_key(v[4 * x + e], i) : 0ull;
-            const bool take = key != 0ull && key >= tau;
-            const unsigned bal = __ballot_sync(0xffffffffu, take);
-            if (bal != 0u) {
-              merge128(best[0], best[1], take ? key : 0ull);
-              have += __popc(bal);
-            }
+        for (int x = 0; x < kPer; ++x) {
+          if (uk[x] >= tau) {
+            const int i = base + (x >> 2) * 128 + lane * 4 + (x & 3);
+            buf[slot++] = make_key(uk[x], i);
           }
         }
-        if (kk <= 32) best[1] = 0ull;
+        __syncwarp();
+        if (m <= 32) {
+          uint64_t x1[1];
+          x1[0] = lane < m ? buf[lane] : 0ull;
+          warp_sort_desc<1>(x1);
+          best[0] = x1[0];
+          best[1] = 0ull;
+        } else if (m <= 64) {
+          sort_buffer<2>(buf, m, best[0], best[1]);
+        } else {
+          sort_buffer<4>(buf, m, best[0], best[1]);
+        }
+        __syncwarp();
+      } else {
+        // rare: merge the survivors one register slot at a time
+#pragma unroll
+        for (int x = 0; x < kPer; ++x) {
+          const bool take = uk[x] >= tau;
+          const unsigned bal = __ballot_sync(0xffffffffu, take);
+          if (bal != 0u) {
+            const int i = base + (x >> 2) * 128 + lane * 4 + (x & 3);
+            merge128(best[0], best[1], take ? make_key(uk[x], i) : 0ull);
+          }
+        }
       }
-      if (have > kk) have = kk;
-      // keep only the kk best
+      have = min(m, kk);
       if (lane >= kk) best[0] = 0ull;
       if (lane + 32 >= kk) best[1] = 0ull;
     }
     // output: the kk chosen blocks plus bt, ascending, then -1 padding
     if (kk < 32) {
-      uint32_t idx = lane < kk ? static_cast<uint32_t>(key_index(best[0]))
-                               : (lane == kk ? static_cast<uint32_t>(bt) : 0xFFFFFFFFu);
-      uint64_t xk[1] = {static_cast<uint64_t>(~idx)};   // descending ~idx = ascending idx
-      warp_sort_desc<1>(xk);
-      const uint32_t sorted = ~static_cast<uint32_t>(xk[0]);
+      const uint32_t idx = lane < kk ? static_cast<uint32_t>(key_index(best[0]))
+                                     : (lane == kk ? static_cast<uint32_t>(bt) : 0xFFFFFFFFu);
+      const uint32_t sorted = ~warp_sort_desc32(~idx);   // ascending
       if (lane < k) out[lane] = lane <= kk ? static_cast<int32_t>(sorted) : -1;
       for (int i = lane + 32; i < k; i += 32) out[i] = -1;
     } else {
-      uint32_t i0 = static_cast<uint32_t>(key_index(best[0]));
+      const uint32_t i0 = static_cast<uint32_t>(key_index(best[0]));
       const int e1 = lane + 32;
-      uint32_t i1 = e1 < kk ? static_cast<uint32_t>(key_index(best[1]))
-                            : (e1 == kk ? static_cast<uint32_t>(bt) : 0xFFFFFFFFu);
+      const uint32_t i1 = e1 < kk ? static_cast<uint32_t>(key_index(best[1]))
+                                  : (e1 == kk ? static_cast<uint32_t>(bt) : 0xFFFFFFFFu);
       uint64_t xk[2] = {static_cast<uint64_t>(~i0), static_cast<uint64_t>(~i1)};
       warp_sort_desc<2>(xk);
       const uint32_t s0 = ~static_cast<uint32_t>(xk[0]), s1 = ~static_cast<uint32_t>(xk[1]);
@@ -251,8 +267,11 @@ cudaError_t launch_block_topk(const msa_shape& s, const float* pooled, int32_t* 
   long long blocks = (rows + kWarps - 1) / kWarps;
   const long long cap = static_cast<long long>(ctx->num_sms) * 32;
   if (blocks > cap) blocks = cap;
-  block_topk_kernel<<<static_cast<unsigned>(blocks), kWarps * 32, 0, st>>>(
+  {
+    ProfScope ps_("block_topk", st);
+    block_topk_kernel<<<static_cast<unsigned>(blocks), kWarps * 32, 0, st>>>(
       pooled, sel, rows, s.seq_q, s.n_kv_heads, s.q_offset, nb, s.topk);
+  }
   return cudaGetLastError();
 }
 

@@ -65,6 +65,10 @@ _SIGS = {
     "msa_dense_attn_decode": ([ctypes.POINTER(Shape), _vp, _vp, _vp, _vp, _vp, _vp,
                                ctypes.c_size_t, _vp], ctypes.c_int),
     "msa_device_status": ([ctypes.POINTER(ctypes.c_uint32)], ctypes.c_int),
+    "msa_profile_enable": ([ctypes.c_int], ctypes.c_int),
+    "msa_profile_read": ([ctypes.c_int, ctypes.POINTER(ctypes.c_char_p),
+                          ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_longlong)],
+                         ctypes.c_int),
 }
 
 _lib = None
@@ -200,6 +204,27 @@ def dense_attn_decode(shape: Shape, q, k, v, o=None, lse=None, ws=None, want_lse
                                        _ptr(lse), _ptr(ws), ws.numel(), _stream(stream)),
            "msa_dense_attn_decode")
     return o, lse
+
+
+def profile_enable(on: bool = True):
+    """Start (clearing the table) or stop per-kernel CUDA-event timing."""
+    _check(lib().msa_profile_enable(1 if on else 0), "msa_profile_enable")
+
+
+def profile_read() -> dict:
+    """{kernel name: (total ms, launches)} of the recorded launches (waits for them)."""
+    out = {}
+    i = 0
+    while True:
+        name = ctypes.c_char_p()
+        ms = ctypes.c_double()
+        n = ctypes.c_longlong()
+        st = lib().msa_profile_read(i, ctypes.byref(name), ctypes.byref(ms), ctypes.byref(n))
+        if st == 1:
+            return out
+        _check(st, "msa_profile_read")
+        out[name.value.decode()] = (ms.value, n.value)
+        i += 1
 
 
 def device_status() -> int:

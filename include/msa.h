@@ -170,6 +170,18 @@ msa_status msa_dense_attn_decode(const msa_shape* shape, const uint16_t* q,
  * NULL) receives the raw word. */
 msa_status msa_device_status(uint32_t* flags);
 
+/* Per-kernel timing with CUDA events (diagnostics; no counterpart on the
+ * pages).  msa_profile_enable(1) clears the table and brackets every later
+ * kernel launch of the library with a pair of events recorded on the launch
+ * stream; msa_profile_enable(0) stops recording.  msa_profile_read waits for
+ * the recorded events and returns entry ``index`` of the table: the kernel's
+ * name (static string), its summed device time in milliseconds and its launch
+ * count.  Returns MSA_ERR_INVALID_SHAPE when ``index`` is past the last
+ * entry, MSA_ERR_CUDA if an event query fails. */
+msa_status msa_profile_enable(int on);
+msa_status msa_profile_read(int index, const char** name, double* total_ms,
+                            long long* launches);
+
 #ifdef __cplusplus
 }
 #endif
