@@ -11,9 +11,9 @@
 //  3. persistent tcgen05 kernel: each selected K/V block is TMA-loaded once per
 //     CTA that works on it and reused by every tile of its column; for a tile,
 //     S = Q K^T (TMEM), softmax over the block (causal mask on the local
-//     block), P (bf16, smem) , O_part = P V (TMEM) -> normalised bf16 partial
-//     and its log-sum-exp per (token, head, slot);
-//  4. combine the k partials of every (token, head) by their log-sum-exp.
+//     block), P (bf16, written back into TMEM), O_part = P V (TMEM) -> bf16
+//     partial plus its (max, sum) per (token, slot, head);
+//  4. combine the k partials of every (token, head).
 #include <math.h>
 
 #include "internal.h"
@@ -23,7 +23,7 @@ namespace msa {
 namespace {
 
 constexpr float kLog2e = 1.4426950408889634f;
-constexpr int kAttnThreads = 192;   // warp 0: TMA, warp 1: MMA, warps 2..5: softmax/epilogue
+constexpr int kAttnThreads = 512;   // 4 warpgroups: TMA+MMA, 2 softmax, epilogue
 constexpr int kHistTokens = 1024;   // tokens per CTA of the inversion passes
 
 struct PrefillWs {
@@ -33,8 +33,9 @@ struct PrefillWs {
   uint32_t* tile_off;    // [ncol + 1]
   uint32_t* entries;     // [B*T*G*k]   (t << 6) | slot
   int4* tiles;           // [max_tiles] (column, entry start, count, 0)
-  uint16_t* part_o;      // [B, T, k, H, d] bf16, normalised partial outputs
-  float* part_lse;       // [B, T, k, H]    log-sum-exp of each partial, log2 units
+  uint32_t* tile_ent;    // [max_tiles * tpt] entries of each tile, 0xFFFFFFFF past its count
+  uint16_t* part_o;      // [B, T, k, H, d] bf16 partial outputs, normalised by their own l
+  float* part_ml;        // [B, T, k, H, 2] (running max m, sum l) of each partial, log2 units
   long long ncol, max_tiles;
 };
 
@@ -59,9 +60,10 @@ PrefillWs carve(const msa_shape& s, void* base) {
   w.tile_off = reinterpret_cast<uint32_t*>(take(4 * (w.ncol + 1)));
   w.entries = reinterpret_cast<uint32_t*>(take(4 * nent));
   w.tiles = reinterpret_cast<int4*>(take(16 * w.max_tiles));
+  w.tile_ent = reinterpret_cast<uint32_t*>(take(4ull * w.max_tiles * tpt));
   w.part_o = reinterpret_cast<uint16_t*>(take(2ull * s.batch * s.seq_q * s.n_q_heads *
                                               s.topk * s.head_dim));
-  w.part_lse = reinterpret_cast<float*>(take(4ull * s.batch * s.seq_q * s.n_q_heads * s.topk));
+  w.part_ml = reinterpret_cast<float*>(take(8ull * s.batch * s.seq_q * s.n_q_heads * s.topk));
   return w;
 }
 
@@ -77,8 +79,9 @@ size_t carve_bytes(const msa_shape& s) {
   b += align_up(4 * (ncol + 1), 256) * 2;
   b += align_up(4 * nent, 256);
   b += align_up(16 * max_tiles, 256);
+  b += align_up(4ull * max_tiles * tpt, 256);
   b += align_up(2ull * s.batch * s.seq_q * s.n_q_heads * s.topk * s.head_dim, 256);
-  b += align_up(4ull * s.batch * s.seq_q * s.n_q_heads * s.topk, 256);
+  b += align_up(8ull * s.batch * s.seq_q * s.n_q_heads * s.topk, 256);
   return b;
 }
 
@@ -183,14 +186,24 @@ __global__ void __launch_bounds__(1024) scan_columns_kernel(PrefillWs w, int tpt
   }
 }
 
+// One thread per tile: find its column (upper bound in the tile offsets),
+// write the descriptor and the tile's entries padded to tpt.
 __global__ void make_tiles_kernel(PrefillWs w, int tpt) {
-  for (long long c = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; c < w.ncol;
-       c += static_cast<long long>(gridDim.x) * blockDim.x) {
-    const uint32_t n = w.col_count[c];
-    const uint32_t t0 = w.tile_off[c], e0 = w.col_off[c];
-    for (uint32_t i = 0; i * tpt < n; ++i)
-      w.tiles[t0 + i] = make_int4(static_cast<int>(c), static_cast<int>(e0 + i * tpt),
-                                  static_cast<int>(min(static_cast<uint32_t>(tpt), n - i * tpt)), 0);
+  const long long ntiles = static_cast<long long>(w.tile_off[w.ncol]);
+  for (long long ti = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; ti < ntiles;
+       ti += static_cast<long long>(gridDim.x) * blockDim.x) {
+    long long lo = 0, hi = w.ncol;   // first column whose tile offset exceeds ti
+    while (lo < hi) {
+      const long long mid = (lo + hi) >> 1;
+      if (static_cast<long long>(w.tile_off[mid]) > ti) hi = mid; else lo = mid + 1;
+    }
+    const long long c = lo - 1;
+    const uint32_t i = static_cast<uint32_t>(ti - w.tile_off[c]);
+    const uint32_t start = w.col_off[c] + i * tpt;
+    const uint32_t cnt = min(static_cast<uint32_t>(tpt), w.col_count[c] - i * tpt);
+    w.tiles[ti] = make_int4(static_cast<int>(c), static_cast<int>(start), static_cast<int>(cnt), 0);
+    for (int j = 0; j < tpt; ++j)
+      w.tile_ent[ti * tpt + j] = j < static_cast<int>(cnt) ? w.entries[start + j] : 0xFFFFFFFFu;
   }
 }
 
@@ -202,66 +215,103 @@ struct AttnParams {
   float scale_log2;
 };
 
+constexpr int kNQ = 2;        // query tile buffers
+constexpr int kMBMax = 16;    // most tiles per metadata batch (two batches in flight)
+constexpr int kTentWords = 256; // entry words in the metadata ring (both batches)
+
 template <int D>
 struct AttnSmem {
   static constexpr uint32_t kKV = 128u * D * 2u;     // one K (or V) block tile
   static constexpr uint32_t kQ = 128u * D * 2u;      // 128 query rows
-  static constexpr uint32_t kP = 128u * 128u * 2u;   // P tile (128 rows x 128 keys)
   static constexpr uint32_t kOffK = 0;
   static constexpr uint32_t kOffV = 2 * kKV;
   static constexpr uint32_t kOffQ = 4 * kKV;
-  static constexpr uint32_t kOffP = 4 * kKV + 2 * kQ;
-  static constexpr uint32_t kOffBar = kOffP + kP;
+  static constexpr uint32_t kOffStage = kOffQ + kNQ * kQ;   // epilogue staging (128 rows x D)
+  static constexpr uint32_t kOffLinv = kOffStage + kQ;      // float [2][128]
+  static constexpr uint32_t kOffMeta = kOffLinv + 1024;     // int [kNQ][4]
+  static constexpr uint32_t kOffTcol = kOffMeta + 64;       // int [2*kMBMax] column of each tile
+  static constexpr uint32_t kOffTlast = kOffTcol + 128;     // int [2*kMBMax] last tile of its column
+  static constexpr uint32_t kOffTent = kOffTlast + 128;     // uint [kTentWords] entries (tpt per tile)
+  static constexpr uint32_t kOffBar = kOffTent + kTentWords * 4;
   static constexpr uint32_t kBytes = kOffBar + 256;
 };
 
+// Roles by warpgroup: WG0 = warp 0 TMA producer + warp 1 MMA issuer (warps 2-3
+// idle), WG1 and WG2 = softmax of alternate tiles, WG3 = epilogue.  Register
+// budget per thread is moved from WG0/WG3 to the softmax warpgroups so that a
+// softmax thread holds its whole 128-score row.
+// TMEM: S/P buffers at columns [0,128) and [128,256) (P is written over the
+// first 64 columns of its tile's S as packed bf16 and consumed from there by
+// the PV MMA), O buffers at [256, 256+D) and [256+D, 256+2D).
 template <int D>
 __global__ void __launch_bounds__(kAttnThreads, 1)
     kvouter_attn_kernel(const __grid_constant__ CUtensorMap tm_q,
                         const __grid_constant__ CUtensorMap tm_k,
-                        const __grid_constant__ CUtensorMap tm_v, const AttnParams p) {
+                        const __grid_constant__ CUtensorMap tm_v,
+                        const __grid_constant__ CUtensorMap tm_o, const AttnParams p) {
   using L = AttnSmem<D>;
   constexpr uint32_t kIdescS = idesc_bf16(128, 128, 0, 0);   // Q (K-major) x K (K-major)
-  constexpr uint32_t kIdescO = idesc_bf16(128, D, 0, 1);     // P (K-major) x V (MN-major)
+  constexpr uint32_t kIdescO = idesc_bf16(128, D, 0, 1);     // P (TMEM) x V (MN-major)
   constexpr uint32_t kTmemCols = 512;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  // the swizzled operand tiles need 1024-byte alignment; the launch reserves no slack
+  if ((smem_u32(smem_raw) & 1023u) != 0) {
+    if (threadIdx.x == 0) atomicOr(p.err, kErrTimeout);
+    return;
+  }
+  uint8_t* smem = smem_raw;
+  const int kmb = min(kMBMax, (kTentWords / 2) / p.tpt);   // tiles per metadata batch
+  float* linv = reinterpret_cast<float*>(smem + L::kOffLinv);
+  int* meta = reinterpret_cast<int*>(smem + L::kOffMeta);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kOffBar);
-  uint64_t* kvfull = bars;        // [2]
-  uint64_t* kvempty = bars + 2;   // [2]
-  uint64_t* qfull = bars + 4;     // [2]
-  uint64_t* qempty = bars + 6;    // [2]
-  uint64_t* sfull = bars + 8;     // [2]
-  uint64_t* sempty = bars + 10;   // [2]
-  uint64_t* pfull = bars + 12;    // [1]
-  uint64_t* pvdone = bars + 13;   // [1]
-  uint64_t* ofree = bars + 14;    // [2]
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 16);
+  uint64_t* kvfull = bars;              // [2]
+  uint64_t* kvempty = bars + 2;         // [2]
+  uint64_t* qfull = bars + 4;           // [kNQ]
+  uint64_t* qempty = bars + 4 + kNQ;    // [kNQ]
+  uint64_t* sfull = bars + 4 + 2 * kNQ; // [2]
+  uint64_t* pfull = sfull + 2;          // [2]
+  uint64_t* ofull = sfull + 4;          // [2]
+  uint64_t* ofree = sfull + 6;          // [2]
+  uint64_t* lfull = sfull + 8;          // [2]
+  uint64_t* lempty = sfull + 10;        // [2]
+  uint64_t* mfull = sfull + 12;         // [2] metadata batch ready
+  uint64_t* mempty = sfull + 14;        // [2] metadata batch consumed
+  int* tcol = reinterpret_cast<int*>(smem + L::kOffTcol);
+  int* tlast = reinterpret_cast<int*>(smem + L::kOffTlast);
+  uint32_t* tent = reinterpret_cast<uint32_t*>(smem + L::kOffTent);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sfull + 16);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int wgid = warp >> 2;
   const long long ntiles = static_cast<long long>(p.w.tile_off[p.w.ncol]);
   const long long t_begin = ntiles * blockIdx.x / gridDim.x;
   const long long t_end = ntiles * (blockIdx.x + 1) / gridDim.x;
+  const long long n = t_end - t_begin;
+  const int tpt = p.tpt;
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < 2; ++i) {
       mbar_init(&kvfull[i], 1);
       mbar_init(&kvempty[i], 1);
+      mbar_init(&sfull[i], 1);
+      mbar_init(&pfull[i], 128);
+      mbar_init(&ofull[i], 1);
+      mbar_init(&ofree[i], 128);
+      mbar_init(&lfull[i], 128);
+      mbar_init(&lempty[i], 128);
+      mbar_init(&mfull[i], 32);
+      mbar_init(&mempty[i], 1);
+    }
+    for (int i = 0; i < kNQ; ++i) {
       mbar_init(&qfull[i], 1);
       mbar_init(&qempty[i], 1);
-      mbar_init(&sfull[i], 1);
-      mbar_init(&sempty[i], 128);
-      mbar_init(&ofree[i], 128);
     }
-    mbar_init(pfull, 128);
-    mbar_init(pvdone, 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
   // zero the Q tiles so that rows of absent tokens hold finite values
-  for (uint32_t x = threadIdx.x; x < 2 * L::kQ / 16; x += blockDim.x)
+  for (uint32_t x = threadIdx.x; x < kNQ * L::kQ / 16; x += blockDim.x)
     reinterpret_cast<uint4*>(smem + L::kOffQ)[x] = make_uint4(0, 0, 0, 0);
   fence_proxy_async_smem();
   if (warp == 1) tmem_alloc(tmem_slot, kTmemCols);
@@ -269,268 +319,343 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t tS = tmem;          // S buffers: columns [0,128) and [128,256)
-  const uint32_t tO = tmem + 256;    // O buffers: columns [256, 256+D) and [256+D, 256+2D)
+  const uint32_t tS = tmem;          // S/P buffers
+  const uint32_t tO = tmem + 256;    // O buffers
 
-  if (warp == 0) {
-    // ----------------------------------------------------------------- TMA
-    // The whole warp walks the tiles: lane j gathers tokens j, j+32, ... of a
-    // tile, so the entry loads and the per-token Q copies proceed in parallel.
-    // Tile descriptors are read two tiles ahead, entries one tile ahead.
-    if (t_begin < t_end) {
-      if (lane == 0) {
-        tma_prefetch_desc(&tm_q);
-        tma_prefetch_desc(&tm_k);
-        tma_prefetch_desc(&tm_v);
-      }
-      const int4 zero4 = make_int4(-1, 0, 0, 0);
-      int4 td_cur = p.w.tiles[t_begin];
-      int4 td_nx = t_begin + 1 < t_end ? p.w.tiles[t_begin + 1] : zero4;
-      uint32_t ent_cur[4];
+  if (wgid == 0) {
+    regs_dec<56>();
+    if (warp == 0) {
+      // --------------------------------------------------------------- TMA
+      // The whole warp walks the tiles: lane j gathers tokens j, j+32, ... of
+      // a tile (up to 128 tokens when r = 1).  Tile metadata comes from the
+      // shared ring filled by warp 2.
+      if (n > 0) {
+        if (lane == 0) {
+          tma_prefetch_desc(&tm_q);
+          tma_prefetch_desc(&tm_k);
+          tma_prefetch_desc(&tm_v);
+        }
+        int prev_col = -1;
+        long long u = -1;   // column ordinal
+        for (long long i = 0; i < n; ++i) {
+          const long long bi = i / kmb;
+          const int ms = static_cast<int>(bi & 1);
+          const int slot = ms * kmb + static_cast<int>(i % kmb);
+          int ok = 1;
+          if (i % kmb == 0) {
+            ok = mbar_wait(&mfull[ms], (bi >> 1) & 1, abort_flag, p.err) ? 1 : 0;
+            ok = __shfl_sync(0xffffffffu, ok, 0);
+            if (!ok) break;
+          }
+          const int col = tcol[ms * kMBMax + static_cast<int>(i % kmb)];
+          const bool last = tlast[ms * kMBMax + static_cast<int>(i % kmb)] != 0;
+          uint32_t ent[4];
 #pragma unroll
-      for (int x = 0; x < 4; ++x)
-        ent_cur[x] = lane + 32 * x < td_cur.z ? p.w.entries[td_cur.y + lane + 32 * x] : 0u;
-      int prev_col = -1;
-      long long u = -1;   // column ordinal
-      for (long long ti = t_begin; ti < t_end; ++ti) {
-        const long long i = ti - t_begin;
-        const int4 td = td_cur;
-        uint32_t ent[4];
+          for (int x = 0; x < 4; ++x)
+            ent[x] = lane + 32 * x < tpt ? tent[slot * tpt + lane + 32 * x] : 0xFFFFFFFFu;
+          __syncwarp();
+          if (lane == 0 && (i % kmb == kmb - 1 || i + 1 == n)) mbar_arrive(&mempty[ms]);
+          const int bg = static_cast<int>(col / p.nb);
+          const int blk = static_cast<int>(col - static_cast<long long>(bg) * p.nb);
+          const bool newcol = col != prev_col;
+          if (newcol) {
+            prev_col = col;
+            ++u;
+            const int st = static_cast<int>(u & 1);
+            if (lane == 0) {
+              ok = mbar_wait(&kvempty[st], ((u >> 1) & 1) ^ 1, abort_flag, p.err) ? 1 : 0;
+              if (ok) {
+                mbar_arrive_expect_tx(&kvfull[st], 2 * L::kKV);
 #pragma unroll
-        for (int x = 0; x < 4; ++x) ent[x] = ent_cur[x];
-        const int4 td_nn = ti + 2 < t_end ? p.w.tiles[ti + 2] : zero4;
-#pragma unroll
-        for (int x = 0; x < 4; ++x)
-          ent_cur[x] = lane + 32 * x < td_nx.z ? p.w.entries[td_nx.y + lane + 32 * x] : 0u;
-        td_cur = td_nx;
-        td_nx = td_nn;
-
-        const int col = td.x;
-        const int bg = static_cast<int>(col / p.nb);
-        const int blk = static_cast<int>(col - static_cast<long long>(bg) * p.nb);
-        int ok = 1;
-        if (col != prev_col) {
-          prev_col = col;
-          ++u;
-          const int st = static_cast<int>(u & 1);
-          if (lane == 0) {
-            ok = mbar_wait(&kvempty[st], ((u >> 1) & 1) ^ 1, abort_flag, p.err) ? 1 : 0;
-            if (ok) {
-              mbar_arrive_expect_tx(&kvfull[st], 2 * L::kKV);
-#pragma unroll
-              for (int c = 0; c < D / 64; ++c) {
-                tma_load_3d(smem + L::kOffK + st * L::kKV + c * 16384, &tm_k, &kvfull[st], c * 64,
-                            blk * 128, bg);
-                tma_load_3d(smem + L::kOffV + st * L::kKV + c * 16384, &tm_v, &kvfull[st], c * 64,
-                            blk * 128, bg);
+                for (int c = 0; c < D / 64; ++c) {
+                  tma_load_3d(smem + L::kOffK + st * L::kKV + c * 16384, &tm_k, &kvfull[st],
+                              c * 64, blk * 128, bg);
+                  tma_load_3d(smem + L::kOffV + st * L::kKV + c * 16384, &tm_v, &kvfull[st],
+                              c * 64, blk * 128, bg);
+                }
               }
+            }
+            ok = __shfl_sync(0xffffffffu, ok, 0);
+            if (!ok) break;
+          }
+          int cnt = 0;
+#pragma unroll
+          for (int x = 0; x < 4; ++x)
+            cnt += __popc(__ballot_sync(0xffffffffu, ent[x] != 0xFFFFFFFFu));
+          const int qb = static_cast<int>(i % kNQ);
+          if (lane == 0) {
+            ok = mbar_wait(&qempty[qb], ((i / kNQ) & 1) ^ 1, abort_flag, p.err) ? 1 : 0;
+            if (ok) {
+              meta[qb * 4 + 0] = static_cast<int>(u & 1);
+              meta[qb * 4 + 1] = newcol ? 1 : 0;
+              meta[qb * 4 + 2] = last ? 1 : 0;
+              mbar_arrive_expect_tx(&qfull[qb], static_cast<uint32_t>(cnt * p.r * D * 2));
             }
           }
           ok = __shfl_sync(0xffffffffu, ok, 0);
           if (!ok) break;
-        }
-        const int qb = static_cast<int>(i & 1);
-        const int cnt = td.z;
-        if (lane == 0) {
-          ok = mbar_wait(&qempty[qb], ((i >> 1) & 1) ^ 1, abort_flag, p.err) ? 1 : 0;
-          if (ok) mbar_arrive_expect_tx(&qfull[qb], static_cast<uint32_t>(cnt * p.r * D * 2));
-        }
-        ok = __shfl_sync(0xffffffffu, ok, 0);
-        if (!ok) break;
-        const int b = bg / p.G, g = bg % p.G;
+          const int b = bg / p.G, g = bg % p.G;
 #pragma unroll
-        for (int x = 0; x < 4; ++x) {
-          const int j = lane + 32 * x;
-          if (j < cnt) {
-            const int t = static_cast<int>(ent[x] >> 6);
-            const int row = (b * p.T + t) * p.H + g * p.r;
+          for (int x = 0; x < 4; ++x) {
+            const int j = lane + 32 * x;
+            if (ent[x] != 0xFFFFFFFFu) {
+              const int row = (b * p.T + static_cast<int>(ent[x] >> 6)) * p.H + g * p.r;
 #pragma unroll
-            for (int c = 0; c < D / 64; ++c)
-              tma_load_2d(smem + L::kOffQ + qb * L::kQ + c * 16384 + j * p.r * 128, &tm_q,
-                          &qfull[qb], c * 64, row);
+              for (int c = 0; c < D / 64; ++c)
+                tma_load_2d(smem + L::kOffQ + qb * L::kQ + c * 16384 + j * p.r * 128, &tm_q,
+                            &qfull[qb], c * 64, row);
+            }
           }
         }
       }
-    }
-    __syncwarp();
-  } else if (warp == 1) {
-    // ----------------------------------------------------------------- MMA
-    if (lane == 0 && t_begin < t_end) {
-      const long long n = t_end - t_begin;
-      bool ok = true;
-      int prev_col = -1;
-      long long u = -1;
-      int cur_stage = 0;
-      // columns of the next two tiles, read ahead of use
-      int col_cur = p.w.tiles[t_begin].x;
-      int col_nx = n > 1 ? p.w.tiles[t_begin + 1].x : -1;
-      int stage_of[2] = {0, 0};
-      bool last_of_col[2] = {false, false};
-      auto issue_s = [&](long long i) -> bool {
-        const long long ti = t_begin + i;
-        const int col = col_cur;
-        const int col_next = col_nx;
-        col_cur = col_nx;
-        col_nx = i + 2 < n ? p.w.tiles[ti + 2].x : -1;
-        if (col != prev_col) {
-          prev_col = col;
-          ++u;
-          cur_stage = static_cast<int>(u & 1);
-          if (!mbar_wait(&kvfull[cur_stage], (u >> 1) & 1, abort_flag, p.err)) return false;
-        }
-        const int qb = static_cast<int>(i & 1);
-        stage_of[qb] = cur_stage;
-        last_of_col[qb] = col_next != col;
-        if (!mbar_wait(&qfull[qb], (i >> 1) & 1, abort_flag, p.err)) return false;
-        if (!mbar_wait(&sempty[qb], ((i >> 1) & 1) ^ 1, abort_flag, p.err)) return false;
-        tc_fence_after();
-        const uint32_t qa = smem_u32(smem + L::kOffQ + qb * L::kQ);
-        const uint32_t ka = smem_u32(smem + L::kOffK + cur_stage * L::kKV);
+      __syncwarp();
+    } else if (warp == 2) {
+      // ---------------------------------------------------------- metadata
+      // Batches of kmb tiles: descriptors and entries into the shared ring
+      // (all loads of a batch in flight together), then the batch's query
+      // rows are prefetched into L2 ahead of the gathers.
+      for (long long bi = 0; bi * kmb < n; ++bi) {
+        const int ms = static_cast<int>(bi & 1);
+        if (!mbar_wait(&mempty[ms], ((bi >> 1) & 1) ^ 1, abort_flag, p.err)) break;
+        const long long a = t_begin + bi * kmb;
+        const int nt = static_cast<int>(min(static_cast<long long>(kmb), t_end - a));
+        // columns of the batch's tiles and of the tile after it
+        const int mycol = lane <= nt && a + lane < ntiles ? p.w.tiles[a + lane].x : -1;
+        const int nextcol = __shfl_down_sync(0xffffffffu, mycol, 1);
+        // entries of tiles a .. a+nt-1 are contiguous: nt * tpt words
+        const int nent = nt * tpt;
+        for (int base = 0; base < nent; base += 8 * 32) {
+          uint32_t ev[8];
 #pragma unroll
-        for (int ks = 0; ks < D / 16; ++ks) {
-          const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
-          tc_mma_ss(tS + qb * 128, smem_desc(qa + off, 16, 1024, 2),
-                    smem_desc(ka + off, 16, 1024, 2), kIdescS, ks > 0 ? 1u : 0u);
-        }
-        tc_commit(&sfull[qb]);
-        tc_commit(&qempty[qb]);
-        return true;
-      };
-      ok = issue_s(0);
-      for (long long i = 0; ok && i < n; ++i) {
-        const int qb = static_cast<int>(i & 1);
-        const int st = stage_of[qb];
-        const bool last = last_of_col[qb];
-        if (i + 1 < n && !(ok = issue_s(i + 1))) break;
-        if (!(ok = mbar_wait(pfull, i & 1, abort_flag, p.err))) break;
-        if (!(ok = mbar_wait(&ofree[qb], ((i >> 1) & 1) ^ 1, abort_flag, p.err))) break;
-        tc_fence_after();
-        const uint32_t pa = smem_u32(smem + L::kOffP);
-        const uint32_t va = smem_u32(smem + L::kOffV + st * L::kKV);
+          for (int x = 0; x < 8; ++x) {
+            const int idx = base + lane + 32 * x;
+            ev[x] = idx < nent ? p.w.tile_ent[a * tpt + idx] : 0xFFFFFFFFu;
+          }
 #pragma unroll
-        for (int ks = 0; ks < 8; ++ks) {   // 128 keys in steps of 16
-          const uint64_t ad = smem_desc(pa + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024, 2);
-          const uint64_t bd = smem_desc(va + ks * 16 * 128, 16384, 1024, 2);
-          tc_mma_ss(tO + qb * D, ad, bd, kIdescO, ks > 0 ? 1u : 0u);
+          for (int x = 0; x < 8; ++x) {
+            const int idx = base + lane + 32 * x;
+            if (idx < nent) tent[(ms * kmb) * tpt + idx] = ev[x];
+          }
         }
-        tc_commit(pvdone);
-        if (last) tc_commit(&kvempty[st]);
+        if (lane < nt) {
+          tcol[ms * kMBMax + lane] = mycol;
+          tlast[ms * kMBMax + lane] = (a + lane + 1 >= t_end || nextcol != mycol) ? 1 : 0;
+        }
+        __syncwarp();
+        mbar_arrive(&mfull[ms]);
+        // L2 prefetch of the query rows these tiles will gather
+        for (int tt = 0; tt < nt; ++tt) {
+          const int col = __shfl_sync(0xffffffffu, mycol, tt);
+          const int bg = static_cast<int>(col / p.nb);
+          const int b = bg / p.G, g = bg % p.G;
+          for (int jj = lane; jj < tpt; jj += 32) {
+            const uint32_t e = tent[(ms * kmb + tt) * tpt + jj];
+            if (e != 0xFFFFFFFFu) {
+              const int row = (b * p.T + static_cast<int>(e >> 6)) * p.H + g * p.r;
+#pragma unroll
+              for (int c = 0; c < D / 64; ++c) tma_prefetch_l2_2d(&tm_q, c * 64, row);
+            }
+          }
+        }
       }
+      __syncwarp();
+    } else if (warp == 1) {
+      // --------------------------------------------------------------- MMA
+      // Order: S(0), S(1), then per tile i: PV(i), S(i+2).  tcgen05 MMAs of
+      // one thread execute in issue order, so S(i+2) may overwrite the S/P
+      // buffer of tile i right after PV(i) has been issued.
+      if (lane == 0 && n > 0) {
+        bool ok = true;
+        long long u = -1;
+        int stage_of[4] = {0, 0, 0, 0};
+        bool last_of_col[4] = {false, false, false, false};
+        auto issue_s = [&](long long j) -> bool {
+          const int qb = static_cast<int>(j % kNQ);
+          if (!mbar_wait(&qfull[qb], (j / kNQ) & 1, abort_flag, p.err)) return false;
+          const int st = meta[qb * 4 + 0];
+          const bool newcol = meta[qb * 4 + 1] != 0;
+          last_of_col[j & 3] = meta[qb * 4 + 2] != 0;
+          stage_of[j & 3] = st;
+          if (newcol) {
+            ++u;
+            if (!mbar_wait(&kvfull[st], (u >> 1) & 1, abort_flag, p.err)) return false;
+          }
+          tc_fence_after();
+          const uint32_t qa = smem_u32(smem + L::kOffQ + qb * L::kQ);
+          const uint32_t ka = smem_u32(smem + L::kOffK + st * L::kKV);
+          const int sb = static_cast<int>(j & 1);
+#pragma unroll
+          for (int ks = 0; ks < D / 16; ++ks) {
+            const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
+            tc_mma_ss(tS + sb * 128, smem_desc(qa + off, 16, 1024, 2),
+                      smem_desc(ka + off, 16, 1024, 2), kIdescS, ks > 0 ? 1u : 0u);
+          }
+          tc_commit(&sfull[sb]);
+          tc_commit(&qempty[qb]);
+          return true;
+        };
+        ok = issue_s(0);
+        if (ok && n > 1) ok = issue_s(1);
+        for (long long i = 0; ok && i < n; ++i) {
+          const int sb = static_cast<int>(i & 1);
+          const int st = stage_of[i & 3];
+          const bool last = last_of_col[i & 3];
+          if (!(ok = mbar_wait(&pfull[sb], (i >> 1) & 1, abort_flag, p.err))) break;
+          if (!(ok = mbar_wait(&ofree[sb], ((i >> 1) & 1) ^ 1, abort_flag, p.err))) break;
+          tc_fence_after();
+          const uint32_t va = smem_u32(smem + L::kOffV + st * L::kKV);
+#pragma unroll
+          for (int ks = 0; ks < 8; ++ks) {   // 128 keys in steps of 16 (8 packed columns)
+            const uint64_t bd = smem_desc(va + ks * 16 * 128, 16384, 1024, 2);
+            tc_mma_ts(tO + sb * D, tS + sb * 128 + ks * 8, bd, kIdescO, ks > 0 ? 1u : 0u);
+          }
+          tc_commit(&ofull[sb]);
+          if (last) tc_commit(&kvempty[st]);
+          if (i + 2 < n && !(ok = issue_s(i + 2))) break;
+        }
+      }
+      __syncwarp();
     }
-    __syncwarp();
+  } else if (wgid <= 2) {
+    // ------------------------------------------- softmax (two warpgroups)
+    regs_inc<176>();
+    const int wg = wgid - 1;                 // takes tiles i with i % 2 == wg
+    const int quarter = warp & 3;
+    const int row = quarter * 32 + lane;
+    const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
+    const uint32_t sbuf = tS + wg * 128 + lane_off;
+    const int tok = row / p.r, head = row % p.r;
+    for (long long i = wg; i < n; i += 2) {
+      const long long ti = t_begin + i;
+      const int col = p.w.tiles[ti].x;
+      const uint32_t e = tok < tpt ? p.w.tile_ent[ti * tpt + tok] : 0xFFFFFFFFu;
+      if (!mbar_wait(&sfull[wg], (i >> 1) & 1, abort_flag, p.err)) break;
+      tc_fence_after();
+      float sv[128];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) tmem_ld32(sbuf + c * 32, sv + c * 32);
+      const int bg = static_cast<int>(col / p.nb);
+      const int blk = static_cast<int>(col - static_cast<long long>(bg) * p.nb);
+      const int b = bg / p.G, g = bg % p.G;
+      const bool valid = e != 0xFFFFFFFFu;
+      int lim = 127;
+      long long prow = 0;
+      if (valid) {
+        const int t = static_cast<int>(e >> 6), slot = static_cast<int>(e & 63u);
+        const int pos = p.q_off + t;
+        if ((pos >> 7) == blk) lim = pos & 127;
+        prow = ((static_cast<long long>(b) * p.T + t) * p.k + slot) * p.H + g * p.r + head;
+      }
+      tc_wait_ld();
+      // Only rows of the local block need the causal mask; the branch is
+      // uniform over the warp in the common case.
+      const bool full = __all_sync(0xffffffffu, lim == 127);
+      if (!full) {
+#pragma unroll
+        for (int x = 0; x < 128; ++x) sv[x] = x <= lim ? sv[x] : -INFINITY;
+      }
+      float m8[8];
+#pragma unroll
+      for (int x = 0; x < 8; ++x) m8[x] = sv[x];
+#pragma unroll
+      for (int x = 8; x < 128; ++x) m8[x & 7] = fmaxf(m8[x & 7], sv[x]);
+      const float mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
+                             fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
+      const float mxs = mx * p.scale_log2;
+      // P = 2^(s*scale - max) as bf16, written over the S columns; l sums the
+      // rounded values the PV product uses
+      float l8[8];
+#pragma unroll
+      for (int x = 0; x < 8; ++x) l8[x] = 0.f;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t pk[16];
+#pragma unroll
+        for (int x = 0; x < 32; x += 2) {
+          const float e0 = fast_exp2(fmaf(sv[c * 32 + x], p.scale_log2, -mxs));
+          const float e1 = fast_exp2(fmaf(sv[c * 32 + x + 1], p.scale_log2, -mxs));
+          __nv_bfloat162 h2 = __floats2bfloat162_rn(e0, e1);
+          const uint32_t w = *reinterpret_cast<uint32_t*>(&h2);
+          pk[x >> 1] = w;
+          l8[(x >> 1) & 7] += __uint_as_float(w << 16) + __uint_as_float(w & 0xFFFF0000u);
+        }
+        tmem_st16(sbuf + c * 16, pk);
+      }
+      const float l = ((l8[0] + l8[1]) + (l8[2] + l8[3])) + ((l8[4] + l8[5]) + (l8[6] + l8[7]));
+      tc_wait_st();
+      tc_fence_before();
+      mbar_arrive(&pfull[wg]);
+      if (valid) reinterpret_cast<float2*>(p.w.part_ml)[prow] = make_float2(mxs, l);
+      // 1/l for the epilogue of this tile
+      if (!mbar_wait(&lempty[wg], ((i >> 1) & 1) ^ 1, abort_flag, p.err)) break;
+      linv[wg * 128 + row] = 1.f / l;
+      mbar_arrive(&lfull[wg]);
+    }
   } else {
-    // ------------------------------------------------ softmax + epilogue
+    // ------------------------------------------------------------- epilogue
+    // O row (scaled by 1/l, bf16) -> swizzled staging tile -> one TMA store
+    // per token of r rows (the rows of a token's heads are contiguous).
+    regs_dec<96>();
     const int quarter = warp & 3;
     const int row = quarter * 32 + lane;
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
     const int tok = row / p.r, head = row % p.r;
-    const long long n = t_end - t_begin;
-    uint8_t* prow = smem + L::kOffP + row * 128;
-    // descriptors two tiles ahead, this row's entry one tile ahead
-    const int4 zero4 = make_int4(-1, 0, 0, 0);
-    int4 td_cur = n > 0 ? p.w.tiles[t_begin] : zero4;
-    int4 td_nx = n > 1 ? p.w.tiles[t_begin + 1] : zero4;
-    uint32_t ent_cur = tok < td_cur.z ? p.w.entries[td_cur.y + tok] : 0u;
-    // state of the tile whose output is pending
-    bool pend_valid = false;
-    long long pend_row = 0;     // row of the part arrays: ((b*T + t)*k + slot)*H + h
-    float pend_inv_l = 0.f;
-    bool ok = true;
-    for (long long i = 0; i <= n && ok; ++i) {
-      bool cur_valid = false;
-      long long cur_row = 0;
-      float cur_inv_l = 0.f;
-      uint32_t pk[64];
-      if (i < n) {
-        const int qb = static_cast<int>(i & 1);
-        const int4 td = td_cur;
-        const uint32_t e = ent_cur;
-        const int4 td_nn = i + 2 < n ? p.w.tiles[t_begin + i + 2] : zero4;
-        ent_cur = tok < td_nx.z ? p.w.entries[td_nx.y + tok] : 0u;
-        td_cur = td_nx;
-        td_nx = td_nn;
-        const int col = td.x;
-        const int bg = static_cast<int>(col / p.nb);
-        const int blk = static_cast<int>(col - static_cast<long long>(bg) * p.nb);
-        const int b = bg / p.G, g = bg % p.G;
-        cur_valid = tok < td.z;
-        int lim = 127;
-        if (cur_valid) {
-          const int t = static_cast<int>(e >> 6), slot = static_cast<int>(e & 63u);
-          const int pos = p.q_off + t;
-          if ((pos >> 7) == blk) lim = pos & 127;
-          cur_row = ((static_cast<long long>(b) * p.T + t) * p.k + slot) * p.H + g * p.r + head;
-        }
-        if (!(ok = mbar_wait(&sfull[qb], (i >> 1) & 1, abort_flag, p.err))) break;
-        tc_fence_after();
-        float sv[128];
+    uint8_t* stage = smem + L::kOffStage;
+    uint8_t* srow = stage + row * 128;
+    bool stored = false;   // this thread has bulk stores in flight
+    for (long long i = 0; i < n; ++i) {
+      const long long ti = t_begin + i;
+      const int col = p.w.tiles[ti].x;
+      const uint32_t e = tok < tpt ? p.w.tile_ent[ti * tpt + tok] : 0xFFFFFFFFu;
+      const int ob = static_cast<int>(i & 1);
+      if (!mbar_wait(&ofull[ob], (i >> 1) & 1, abort_flag, p.err)) break;
+      if (!mbar_wait(&lfull[ob], (i >> 1) & 1, abort_flag, p.err)) break;
+      tc_fence_after();
+      const float il = linv[ob * 128 + row];
+      mbar_arrive(&lempty[ob]);
+      // the staging tile must be free: own stores read out, then everyone's
+      if (stored) {
+        bulk_wait_read0();
+        stored = false;
+      }
+      named_bar_sync(1, 128);
 #pragma unroll
-        for (int c = 0; c < 4; ++c) tmem_ld32(tS + qb * 128 + lane_off + c * 32, sv + c * 32);
+      for (int c = 0; c < D / 32; c += 2) {
+        float ov[64];
+        tmem_ld32(tO + ob * D + lane_off + c * 32, ov);
+        tmem_ld32(tO + ob * D + lane_off + c * 32 + 32, ov + 32);
         tc_wait_ld();
-        tc_fence_before();
-        mbar_arrive(&sempty[qb]);
-        float mx = -INFINITY;
-#pragma unroll
-        for (int c = 0; c < 128; ++c) {
-          sv[c] = c <= lim ? sv[c] : -INFINITY;
-          mx = fmaxf(mx, sv[c]);
+        if (c + 2 >= D / 32) {
+          tc_fence_before();
+          mbar_arrive(&ofree[ob]);
         }
-        const float mxs = mx * p.scale_log2;
-        float l = 0.f;
 #pragma unroll
-        for (int c = 0; c < 128; c += 2) {
-          const float e0 = fast_exp2(fmaf(sv[c], p.scale_log2, -mxs));
-          const float e1 = fast_exp2(fmaf(sv[c + 1], p.scale_log2, -mxs));
-          __nv_bfloat162 h2 = __floats2bfloat162_rn(e0, e1);
-          pk[c >> 1] = *reinterpret_cast<uint32_t*>(&h2);
-          const float2 back = __bfloat1622float2(h2);
-          l += back.x + back.y;
+        for (int x = 0; x < 8; ++x) {
+          __nv_bfloat162 h0 = __floats2bfloat162_rn(ov[8 * x] * il, ov[8 * x + 1] * il);
+          __nv_bfloat162 h1 = __floats2bfloat162_rn(ov[8 * x + 2] * il, ov[8 * x + 3] * il);
+          __nv_bfloat162 h2 = __floats2bfloat162_rn(ov[8 * x + 4] * il, ov[8 * x + 5] * il);
+          __nv_bfloat162 h3 = __floats2bfloat162_rn(ov[8 * x + 6] * il, ov[8 * x + 7] * il);
+          const int u = (c * 32 + 8 * x) >> 3;            // 16-byte unit of the row
+          uint4* dst = reinterpret_cast<uint4*>(srow + (u >> 3) * 16384 + (((u & 7) ^ (row & 7)) << 4));
+          *dst = make_uint4(*reinterpret_cast<uint32_t*>(&h0), *reinterpret_cast<uint32_t*>(&h1),
+                            *reinterpret_cast<uint32_t*>(&h2), *reinterpret_cast<uint32_t*>(&h3));
         }
-        cur_inv_l = 1.f / l;
-        if (cur_valid) p.w.part_lse[cur_row] = mxs + log2f(l);
       }
-      // epilogue of the previous tile (its PV also frees the P buffer)
-      if (i > 0) {
-        const long long ip = i - 1;
-        const int ob = static_cast<int>(ip & 1);
-        if (!(ok = mbar_wait(pvdone, ip & 1, abort_flag, p.err))) break;
-        tc_fence_after();
+      fence_proxy_async_smem();
+      named_bar_sync(1, 128);
+      if (head == 0 && e != 0xFFFFFFFFu) {
+        const int bg = static_cast<int>(col / p.nb);
+        const int b = bg / p.G, g = bg % p.G;
+        const int t = static_cast<int>(e >> 6), slot = static_cast<int>(e & 63u);
+        const int orow = ((b * p.T + t) * p.k + slot) * p.H + g * p.r;
 #pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-          float ov[32];
-          tmem_ld32(tO + ob * D + lane_off + c * 32, ov);
-          tc_wait_ld();
-          if (pend_valid) {
-            uint4* dst = reinterpret_cast<uint4*>(p.w.part_o + pend_row * D + c * 32);
-#pragma unroll
-            for (int x = 0; x < 4; ++x) {
-              __nv_bfloat162 h0 = __floats2bfloat162_rn(ov[8 * x] * pend_inv_l, ov[8 * x + 1] * pend_inv_l);
-              __nv_bfloat162 h1 = __floats2bfloat162_rn(ov[8 * x + 2] * pend_inv_l, ov[8 * x + 3] * pend_inv_l);
-              __nv_bfloat162 h2 = __floats2bfloat162_rn(ov[8 * x + 4] * pend_inv_l, ov[8 * x + 5] * pend_inv_l);
-              __nv_bfloat162 h3 = __floats2bfloat162_rn(ov[8 * x + 6] * pend_inv_l, ov[8 * x + 7] * pend_inv_l);
-              dst[x] = make_uint4(*reinterpret_cast<uint32_t*>(&h0), *reinterpret_cast<uint32_t*>(&h1),
-                                  *reinterpret_cast<uint32_t*>(&h2), *reinterpret_cast<uint32_t*>(&h3));
-            }
-          }
-        }
-        tc_fence_before();
-        mbar_arrive(&ofree[ob]);
-      }
-      if (i < n) {
-        // P row -> shared memory, 128-byte swizzled K-major layout (2 chunks of 64 keys)
-#pragma unroll
-        for (int u = 0; u < 16; ++u) {
-          const int chunk = u >> 3, unit = u & 7;
-          uint4* dst = reinterpret_cast<uint4*>(prow + chunk * 16384 + ((unit ^ (row & 7)) << 4));
-          *dst = make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
-        }
-        fence_proxy_async_smem();
-        mbar_arrive(pfull);
-        pend_valid = cur_valid;
-        pend_row = cur_row;
-        pend_inv_l = cur_inv_l;
+        for (int c = 0; c < D / 64; ++c)
+          tma_store_2d(&tm_o, stage + c * 16384 + tok * p.r * 128, c * 64, orow);
+        bulk_commit_group();
+        stored = true;
       }
     }
+    if (stored) bulk_wait0();
   }
 
   tc_fence_before();
@@ -542,38 +667,39 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 }
 
 // ------------------------------------------------------------- 4. combine
-// One CTA per (sequence, token): merge the k normalised partials of each of
-// the H heads by their log-sum-exp.  Partials of one token are laid out
-// [slot][head][d], so each slot is one contiguous H*d run.
+// One CTA per (sequence, token): merge the k partials of each of the H heads.
+// Partial s of a row holds the normalised output O_s (bf16), its running max
+// m_s and sum l_s = sum_j 2^(x_j - m_s) (x in log2 units).  With M = max_s m_s
+// and w_s = 2^(m_s - M) l_s:  o = sum_s w_s O_s / sum_s w_s.
 template <int D>
 __global__ void __launch_bounds__(256) combine_kernel(const int32_t* __restrict__ sel,
                                                       const PrefillWs w, uint16_t* __restrict__ o,
                                                       float* __restrict__ lse, int H, int G,
                                                       int r, int k) {
   constexpr int CH = D / 8;                  // 16-byte chunks per head row
-  extern __shared__ float sm_lse[];          // [k][H] log2 units, -inf for unused slots
+  extern __shared__ float2 sm_ml[];          // [k][H] (m, l), m = -inf for unused slots
   const long long bt = blockIdx.x;           // b*T + t
-  const float* lsrc = w.part_lse + bt * k * H;
+  const float2* msrc = reinterpret_cast<const float2*>(w.part_ml) + bt * k * H;
   const int32_t* srow = sel + bt * G * k;
   for (int x = threadIdx.x; x < k * H; x += blockDim.x) {
     const int s = x / H, h = x % H;
-    sm_lse[x] = srow[(h / r) * k + s] >= 0 ? lsrc[x] : -INFINITY;
+    sm_ml[x] = srow[(h / r) * k + s] >= 0 ? msrc[x] : make_float2(-INFINITY, 0.f);
   }
   __syncthreads();
   const uint16_t* osrc = w.part_o + bt * k * H * D;
   for (int item = threadIdx.x; item < H * CH; item += blockDim.x) {
     const int h = item / CH, c = item % CH;
     float M = -INFINITY;
-    for (int s = 0; s < k; ++s) M = fmaxf(M, sm_lse[s * H + h]);
+    for (int s = 0; s < k; ++s) M = fmaxf(M, sm_ml[s * H + h].x);
     float acc[8];
 #pragma unroll
     for (int e = 0; e < 8; ++e) acc[e] = 0.f;
     float den = 0.f;
 #pragma unroll 4
     for (int s = 0; s < k; ++s) {
-      const float ls = sm_lse[s * H + h];
-      if (ls == -INFINITY) continue;
-      const float ws = exp2f(ls - M);
+      const float2 ml = sm_ml[s * H + h];
+      if (ml.x == -INFINITY) continue;
+      const float ws = exp2f(ml.x - M) * ml.y;
       den += ws;
       const uint4 u = __ldcs(reinterpret_cast<const uint4*>(osrc + (static_cast<long long>(s) * H + h) * D) + c);
       const uint32_t wds[4] = {u.x, u.y, u.z, u.w};
@@ -600,7 +726,7 @@ template <int D>
 cudaError_t launch_attn(const msa_shape& s, const uint16_t* q, const uint16_t* k,
                         const uint16_t* v, const AttnParams& p, const DevCtx* ctx,
                         cudaStream_t st) {
-  CUtensorMap tq, tk, tv;
+  CUtensorMap tq, tk, tv, to;
   const uint64_t dq[2] = {static_cast<uint64_t>(D),
                           static_cast<uint64_t>(s.batch) * s.seq_q * s.n_q_heads};
   const uint64_t sq[1] = {static_cast<uint64_t>(D) * 2};
@@ -610,21 +736,25 @@ cudaError_t launch_attn(const msa_shape& s, const uint16_t* q, const uint16_t* k
   const uint64_t sk[2] = {static_cast<uint64_t>(D) * 2,
                           static_cast<uint64_t>(s.seq_kv) * D * 2};
   const uint32_t bk[3] = {64, 128, 1};
+  const uint64_t dpo[2] = {static_cast<uint64_t>(D),
+                           static_cast<uint64_t>(s.batch) * s.seq_q * s.topk * s.n_q_heads};
   if (!encode_tmap(&tq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, q, dq, sq, bq,
                    CU_TENSOR_MAP_SWIZZLE_128B) ||
       !encode_tmap(&tk, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, k, dk, sk, bk,
                    CU_TENSOR_MAP_SWIZZLE_128B) ||
       !encode_tmap(&tv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, v, dk, sk, bk,
+                   CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !encode_tmap(&to, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, p.w.part_o, dpo, sq, bq,
                    CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorInvalidValue;
-  const size_t smem = AttnSmem<D>::kBytes + 1024;
+  const size_t smem = AttnSmem<D>::kBytes;
   cudaError_t e = cudaFuncSetAttribute(kvouter_attn_kernel<D>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   {
     ProfScope ps_("kvouter_attn", st);
-    kvouter_attn_kernel<D><<<ctx->num_sms, kAttnThreads, smem, st>>>(tq, tk, tv, p);
+    kvouter_attn_kernel<D><<<ctx->num_sms, kAttnThreads, smem, st>>>(tq, tk, tv, to, p);
   }
   return cudaGetLastError();
 }
@@ -666,7 +796,7 @@ cudaError_t launch_sparse_prefill(const msa_shape& s, const uint16_t* q, const u
   }
   {
     ProfScope ps_("make_tiles", st);
-    make_tiles_kernel<<<static_cast<unsigned>(ceil_div(w.ncol, 256)), 256, 0, st>>>(w, tpt);
+    make_tiles_kernel<<<static_cast<unsigned>(ceil_div(w.max_tiles, 256)), 256, 0, st>>>(w, tpt);
   }
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
 
@@ -687,7 +817,7 @@ cudaError_t launch_sparse_prefill(const msa_shape& s, const uint16_t* q, const u
                         : launch_attn<64>(s, q, k, v, p, ctx, st);
   if (e != cudaSuccess) return e;
   const unsigned ntok = static_cast<unsigned>(static_cast<long long>(s.batch) * s.seq_q);
-  const size_t csmem = sizeof(float) * s.topk * s.n_q_heads;
+  const size_t csmem = sizeof(float2) * s.topk * s.n_q_heads;
   {
     ProfScope ps_("combine", st);
     if (s.head_dim == 128)
