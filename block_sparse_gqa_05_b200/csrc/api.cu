@@ -302,6 +302,22 @@ msa_status msa_sparse_attn_decode(const msa_shape* s, const uint16_t* q, const u
                                  static_cast<cudaStream_t>(stream)));
 }
 
+}  // extern "C"
+
+namespace msa {
+// Argument checks of the decode entry point without a workspace argument.
+msa_status check_decode_static_args(const msa_shape* s, const uint16_t* q, const uint16_t* k,
+                                    const uint16_t* v, const int32_t* sel, const uint16_t* o,
+                                    const float* lse) {
+  msa_status st = check_shape(s, true, false);
+  if (st != MSA_OK) return st;
+  if ((st = check_decode(s)) != MSA_OK) return st;
+  return check_attn_ptrs(q, k, v, sel, true, o, lse);
+}
+}  // namespace msa
+
+extern "C" {
+
 msa_status msa_forward(const msa_shape* s, const uint16_t* q, const uint16_t* k,
                        const uint16_t* v, const uint16_t* q_idx, const uint16_t* k_idx,
                        uint16_t* o, float* lse, int32_t* sel_out, void* ws, size_t ws_bytes,

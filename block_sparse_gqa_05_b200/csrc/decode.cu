@@ -13,6 +13,8 @@
 // bandwidth on the K/V bytes.
 #include <math.h>
 
+#include <mutex>
+
 #include "internal.h"
 #include "ptx.cuh"
 
@@ -390,3 +392,46 @@ cudaError_t launch_decode(const msa_shape& s, const uint16_t* q, const uint16_t*
 }
 
 }  // namespace msa
+
+// ------------------------------------------------ decode without allocation
+// Split-K scratch of msa_sparse_attn_decode_static: one static array in
+// device memory, shared by every call on a device.  Host code only ever
+// passes its device address, looked up once per device.
+namespace msa {
+namespace {
+
+static __device__ __align__(256) unsigned char g_decode_static_scratch[MSA_DECODE_STATIC_SCRATCH_BYTES];
+
+std::mutex g_static_mu;
+void* g_static_addr[64] = {};
+
+// Device address of the scratch array on the current device (nullptr on error).
+void* static_scratch_address() {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  std::lock_guard<std::mutex> lk(g_static_mu);
+  if (!g_static_addr[dev]) {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_decode_static_scratch) != cudaSuccess) return nullptr;
+    g_static_addr[dev] = ptr;
+  }
+  return g_static_addr[dev];
+}
+
+}  // namespace
+}  // namespace msa
+
+extern "C" msa_status msa_sparse_attn_decode_static(const msa_shape* s, const uint16_t* q,
+                                                    const uint16_t* k, const uint16_t* v,
+                                                    const int32_t* sel, uint16_t* o, float* lse,
+                                                    void* stream) {
+  msa_status st = msa::check_decode_static_args(s, q, k, v, sel, o, lse);
+  if (st != MSA_OK) return st;
+  if (msa::decode_workspace_bytes(*s, false) > MSA_DECODE_STATIC_SCRATCH_BYTES)
+    return MSA_ERR_WORKSPACE_TOO_SMALL;
+  void* scratch = msa::static_scratch_address();
+  if (!scratch) return MSA_ERR_CUDA;
+  const cudaError_t e = msa::launch_decode(*s, q, k, v, sel, o, lse, scratch, false,
+                                           static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? MSA_OK : MSA_ERR_CUDA;
+}

@@ -56,6 +56,9 @@ size_t decode_workspace_bytes(const msa_shape& s, bool dense);
 cudaError_t launch_decode(const msa_shape& s, const uint16_t* q, const uint16_t* k,
                           const uint16_t* v, const int32_t* sel, uint16_t* o, float* lse,
                           void* ws, bool dense, cudaStream_t st);
+msa_status check_decode_static_args(const msa_shape* s, const uint16_t* q, const uint16_t* k,
+                                    const uint16_t* v, const int32_t* sel, const uint16_t* o,
+                                    const float* lse);
 cudaError_t launch_dense_prefill(const msa_shape& s, const uint16_t* q, const uint16_t* k,
                                  const uint16_t* v, uint16_t* o, float* lse, cudaStream_t st);
 

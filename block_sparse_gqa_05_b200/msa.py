@@ -58,6 +58,8 @@ _SIGS = {
                                  ctypes.c_size_t, _vp], ctypes.c_int),
     "msa_sparse_attn_decode": ([ctypes.POINTER(Shape), _vp, _vp, _vp, _vp, _vp, _vp, _vp,
                                 ctypes.c_size_t, _vp], ctypes.c_int),
+    "msa_sparse_attn_decode_static": ([ctypes.POINTER(Shape), _vp, _vp, _vp, _vp, _vp, _vp, _vp],
+                                      ctypes.c_int),
     "msa_forward": ([ctypes.POINTER(Shape), _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
                      ctypes.c_size_t, _vp], ctypes.c_int),
     "msa_dense_attn_prefill": ([ctypes.POINTER(Shape), _vp, _vp, _vp, _vp, _vp, _vp,
@@ -172,6 +174,18 @@ def sparse_attn_decode(shape: Shape, q, k, v, sel, o=None, lse=None, ws=None, wa
     _check(lib().msa_sparse_attn_decode(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(sel),
                                         _ptr(o), _ptr(lse), _ptr(ws), ws.numel(), _stream(stream)),
            "msa_sparse_attn_decode")
+    return o, lse
+
+
+def sparse_attn_decode_static(shape: Shape, q, k, v, sel, o=None, lse=None, want_lse=True,
+                              stream=None):
+    """msa_sparse_attn_decode_static: decode attention whose scratch is the
+    library's static device array, so nothing is allocated for it.  Calls
+    that may overlap on the GPU share that array and must be serialised."""
+    o, lse = _attn_out(shape, q, o, lse, want_lse)
+    _check(lib().msa_sparse_attn_decode_static(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v),
+                                               _ptr(sel), _ptr(o), _ptr(lse), _stream(stream)),
+           "msa_sparse_attn_decode_static")
     return o, lse
 
 

@@ -164,6 +164,30 @@ msa_status msa_dense_attn_decode(const msa_shape* shape, const uint16_t* q,
                                  const uint16_t* k, const uint16_t* v, uint16_t* o,
                                  float* lse, void* ws, size_t ws_bytes, void* stream);
 
+/* Sparse decode attention that allocates nothing and takes no workspace (no
+ * counterpart on the pages; it serves callers that cannot allocate device
+ * memory on the decode path: for example a serving loop whose memory manager
+ * owns every device buffer in a fixed arena, or one that must not call
+ * cudaMalloc/cudaFree there because those calls synchronise the device and
+ * stall concurrent work).  Same arguments, result and layouts as
+ * msa_sparse_attn_decode, minus ws/ws_bytes: its split-K scratch lives in one
+ * static device array of MSA_DECODE_STATIC_SCRATCH_BYTES compiled into the
+ * library, which every GPU that loads the library holds until the process
+ * exits.  Shapes whose scratch would exceed it (round256(4*B*G) +
+ * round256(4*B*G*k*r) + round256(4*B*G*k*r*d) bytes) return
+ * MSA_ERR_WORKSPACE_TOO_SMALL before any launch; B=32, G=8, k=16, r=8, d=128
+ * fits.  The first call on a device looks up the array's device address with
+ * that device current; make that first call before any stream capture.  All
+ * calls share the one array and it keeps the previous call's contents (the
+ * counters that must start at zero are cleared by every call): calls that can
+ * overlap on the GPU (other streams, other host threads) race, so the caller
+ * must serialise them. */
+#define MSA_DECODE_STATIC_SCRATCH_BYTES (24u << 20)
+msa_status msa_sparse_attn_decode_static(const msa_shape* shape, const uint16_t* q,
+                                         const uint16_t* k, const uint16_t* v,
+                                         const int32_t* sel, uint16_t* o, float* lse,
+                                         void* stream);
+
 /* Reads and clears the device error word of the current device (bit 0: a
  * bounded wait timed out).  Synchronises the current device.  Returns
  * MSA_ERR_DEVICE_TIMEOUT if any bit was set, MSA_OK otherwise; *flags (may be
