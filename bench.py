@@ -290,7 +290,8 @@ def run_msa(args, world, rank, pg):
 
     # ---- decode at 128K, batch 32
     if not args.skip_decode:
-        out["decode"] = run_decode(M, synth.workload("decode_128k_b32", seed=4 + 1000 * rank),
+        dw = synth.workload(args.decode_workload)
+        out["decode"] = run_decode(M, synth.workload(args.decode_workload, seed=dw.seed + 1000 * rank),
                                    args, pg, stream, world, peaks, dense=False)
     # ---- 1M context: prefill chunk + decode, against the dense kernels
     if not args.skip_long:
@@ -314,7 +315,7 @@ def run_decode(M, sp, args, pg, stream, world, peaks, dense):
     prof = M.profile_read()
     M.profile_enable(False)
     kernels = {k: v[0] / v[1] for k, v in prof.items()}
-    res = {"workload": "decode_128k_b32" if sp.seq_kv == 131072 else f"decode_L{sp.seq_kv}_b{sp.batch}",
+    res = {"workload": f"decode_L{sp.seq_kv}_b{sp.batch}",
            "value": sp.batch * world / (ms / 1e3), "unit": "tokens/s", "ms_per_step": ms,
            "kernels_ms_per_launch": {k: round(v, 4) for k, v in kernels.items()}}
     if "decode_attn" in kernels:
@@ -489,6 +490,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="msa", choices=["msa", "reference"])
     ap.add_argument("--workload", default="prefill_128k")
+    ap.add_argument("--decode-workload", default="decode_128k_b32")
     ap.add_argument("--skip-long", action="store_true")
     ap.add_argument("--skip-decode", action="store_true")
     ap.add_argument("--skip-cpu", action="store_true")

@@ -21,6 +21,9 @@ WORKLOADS = {
                                        seed=5, planted=4),
     # 4 sequences x 1M cache, one query each
     "decode_1m_b4": WorkloadSpec(4, 1, 1048576, 1048575, _H, _G, _D, _DI, 128, 16, seed=5, planted=4),
+    # small cases of the same shapes, sized for profiler captures (a few GB on the device)
+    "prefill_16k": WorkloadSpec(1, 16384, 16384, 0, _H, _G, _D, _DI, 128, 16, seed=7, planted=4),
+    "decode_16k_b8": WorkloadSpec(8, 1, 16384, 16383, _H, _G, _D, _DI, 128, 16, seed=8, planted=4),
 }
 
 
