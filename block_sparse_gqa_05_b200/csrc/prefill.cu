@@ -215,7 +215,7 @@ struct AttnParams {
   float scale_log2;
 };
 
-constexpr int kNQ = 2;        // query tile buffers
+constexpr int kNQ = 3;        // query tile buffers
 constexpr int kMBMax = 16;    // most tiles per metadata batch (two batches in flight)
 constexpr int kTentWords = 256; // entry words in the metadata ring (both batches)
 
@@ -223,9 +223,9 @@ template <int D>
 struct AttnSmem {
   static constexpr uint32_t kKV = 128u * D * 2u;     // one K (or V) block tile
   static constexpr uint32_t kQ = 128u * D * 2u;      // 128 query rows
-  static constexpr uint32_t kOffK = 0;
-  static constexpr uint32_t kOffV = 2 * kKV;
-  static constexpr uint32_t kOffQ = 4 * kKV;
+  static constexpr uint32_t kOffK = 0;                      // two K stages
+  static constexpr uint32_t kOffV = 2 * kKV;                // one V tile
+  static constexpr uint32_t kOffQ = 3 * kKV;
   static constexpr uint32_t kOffStage = kOffQ + kNQ * kQ;   // epilogue staging (128 rows x D)
   static constexpr uint32_t kOffLinv = kOffStage + kQ;      // float [2][128]
   static constexpr uint32_t kOffMeta = kOffLinv + 1024;     // int [kNQ][4]
@@ -264,11 +264,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   float* linv = reinterpret_cast<float*>(smem + L::kOffLinv);
   int* meta = reinterpret_cast<int*>(smem + L::kOffMeta);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kOffBar);
-  uint64_t* kvfull = bars;              // [2]
-  uint64_t* kvempty = bars + 2;         // [2]
-  uint64_t* qfull = bars + 4;           // [kNQ]
-  uint64_t* qempty = bars + 4 + kNQ;    // [kNQ]
-  uint64_t* sfull = bars + 4 + 2 * kNQ; // [2]
+  uint64_t* kfull = bars;               // [2]  K stage loaded
+  uint64_t* kempty = bars + 2;          // [2]  K stage free (last S of its column done)
+  uint64_t* vfull = bars + 4;           // V tile loaded
+  uint64_t* vempty = bars + 5;          // V tile free (last PV of its column done)
+  uint64_t* qfull = bars + 6;           // [kNQ]
+  uint64_t* qempty = bars + 6 + kNQ;    // [kNQ]
+  uint64_t* sfull = bars + 6 + 2 * kNQ; // [2]
   uint64_t* pfull = sfull + 2;          // [2]
   uint64_t* ofull = sfull + 4;          // [2]
   uint64_t* ofree = sfull + 6;          // [2]
@@ -292,8 +294,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < 2; ++i) {
-      mbar_init(&kvfull[i], 1);
-      mbar_init(&kvempty[i], 1);
+      mbar_init(&kfull[i], 1);
+      mbar_init(&kempty[i], 1);
       mbar_init(&sfull[i], 1);
       mbar_init(&pfull[i], 128);
       mbar_init(&ofull[i], 1);
@@ -303,6 +305,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       mbar_init(&mfull[i], 32);
       mbar_init(&mempty[i], 1);
     }
+    mbar_init(vfull, 1);
+    mbar_init(vempty, 1);
     for (int i = 0; i < kNQ; ++i) {
       mbar_init(&qfull[i], 1);
       mbar_init(&qempty[i], 1);
@@ -363,16 +367,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             ++u;
             const int st = static_cast<int>(u & 1);
             if (lane == 0) {
-              ok = mbar_wait(&kvempty[st], ((u >> 1) & 1) ^ 1, abort_flag, p.err) ? 1 : 0;
+              ok = mbar_wait(&kempty[st], ((u >> 1) & 1) ^ 1, abort_flag, p.err) ? 1 : 0;
               if (ok) {
-                mbar_arrive_expect_tx(&kvfull[st], 2 * L::kKV);
+                mbar_arrive_expect_tx(&kfull[st], L::kKV);
 #pragma unroll
-                for (int c = 0; c < D / 64; ++c) {
-                  tma_load_3d(smem + L::kOffK + st * L::kKV + c * 16384, &tm_k, &kvfull[st],
+                for (int c = 0; c < D / 64; ++c)
+                  tma_load_3d(smem + L::kOffK + st * L::kKV + c * 16384, &tm_k, &kfull[st],
                               c * 64, blk * 128, bg);
-                  tma_load_3d(smem + L::kOffV + st * L::kKV + c * 16384, &tm_v, &kvfull[st],
-                              c * 64, blk * 128, bg);
-                }
               }
             }
             ok = __shfl_sync(0xffffffffu, ok, 0);
@@ -411,9 +412,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       __syncwarp();
     } else if (warp == 2) {
       // ---------------------------------------------------------- metadata
-      // Batches of kmb tiles: descriptors and entries into the shared ring
-      // (all loads of a batch in flight together), then the batch's query
-      // rows are prefetched into L2 ahead of the gathers.
+      // Batches of kmb tiles: descriptors and entries into the shared ring,
+      // all loads of a batch in flight together.
       for (long long bi = 0; bi * kmb < n; ++bi) {
         const int ms = static_cast<int>(bi & 1);
         if (!mbar_wait(&mempty[ms], ((bi >> 1) & 1) ^ 1, abort_flag, p.err)) break;
@@ -443,76 +443,132 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         }
         __syncwarp();
         mbar_arrive(&mfull[ms]);
-        // L2 prefetch of the query rows these tiles will gather
-        for (int tt = 0; tt < nt; ++tt) {
-          const int col = __shfl_sync(0xffffffffu, mycol, tt);
-          const int bg = static_cast<int>(col / p.nb);
-          const int b = bg / p.G, g = bg % p.G;
-          for (int jj = lane; jj < tpt; jj += 32) {
-            const uint32_t e = tent[(ms * kmb + tt) * tpt + jj];
-            if (e != 0xFFFFFFFFu) {
-              const int row = (b * p.T + static_cast<int>(e >> 6)) * p.H + g * p.r;
+      }
+      __syncwarp();
+    } else if (warp == 3) {
+      // ------------------------------------------------------------ V loader
+      // One V tile, reloaded when the column changes, as soon as the last PV
+      // of the previous column has completed.  Columns are read 32 tiles at a
+      // time.
+      long long u = -1;
+      int prev_col = -1;
+      bool ok = true;
+      for (long long base = 0; ok && base < n; base += 32) {
+        const int mycol = base + lane < n ? p.w.tiles[t_begin + base + lane].x : -1;
+        const int prevlane = __shfl_up_sync(0xffffffffu, mycol, 1);
+        const bool starts = base + lane < n && (lane == 0 ? mycol != prev_col : mycol != prevlane);
+        unsigned m = __ballot_sync(0xffffffffu, starts);
+        prev_col = __shfl_sync(0xffffffffu, mycol, 31);
+        if (base + 32 > n) prev_col = __shfl_sync(0xffffffffu, mycol, static_cast<int>(n - 1 - base));
+        while (m) {
+          const int src = __ffs(m) - 1;
+          m &= m - 1;
+          const int col = __shfl_sync(0xffffffffu, mycol, src);
+          ++u;
+          if (lane == 0) {
+            ok = mbar_wait(vempty, (u & 1) ^ 1, abort_flag, p.err);
+            if (ok) {
+              const int bg = static_cast<int>(col / p.nb);
+              const int blk = static_cast<int>(col - static_cast<long long>(bg) * p.nb);
+              mbar_arrive_expect_tx(vfull, L::kKV);
 #pragma unroll
-              for (int c = 0; c < D / 64; ++c) tma_prefetch_l2_2d(&tm_q, c * 64, row);
+              for (int c = 0; c < D / 64; ++c)
+                tma_load_3d(smem + L::kOffV + c * 16384, &tm_v, vfull, c * 64, blk * 128, bg);
             }
           }
+          ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+          if (!ok) break;
         }
       }
       __syncwarp();
     } else if (warp == 1) {
       // --------------------------------------------------------------- MMA
-      // Order: S(0), S(1), then per tile i: PV(i), S(i+2).  tcgen05 MMAs of
-      // one thread execute in issue order, so S(i+2) may overwrite the S/P
-      // buffer of tile i right after PV(i) has been issued.
+      // Two in-order streams, S(j) = Q K^T and PV(i) = P V, issued by one
+      // thread as soon as each is ready (polling), so a query gather that is
+      // late never holds back the PV of an earlier tile.  S(j) reuses the S/P
+      // buffer of tile j-2, so it is issued only after PV(j-2); tcgen05 MMAs of
+      // one thread execute in issue order, which makes that reuse safe.
       if (lane == 0 && n > 0) {
-        bool ok = true;
-        long long u = -1;
+        long long ns = 0, np = 0;   // next S, next PV
+        long long u = -1;           // K column ordinal (S side)
+        long long uv = -1;          // V column ordinal (PV side)
         int stage_of[4] = {0, 0, 0, 0};
         bool last_of_col[4] = {false, false, false, false};
-        auto issue_s = [&](long long j) -> bool {
-          const int qb = static_cast<int>(j % kNQ);
-          if (!mbar_wait(&qfull[qb], (j / kNQ) & 1, abort_flag, p.err)) return false;
-          const int st = meta[qb * 4 + 0];
-          const bool newcol = meta[qb * 4 + 1] != 0;
-          last_of_col[j & 3] = meta[qb * 4 + 2] != 0;
-          stage_of[j & 3] = st;
-          if (newcol) {
-            ++u;
-            if (!mbar_wait(&kvfull[st], (u >> 1) & 1, abort_flag, p.err)) return false;
-          }
-          tc_fence_after();
-          const uint32_t qa = smem_u32(smem + L::kOffQ + qb * L::kQ);
-          const uint32_t ka = smem_u32(smem + L::kOffK + st * L::kKV);
-          const int sb = static_cast<int>(j & 1);
+        bool first_of_col[4] = {false, false, false, false};
+        bool s_meta = false;        // meta of S(ns) read, waiting for its K stage
+        int s_st = 0;
+        bool s_last = false;
+        uint64_t t_idle = 0;
+        while (np < n) {
+          bool progress = false;
+          // ---- S(ns)
+          if (ns < n && ns < np + 2) {
+            const int qb = static_cast<int>(ns % kNQ);
+            if (!s_meta && mbar_test(&qfull[qb], (ns / kNQ) & 1)) {
+              s_st = meta[qb * 4 + 0];
+              const bool newcol = meta[qb * 4 + 1] != 0;
+              s_last = meta[qb * 4 + 2] != 0;
+              last_of_col[ns & 3] = s_last;
+              first_of_col[ns & 3] = newcol;
+              stage_of[ns & 3] = s_st;
+              if (newcol) ++u;
+              s_meta = true;
+              s_st |= newcol ? 0x100 : 0;
+            }
+            if (s_meta && (!(s_st & 0x100) || mbar_test(&kfull[s_st & 1], (u >> 1) & 1))) {
+              const int st = s_st & 1;
+              tc_fence_after();
+              const uint32_t qa = smem_u32(smem + L::kOffQ + qb * L::kQ);
+              const uint32_t ka = smem_u32(smem + L::kOffK + st * L::kKV);
+              const int sb = static_cast<int>(ns & 1);
 #pragma unroll
-          for (int ks = 0; ks < D / 16; ++ks) {
-            const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
-            tc_mma_ss(tS + sb * 128, smem_desc(qa + off, 16, 1024, 2),
-                      smem_desc(ka + off, 16, 1024, 2), kIdescS, ks > 0 ? 1u : 0u);
+              for (int ks = 0; ks < D / 16; ++ks) {
+                const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
+                tc_mma_ss(tS + sb * 128, smem_desc(qa + off, 16, 1024, 2),
+                          smem_desc(ka + off, 16, 1024, 2), kIdescS, ks > 0 ? 1u : 0u);
+              }
+              tc_commit(&sfull[sb]);
+              tc_commit(&qempty[qb]);
+              if (s_last) tc_commit(&kempty[st]);
+              s_meta = false;
+              ++ns;
+              progress = true;
+            }
           }
-          tc_commit(&sfull[sb]);
-          tc_commit(&qempty[qb]);
-          return true;
-        };
-        ok = issue_s(0);
-        if (ok && n > 1) ok = issue_s(1);
-        for (long long i = 0; ok && i < n; ++i) {
-          const int sb = static_cast<int>(i & 1);
-          const int st = stage_of[i & 3];
-          const bool last = last_of_col[i & 3];
-          if (!(ok = mbar_wait(&pfull[sb], (i >> 1) & 1, abort_flag, p.err))) break;
-          if (!(ok = mbar_wait(&ofree[sb], ((i >> 1) & 1) ^ 1, abort_flag, p.err))) break;
-          tc_fence_after();
-          const uint32_t va = smem_u32(smem + L::kOffV + st * L::kKV);
+          // ---- PV(np)
+          if (np < ns) {
+            const int sb = static_cast<int>(np & 1);
+            const bool need_v = first_of_col[np & 3];
+            if ((!need_v || mbar_test(vfull, (uv + 1) & 1)) &&
+                mbar_test(&pfull[sb], (np >> 1) & 1) &&
+                mbar_test(&ofree[sb], ((np >> 1) & 1) ^ 1)) {
+              if (need_v) ++uv;
+              tc_fence_after();
+              const uint32_t va = smem_u32(smem + L::kOffV);
 #pragma unroll
-          for (int ks = 0; ks < 8; ++ks) {   // 128 keys in steps of 16 (8 packed columns)
-            const uint64_t bd = smem_desc(va + ks * 16 * 128, 16384, 1024, 2);
-            tc_mma_ts(tO + sb * D, tS + sb * 128 + ks * 8, bd, kIdescO, ks > 0 ? 1u : 0u);
+              for (int ks = 0; ks < 8; ++ks) {   // 128 keys in steps of 16 (8 packed columns)
+                const uint64_t bd = smem_desc(va + ks * 16 * 128, 16384, 1024, 2);
+                tc_mma_ts(tO + sb * D, tS + sb * 128 + ks * 8, bd, kIdescO, ks > 0 ? 1u : 0u);
+              }
+              tc_commit(&ofull[sb]);
+              if (last_of_col[np & 3]) tc_commit(vempty);
+              ++np;
+              progress = true;
+            }
           }
-          tc_commit(&ofull[sb]);
-          if (last) tc_commit(&kvempty[st]);
-          if (i + 2 < n && !(ok = issue_s(i + 2))) break;
+          if (progress) {
+            t_idle = 0;
+          } else if (*abort_flag) {
+            break;
+          } else if (t_idle == 0) {
+            t_idle = globaltimer();
+          } else if (globaltimer() - t_idle > kWaitLimitNs) {
+            atomicOr(p.err, kErrTimeout);
+            *abort_flag = 1;
+            break;
+          }
         }
+        (void)stage_of;
       }
       __syncwarp();
     }

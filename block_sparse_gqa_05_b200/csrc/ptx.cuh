@@ -63,6 +63,19 @@ MSA_DEV bool mbar_try_wait(uint64_t* bar, uint32_t phase) {
   return ok != 0;
 }
 
+// Non-blocking test of phase completion (parity).
+MSA_DEV bool mbar_test(uint64_t* bar, uint32_t phase) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(phase)
+      : "memory");
+  return ok != 0;
+}
+
 // Bounded wait for the completion of phase ``phase`` (parity).  Gives up after
 // kWaitLimitNs or as soon as *abort is set by another role of the CTA; on a
 // timeout it sets the device error word and *abort.  Returns false when the
