@@ -3,7 +3,7 @@
 // shared by all heads, score Q_idx . K_idx, block max-pooling).
 //
 // Prefill: persistent tcgen05 GEMM.  A = 128 (token, group) rows of q_idx,
-// B = one 128-key block of k_idx, D = 128 x 128 fp32 scores in TMEM.  The
+// B = two 128-key blocks of k_idx, D = 128 x 256 fp32 scores in TMEM.  The
 // epilogue masks keys past each row's position and reduces the 128 columns to
 // one pooled value, so token scores never leave the SM.
 // Decode (T*G < 128): a bandwidth-bound scan of k_idx with mma.sync.
@@ -15,8 +15,8 @@
 namespace msa {
 namespace {
 
-constexpr int kStages = 6;
-constexpr int kAcc = 4;          // TMEM accumulator buffers of 128 columns
+constexpr int kStages = 4;       // 256-key k_idx tiles in flight
+constexpr int kAcc = 2;          // TMEM accumulator buffers of 256 columns
 constexpr int kThreads = 320;    // warp 0: TMA, warp 1: MMA, warps 2..9: epilogue
 constexpr int kChunkBlocks = 32; // key blocks per work item
 
@@ -81,17 +81,18 @@ template <int DI>
 __global__ void __launch_bounds__(kThreads, 1)
     index_scores_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
                            const __grid_constant__ CUtensorMap tm_k, const IdxParams p) {
-  constexpr uint32_t kTile = 128u * DI * 2u;        // bytes of one 128-row operand tile
+  constexpr uint32_t kQTile = 128u * DI * 2u;       // 128 (token, group) rows
+  constexpr uint32_t kKTile = 256u * DI * 2u;       // 256 keys = two blocks
   constexpr uint32_t kLayout = DI == 64 ? 2u : 4u;  // 128-byte / 64-byte swizzle
   constexpr uint32_t kSbo = 8u * DI * 2u;           // 8-row swizzle atom
-  constexpr uint32_t kIdesc = idesc_bf16(128, 128, 0, 0);
+  constexpr uint32_t kIdesc = idesc_bf16(128, 256, 0, 0);
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint8_t* qbuf = smem;
-  uint8_t* kbuf = smem + 2 * kTile;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(kbuf + kStages * kTile);
+  uint8_t* kbuf = smem + 2 * kQTile;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(kbuf + kStages * kKTile);
   uint64_t* kfull = bars;
   uint64_t* kempty = bars + kStages;
   uint64_t* qfull = bars + 2 * kStages;
@@ -139,13 +140,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         item_decode(p, w, cur, seq, m, b0, b1);
         const int qb = static_cast<int>(q & 1);
         if (!(ok = mbar_wait(&qempty[qb], ((q >> 1) & 1) ^ 1, abort_flag, p.err))) break;
-        mbar_arrive_expect_tx(&qfull[qb], kTile);
-        tma_load_2d(qbuf + qb * kTile, &tm_q, &qfull[qb], 0, seq * p.T * p.G + m * 128);
-        for (int b = b0; b < b1; ++b, ++j) {
+        mbar_arrive_expect_tx(&qfull[qb], kQTile);
+        tma_load_2d(qbuf + qb * kQTile, &tm_q, &qfull[qb], 0, seq * p.T * p.G + m * 128);
+        for (int b = b0; b < b1; b += 2, ++j) {
           const int s = static_cast<int>(j % kStages);
           if (!(ok = mbar_wait(&kempty[s], ((j / kStages) & 1) ^ 1, abort_flag, p.err))) break;
-          mbar_arrive_expect_tx(&kfull[s], kTile);
-          tma_load_2d(kbuf + s * kTile, &tm_k, &kfull[s], 0, seq * p.N + b * 128);
+          mbar_arrive_expect_tx(&kfull[s], kKTile);
+          tma_load_2d(kbuf + s * kKTile, &tm_k, &kfull[s], 0, seq * p.N + b * 128);
         }
       }
     }
@@ -154,26 +155,26 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------- MMA issuer
     if (lane == 0) {
       ItemCursor cur;
-      long long j = 0, i = 0, q = 0;
+      long long j = 0, q = 0;
       bool ok = true;
       for (long long w = blockIdx.x; ok && w < p.items_total; w += gridDim.x, ++q) {
         int seq, m, b0, b1;
         item_decode(p, w, cur, seq, m, b0, b1);
         const int qb = static_cast<int>(q & 1);
         if (!(ok = mbar_wait(&qfull[qb], (q >> 1) & 1, abort_flag, p.err))) break;
-        const uint32_t qaddr = smem_u32(qbuf + qb * kTile);
-        for (int b = b0; b < b1; ++b, ++j, ++i) {
+        const uint32_t qaddr = smem_u32(qbuf + qb * kQTile);
+        for (int b = b0; b < b1; b += 2, ++j) {
           const int s = static_cast<int>(j % kStages);
-          const int a = static_cast<int>(i % kAcc);
+          const int a = static_cast<int>(j % kAcc);
           if (!(ok = mbar_wait(&kfull[s], (j / kStages) & 1, abort_flag, p.err))) break;
-          if (!(ok = mbar_wait(&accempty[a], ((i / kAcc) & 1) ^ 1, abort_flag, p.err))) break;
+          if (!(ok = mbar_wait(&accempty[a], ((j / kAcc) & 1) ^ 1, abort_flag, p.err))) break;
           tc_fence_after();
-          const uint32_t kaddr = smem_u32(kbuf + s * kTile);
+          const uint32_t kaddr = smem_u32(kbuf + s * kKTile);
 #pragma unroll
           for (int ks = 0; ks < DI / 16; ++ks) {
             const uint64_t ad = smem_desc(qaddr + ks * 32, 16, kSbo, kLayout);
             const uint64_t bd = smem_desc(kaddr + ks * 32, 16, kSbo, kLayout);
-            tc_mma_ss(tmem + a * 128, ad, bd, kIdesc, ks > 0 ? 1u : 0u);
+            tc_mma_ss(tmem + a * 256, ad, bd, kIdesc, ks > 0 ? 1u : 0u);
           }
           tc_commit(&kempty[s]);
           tc_commit(&accfull[a]);
@@ -184,12 +185,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncwarp();
   } else {
     // --------------------------------------------- epilogue: mask + block max
-    const int wg = (warp - 2) >> 2;          // which accumulator buffers (parity)
+    // Warpgroup wg owns accumulator wg and takes every other 256-key tile;
+    // each tile holds two key blocks.
+    const int wg = (warp - 2) >> 2;
     const int quarter = warp & 3;            // TMEM lanes 32*quarter .. +31
     const int row = quarter * 32 + lane;
-    const uint32_t taddr_row = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
+    const uint32_t taddr_row = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + wg * 256;
     ItemCursor cur;
-    long long i = 0;
+    long long j = 0;
     bool ok = true;
     const int rows_per_seq = p.T * p.G;
     for (long long w = blockIdx.x; ok && w < p.items_total; w += gridDim.x) {
@@ -202,35 +205,41 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int bt = pos >> 7;
       float* out = p.pooled + (static_cast<long long>(seq) * rows_per_seq + trow) *
                                   static_cast<long long>(p.nb);
-      for (int b = b0; b < b1; ++b, ++i) {
-        if ((i & 1) != wg) continue;
-        const int a = static_cast<int>(i % kAcc);
-        if (!(ok = mbar_wait(&accfull[a], (i / kAcc) & 1, abort_flag, p.err))) break;
+      for (int b = b0; b < b1; b += 2, ++j) {
+        if ((j & 1) != wg) continue;
+        if (!(ok = mbar_wait(&accfull[wg], (j >> 1) & 1, abort_flag, p.err))) break;
         tc_fence_after();
-        float v[128];
 #pragma unroll
-        for (int c = 0; c < 4; ++c) tmem_ld32(taddr_row + a * 128 + c * 32, v + c * 32);
-        tc_wait_ld();
-        tc_fence_before();
-        mbar_arrive(&accempty[a]);
-        if (valid && b <= bt) {
-          const int lim = (b == bt) ? (pos & 127) : 127;
-          float mx = -INFINITY;
-          if (lim == 127) {
-            float m4[4] = {v[0], v[1], v[2], v[3]};
+        for (int h = 0; h < 2; ++h) {
+          float v[128];
 #pragma unroll
-            for (int c = 4; c < 128; c += 4) {
-              m4[0] = fmaxf(m4[0], v[c]);
-              m4[1] = fmaxf(m4[1], v[c + 1]);
-              m4[2] = fmaxf(m4[2], v[c + 2]);
-              m4[3] = fmaxf(m4[3], v[c + 3]);
-            }
-            mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
-          } else {
-#pragma unroll
-            for (int c = 0; c < 128; ++c) mx = fmaxf(mx, c <= lim ? v[c] : -INFINITY);
+          for (int c = 0; c < 4; ++c) tmem_ld32(taddr_row + h * 128 + c * 32, v + c * 32);
+          tc_wait_ld();
+          if (h == 1) {
+            tc_fence_before();
+            mbar_arrive(&accempty[wg]);
           }
-          out[b] = mx;
+          const int bb = b + h;
+          if (valid && bb < b1 && bb <= bt) {
+            const int lim = (bb == bt) ? (pos & 127) : 127;
+            float mx;
+            if (lim == 127) {
+              float m4[4] = {v[0], v[1], v[2], v[3]};
+#pragma unroll
+              for (int c = 4; c < 128; c += 4) {
+                m4[0] = fmaxf(m4[0], v[c]);
+                m4[1] = fmaxf(m4[1], v[c + 1]);
+                m4[2] = fmaxf(m4[2], v[c + 2]);
+                m4[3] = fmaxf(m4[3], v[c + 3]);
+              }
+              mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
+            } else {
+              mx = -INFINITY;
+#pragma unroll
+              for (int c = 0; c < 128; ++c) mx = fmaxf(mx, c <= lim ? v[c] : -INFINITY);
+            }
+            out[bb] = mx;
+          }
         }
       }
     }
@@ -387,13 +396,14 @@ cudaError_t launch_tc(const msa_shape& s, const uint16_t* q_idx, const uint16_t*
   const uint64_t dk[2] = {static_cast<uint64_t>(DI), static_cast<uint64_t>(s.batch) * s.seq_kv};
   const uint64_t stride[1] = {static_cast<uint64_t>(DI) * 2};
   const uint32_t box[2] = {static_cast<uint32_t>(DI), 128};
+  const uint32_t kbox[2] = {static_cast<uint32_t>(DI), 256};
   const CUtensorMapSwizzle sw =
       DI == 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
   if (!encode_tmap(&tq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, q_idx, dq, stride, box, sw) ||
-      !encode_tmap(&tk, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, k_idx, dk, stride, box, sw))
+      !encode_tmap(&tk, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, k_idx, dk, stride, kbox, sw))
     return cudaErrorInvalidValue;
 
-  const size_t smem = 1024 + (2 + kStages) * 128 * DI * 2 + 256;
+  const size_t smem = 1024 + (2 * 128 + kStages * 256) * DI * 2 + 256;
   cudaError_t e = cudaFuncSetAttribute(index_scores_tc_kernel<DI>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
@@ -415,7 +425,9 @@ cudaError_t launch_index_scores(const msa_shape& s, const uint16_t* q_idx, const
   const int nb = static_cast<int>(ceil_div(s.seq_kv, 128));
   const long long rows = static_cast<long long>(s.batch) * s.seq_q * s.n_kv_heads;
   cudaError_t e;
-  if (static_cast<long long>(s.seq_q) * s.n_kv_heads < 128) {
+  // the tensor-core path needs a full 128-row query tile and a 256-key box
+  if (static_cast<long long>(s.seq_q) * s.n_kv_heads < 128 ||
+      static_cast<long long>(s.batch) * s.seq_kv < 256) {
     const int last_bt = (s.q_offset + s.seq_q - 1) / 128;
     dim3 grid(static_cast<unsigned>(ceil_div(last_bt + 1, 8)),
               static_cast<unsigned>(s.batch * s.seq_q));
