@@ -288,6 +288,9 @@ def run_msa(args, world, rank, pg):
     del inp, ws, o, sel
     torch.cuda.empty_cache()
 
+    # ---- isolated top-k over 1024 block scores per (query, group), against torch.topk
+    if not args.skip_topk_micro and world == 1:
+        out["topk_microbench"] = run_topk_micro(M, args, stream, peaks)
     # ---- decode at 128K, batch 32
     if not args.skip_decode:
         dw = synth.workload(args.decode_workload)
@@ -297,6 +300,30 @@ def run_msa(args, world, rank, pg):
     if not args.skip_long:
         out["ctx_1m"] = run_long(M, args, pg, stream, world, rank, peaks)
     return out, sp
+
+
+def run_topk_micro(M, args, stream, peaks):
+    """131072 queries x 8 groups x 1024 pooled block scores (every query at
+    position 131071 of a 131072-key context, so all 1024 blocks are
+    candidates): msa_block_topk (top-15 + the local block) vs
+    torch.topk(pooled, 16, dim=-1) on the same tensor."""
+    q, G, nb = 131072, 8, 1024
+    sh = M.Shape(batch=q, seq_q=1, seq_kv=nb * 128, q_offset=nb * 128 - 1, n_q_heads=64,
+                 n_kv_heads=G, head_dim=128, index_dim=64, block=128, topk=16)
+    gen = torch.Generator(device="cuda").manual_seed(33)
+    pooled = torch.round(torch.randn((q, 1, G, nb), device="cuda", generator=gen) * 30.0)
+    sel = torch.empty((q, 1, G, 16), dtype=torch.int32, device="cuda")
+    ms = timed_loop(lambda: M.block_topk(sh, pooled, sel), max(args.steps, 5), 3, None, stream)
+    tms = timed_loop(lambda: torch.topk(pooled, 16, dim=-1), max(args.steps, 5), 3, None, stream)
+    byts = float(pooled.numel() * 4 + sel.numel() * 4)
+    a = byts / (ms / 1e3) / 1e9
+    res = {"rows": q * G, "candidates_per_row": nb, "msa_block_topk_ms": round(ms, 4),
+           "torch_topk_ms": round(tms, 4), "speedup_vs_torch_topk": round(tms / ms, 2),
+           "achieved_gbs": round(a, 1), "frac_of_hbm": round(a / peaks["hbm_gbs"], 4),
+           "values": "round(30 * N(0,1)) (integer-valued, many ties)"}
+    del pooled, sel
+    torch.cuda.empty_cache()
+    return res
 
 
 def run_decode(M, sp, args, pg, stream, world, peaks, dense):
@@ -495,6 +522,7 @@ def main():
     ap.add_argument("--skip-decode", action="store_true")
     ap.add_argument("--skip-cpu", action="store_true")
     ap.add_argument("--skip-e2e", action="store_true")
+    ap.add_argument("--skip-topk-micro", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--ref-step-s", type=float, default=4.0)
     args = ap.parse_args()
@@ -522,7 +550,7 @@ def main():
                 "gpu_launches": res["gpu_launches"], "roofline": res["roofline"],
                 "stages": res["stages"], "kernels_ms_per_launch": res["kernels_ms_per_launch"],
                 "clocks": res["clocks"]}
-        for key in ("e2e", "decode", "ctx_1m"):
+        for key in ("e2e", "topk_microbench", "decode", "ctx_1m"):
             if key in res:
                 line[key] = res[key]
         if world == 1 and not args.skip_cpu:

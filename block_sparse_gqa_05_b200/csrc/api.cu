@@ -45,11 +45,14 @@ msa_status check_shape(const msa_shape* s, bool need_attn, bool need_index) {
   if (s->n_q_heads % s->n_kv_heads != 0) return MSA_ERR_INVALID_SHAPE;
   if (!is_pow2_upto(s->n_kv_heads, 128)) return MSA_ERR_UNSUPPORTED;   // G divides 128
   if (!is_pow2_upto(s->n_q_heads / s->n_kv_heads, 16)) return MSA_ERR_UNSUPPORTED;
-  // 32-bit coordinates / packed (token, slot) entries
+  // 32-bit row indices, TMA coordinates and packed (token, slot) entries
   if (s->seq_q >= (1 << 25)) return MSA_ERR_UNSUPPORTED;
-  if (static_cast<int64_t>(s->batch) * s->seq_q * s->n_q_heads >= (1ll << 31) ||
-      static_cast<int64_t>(s->batch) * s->n_kv_heads * s->seq_kv >= (1ll << 31) ||
-      static_cast<int64_t>(s->batch) * s->seq_kv >= (1ll << 31))
+  if (static_cast<int64_t>(s->batch) * s->seq_q * s->n_kv_heads >= (1ll << 31))
+    return MSA_ERR_UNSUPPORTED;
+  if (need_attn && (static_cast<int64_t>(s->batch) * s->seq_q * s->n_q_heads >= (1ll << 31) ||
+                    static_cast<int64_t>(s->batch) * s->n_kv_heads * s->seq_kv >= (1ll << 31)))
+    return MSA_ERR_UNSUPPORTED;
+  if (need_index && static_cast<int64_t>(s->batch) * s->seq_kv >= (1ll << 31))
     return MSA_ERR_UNSUPPORTED;
   if (need_attn && s->head_dim != 64 && s->head_dim != 128) return MSA_ERR_UNSUPPORTED;
   if (need_index && s->index_dim != 32 && s->index_dim != 64) return MSA_ERR_UNSUPPORTED;

@@ -128,7 +128,9 @@ __global__ void __launch_bounds__(kWarps * 32, 3)
   const long long nwarps = static_cast<long long>(gridDim.x) * kWarps;
   const bool vec = (nb & 3) == 0;
   for (long long r = static_cast<long long>(blockIdx.x) * kWarps + warp; r < rows; r += nwarps) {
-    const int t = static_cast<int>((r / G) % T);
+    // rows < 2^31 (checked by the API): 32-bit index math
+    const int t = static_cast<int>((static_cast<uint32_t>(r) / static_cast<uint32_t>(G)) %
+                                   static_cast<uint32_t>(T));
     const int bt = (q_off + t) >> 7;
     const int n = bt;                         // candidates 0 .. bt-1
     const int kk = min(k - 1, n);

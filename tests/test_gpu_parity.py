@@ -139,6 +139,19 @@ def test_sparse_prefill_ragged(sp):
         assert np.abs(lse[b].double().cpu().numpy() - L_ref).max() < LSE_ABS
 
 
+def test_sparse_prefill_spans_token_chunks():
+    # more than one 8192-token chunk of the prefill work decomposition, ragged end
+    sp = spec(1, 9000, 9100, 100, 8, 2, 64, 32, 6, seed=14, planted=2)
+    inp = inputs_cpu(sp)
+    sel_ref = oracle_sel(sp, oracle_pooled(sp, inp, 0))
+    sel = cuda(torch.from_numpy(sel_ref)[None])
+    o, lse = M.sparse_attn_prefill(M.Shape.of(sp), cuda(inp.q), cuda(inp.k), cuda(inp.v), sel)
+    torch.cuda.synchronize()
+    O_ref, L_ref = oracle_attention(sp, inp, sel_ref, 0)
+    check_attn(o[0], O_ref, "multi-chunk prefill")
+    assert np.abs(lse[0].double().cpu().numpy() - L_ref).max() < LSE_ABS
+
+
 @pytest.mark.parametrize("sp", [spec(3, 1, 3000, 2999, 16, 2, 128, 64, 4, seed=21),
                                 spec(2, 1, 5000, 4999, 8, 2, 64, 32, 16, seed=22),
                                 spec(2, 1, 129, 128, 16, 1, 128, 64, 16, seed=23)])
@@ -163,6 +176,33 @@ def test_dense_decode():
         O_ref, L_ref = O.dense_attention(inp.q[b], inp.k[b], inp.v[b], positions(sp))
         check_attn(o[b], O_ref, f"dense decode b={b}")
         assert np.abs(lse[b].double().cpu().numpy() - L_ref).max() < LSE_ABS
+
+
+@pytest.mark.parametrize("sp", [spec(1, 1000, 1000, 0, 8, 2, 64, 32, 4, seed=32),
+                                spec(2, 300, 1000, 700, 16, 2, 128, 64, 4, seed=33),
+                                spec(1, 130, 5000, 4870, 16, 8, 128, 64, 4, seed=34)])
+def test_dense_prefill(sp):
+    inp = inputs_cpu(sp)
+    o, lse = M.dense_attn_prefill(M.Shape.of(sp), cuda(inp.q), cuda(inp.k), cuda(inp.v))
+    torch.cuda.synchronize()
+    for b in range(sp.batch):
+        O_ref, L_ref = O.dense_attention(inp.q[b], inp.k[b], inp.v[b], positions(sp))
+        check_attn(o[b], O_ref, f"dense prefill b={b}")
+        assert np.abs(lse[b].double().cpu().numpy() - L_ref).max() < LSE_ABS
+
+
+def test_dense_prefill_growing_logits_rescale():
+    # key norms grow along the sequence, so row maxima keep rising block after
+    # block and the accumulated output has to be rescaled
+    sp = spec(1, 256, 2048, 1792, 8, 1, 64, 32, 4, seed=35)
+    inp = inputs_cpu(sp)
+    ramp = torch.linspace(0.2, 6.0, sp.seq_kv).view(1, 1, -1, 1)
+    k = (inp.k.float() * ramp).to(torch.bfloat16)
+    o, lse = M.dense_attn_prefill(M.Shape.of(sp), cuda(inp.q), cuda(k), cuda(inp.v))
+    torch.cuda.synchronize()
+    O_ref, L_ref = O.dense_attention(inp.q[0], k[0], inp.v[0], positions(sp))
+    check_attn(o[0], O_ref, "dense prefill with rescales")
+    assert np.abs(lse[0].double().cpu().numpy() - L_ref).max() < LSE_ABS
 
 
 # ------------------------------------------------------------- whole layer
