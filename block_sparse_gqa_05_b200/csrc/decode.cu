@@ -2,15 +2,20 @@
 // yhxrc.cn article, section 第二步; lumi-systems AI news: exact block-sparse
 // attention over the selected blocks) and dense causal GQA (the baseline).
 //
-// Split-K: one CTA per (sequence, group, split), a split being one selected
-// block (sparse) or a run of consecutive causal blocks (dense).  The K and V
-// rows of a block are brought into shared memory once by TMA (128-byte
-// swizzle) and shared by all r = H/G query heads of the group: the heads are
-// the 16 rows of an mma.sync m16n8k16 tile (zero-padded when r < 16).  Each
-// warp owns 16 keys of the block and keeps its own online softmax; warps are
-// merged in shared memory, splits in a last-arriving CTA chosen by an atomic
-// counter (no CTA ever waits for another).  The workload is bound by HBM
-// bandwidth on the K/V bytes.
+// Work items are (sequence, group, block) visits: the k selected blocks of a
+// (sequence, group) for sparse decode, all of its causal blocks for dense
+// decode.  A persistent grid of one CTA per SM takes a contiguous range of
+// items; one TMA warp streams the K and V tiles of its blocks (128-byte
+// swizzle) through a ring of stages while eight consumer warps compute.
+// The heads of a group are the 16 rows of mma.sync m16n8k16 tiles
+// (zero-padded when r < 16): for Q K^T each warp owns 16 keys of the block,
+// the row maxima and sums are exchanged through shared memory, P is staged
+// there in bf16, and for P V each warp owns D/8 output columns, so no
+// per-warp state has to be merged at the end.  A (sequence, group) whose
+// items all fall in one CTA is written directly; one that spans CTAs leaves
+// a normalised partial per CTA, merged by the last CTA to finish it (chosen
+// by an atomic counter: no CTA ever waits for another).  The kernel is bound
+// by HBM bandwidth on the K/V bytes.
 #include <math.h>
 
 #include <mutex>
@@ -21,8 +26,11 @@
 namespace msa {
 namespace {
 
-constexpr int kThreads = 256;          // 8 warps x 16 keys = one 128-key block
-constexpr int kDenseBlocksPerSplit = 16;
+constexpr int kConsumerWarps = 8;
+constexpr int kThreads = (kConsumerWarps + 1) * 32;   // 8 consumer warps + 1 TMA warp
+constexpr int kConsumerThreads = kConsumerWarps * 32;
+constexpr int kMaxGrid = 256;
+constexpr int kPStride = 136;    // bf16 per row of the P tile: rows 272 B apart, no bank conflicts
 constexpr float kLog2e = 1.4426950408889634f;
 
 struct DecParams {
@@ -30,12 +38,25 @@ struct DecParams {
   const int32_t* sel;     // [B, 1, G, k] (sparse) or nullptr (dense)
   uint16_t* o;            // [B, 1, H, d]
   float* lse;             // [B, 1, H] or nullptr
-  uint32_t* counters;     // [B*G]
-  float* part_lse;        // [B*G, nsplit, r]   (log2 units)
-  float* part_o;          // [B*G, nsplit, r, d] normalised partial outputs
+  uint32_t* counters;     // [B*G] CTAs done with a (sequence, group)
+  float* part_lse;        // [2*grid, r]   (log2 units)
+  float* part_o;          // [2*grid, r, d] normalised partial outputs
   uint32_t* err;
-  int N, H, G, r, k, nsplit, bps;   // bps: blocks per split (dense)
+  long long n_items;      // B*G*per_bg
+  int per_bg;             // items of one (sequence, group): k, or the causal blocks
+  int N, H, G, r, k;
   float scale_log2;
+};
+
+template <int D>
+struct DecLayout {
+  static constexpr uint32_t kTile = 128u * D * 2u;             // K (or V) of one block
+  static constexpr int kStages = D == 128 ? 3 : 6;
+  static constexpr uint32_t kOffP = kStages * 2u * kTile;      // P [16][kPStride] bf16
+  static constexpr uint32_t kOffRed = kOffP + 16u * kPStride * 2u;   // wmax, wsum [8][16]
+  static constexpr uint32_t kOffBar = kOffRed + 2u * 8u * 16u * 4u;
+  static constexpr uint32_t kOffFlag = kOffBar + 3u * kStages * 8u;  // abort, last
+  static constexpr uint32_t kBytes = kOffFlag + 16u;
 };
 
 __device__ __forceinline__ void mma16816(float* d, const uint32_t* a, const uint32_t* b) {
@@ -51,9 +72,21 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t* r) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+
 __device__ __forceinline__ void ldsm_x4_trans(uint32_t addr, uint32_t* r) {
   asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
                : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+
+__device__ __forceinline__ void ldsm_x2_trans(uint32_t addr, uint32_t* r) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x2.trans.shared.b16 {%0,%1}, [%2];"
+               : "=r"(r[0]), "=r"(r[1])
                : "r"(addr));
 }
 
@@ -66,255 +99,372 @@ __device__ __forceinline__ uint32_t sw128_off(int row, int col) {
   return static_cast<uint32_t>(chunk * (128 * 128) + row * 128 + unit * 16 + (c & 7) * 2);
 }
 
+// Block of item i (-1 when it has nothing to attend to: an empty selection
+// slot or a block past the query), and its (sequence, group) in *bg.
+__device__ __forceinline__ int item_block(const DecParams& p, long long i, int bt, int* bg) {
+  const int g = static_cast<int>(i / p.per_bg);
+  const int j = static_cast<int>(i - static_cast<long long>(g) * p.per_bg);
+  *bg = g;
+  const int blk = p.sel ? __ldg(p.sel + static_cast<long long>(g) * p.k + j) : j;
+  return (blk >= 0 && blk <= bt) ? blk : -1;
+}
+
+// First item of CTA c, and the CTA holding item i (ranges split evenly).
+__device__ __forceinline__ long long cta_first(long long c, long long n, long long grid) {
+  return c * n / grid;
+}
+__device__ __forceinline__ int cta_of(long long i, long long n, long long grid) {
+  return static_cast<int>(((i + 1) * grid + n - 1) / n - 1);
+}
+
 template <int D>
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kThreads, 1)
     decode_attn_kernel(const __grid_constant__ CUtensorMap tm_k,
                        const __grid_constant__ CUtensorMap tm_v, const DecParams p) {
-  constexpr int KS = D / 16;              // k-steps of the QK^T product
-  constexpr int NT = D / 8;               // n8 tiles of the PV product
-  constexpr uint32_t kTile = 128u * D * 2u;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  uint8_t* ks_ = smem;
-  uint8_t* vs_ = smem + kTile;
-  uint64_t* bar = reinterpret_cast<uint64_t*>(smem + 2 * kTile);
-  float* red = reinterpret_cast<float*>(smem);   // reused after the last block
-  __shared__ float wm[8][16], wl[8][16];
-  __shared__ int s_last;
-  __shared__ int s_abort;
+  using L = DecLayout<D>;
+  constexpr int S = L::kStages;
+  constexpr int KS = D / 16;          // k-steps of Q K^T
+  constexpr int NW = D / 64;          // n8 tiles of P V per warp (D/8 columns)
+  extern __shared__ __align__(1024) uint8_t smem[];
+  uint16_t* ps = reinterpret_cast<uint16_t*>(smem + L::kOffP);
+  float* wmax = reinterpret_cast<float*>(smem + L::kOffRed);
+  float* wsum = wmax + 8 * 16;
+  uint64_t* kfull = reinterpret_cast<uint64_t*>(smem + L::kOffBar);
+  uint64_t* vfull = kfull + S;
+  uint64_t* empty = vfull + S;
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kOffFlag);
+  volatile int* s_last = abort_flag + 1;
 
-  const int split = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int gq = lane >> 2, qd = lane & 3;
+  const long long n = p.n_items, grid = gridDim.x;
+  const long long i0 = cta_first(blockIdx.x, n, grid);
+  const long long i1 = cta_first(blockIdx.x + 1, n, grid);
   const int pos = p.N - 1;
   const int bt = pos >> 7;
-  const int bg = b * p.G + g;
 
-  // blocks of this split
-  int blk_begin, blk_end;
-  if (p.sel) {
-    const int sb = p.sel[static_cast<long long>(bg) * p.k + split];
-    blk_begin = sb;
-    blk_end = (sb >= 0 && sb <= bt) ? sb + 1 : sb;   // empty when sb < 0
-    if (sb < 0) blk_begin = blk_end = 0;
-  } else {
-    blk_begin = split * p.bps;
-    blk_end = min(blk_begin + p.bps, bt + 1);
+  // the swizzled K/V tiles need 1024-byte alignment; the launch reserves no slack
+  if ((smem_u32(smem) & 1023u) != 0u) {
+    if (threadIdx.x == 0) atomicOr(p.err, kErrTimeout);
+    return;
   }
-
   if (threadIdx.x == 0) {
-    mbar_init(bar, 1);
-    s_abort = 0;
+    for (int s = 0; s < S; ++s) {
+      mbar_init(&kfull[s], 1);
+      mbar_init(&vfull[s], 1);
+      mbar_init(&empty[s], kConsumerWarps);
+    }
+    *abort_flag = 0;
     fence_barrier_init();
   }
   __syncthreads();
 
-  // query fragments: rows = heads g*r + i (i < r), zero rows above r
+  if (warp == kConsumerWarps) {
+    // ------------------------------------------------------------ TMA warp
+    if (lane == 0) {
+      tma_prefetch_desc(&tm_k);
+      tma_prefetch_desc(&tm_v);
+    }
+    int cnt = 0;
+    bool ok = true;
+    for (long long base = i0; ok && base < i1; base += 32) {
+      int bgv = 0;
+      const int blk = base + lane < i1 ? item_block(p, base + lane, bt, &bgv) : -1;
+      unsigned m = __ballot_sync(0xffffffffu, blk >= 0);
+      while (m) {
+        const int src = __ffs(m) - 1;
+        m &= m - 1;
+        const int b_ = __shfl_sync(0xffffffffu, blk, src);
+        const int bg_ = __shfl_sync(0xffffffffu, bgv, src);
+        const int s = cnt % S;
+        if (lane == 0) {
+          ok = mbar_wait(&empty[s], ((cnt / S) & 1) ^ 1, abort_flag, p.err);
+          if (ok) {
+            mbar_arrive_expect_tx(&kfull[s], L::kTile);
+#pragma unroll
+            for (int c = 0; c < D / 64; ++c)
+              tma_load_3d(smem + s * 2 * L::kTile + c * 16384, &tm_k, &kfull[s], c * 64, b_ * 128,
+                          bg_);
+            mbar_arrive_expect_tx(&vfull[s], L::kTile);
+#pragma unroll
+            for (int c = 0; c < D / 64; ++c)
+              tma_load_3d(smem + s * 2 * L::kTile + L::kTile + c * 16384, &tm_v, &vfull[s],
+                          c * 64, b_ * 128, bg_);
+          }
+        }
+        ok = __shfl_sync(0xffffffffu, ok, 0) != 0;
+        if (!ok) break;
+        ++cnt;
+      }
+    }
+    // Every load this warp issued lands before the CTA may exit.
+    if (lane == 0) {
+      for (int x = max(0, cnt - S); x < cnt; ++x) {
+        const int s = x % S;
+        const uint32_t ph = (x / S) & 1;
+        const uint64_t t0 = globaltimer();
+        while (!(mbar_test(&kfull[s], ph) && mbar_test(&vfull[s], ph)))
+          if (globaltimer() - t0 > kWaitLimitNs) {
+            atomicOr(p.err, kErrTimeout);
+            break;
+          }
+      }
+    }
+    return;
+  }
+
+  // ---------------------------------------------------------- consumer warps
+  const int w = warp;
+  const int gq = lane >> 2, qd = lane & 3;
+  const uint32_t pbase = smem_u32(ps);
+  int cnt = 0;
+  int cur_bg = -1;
+  long long seg_first = 0;
+  bool failed = false;
   uint32_t qa[KS][4];
-  {
-    const uint16_t* qb = p.q + (static_cast<long long>(b) * p.H + g * p.r) * D;
-#pragma unroll
-    for (int ks = 0; ks < KS; ++ks) {
-      const int c0 = ks * 16 + 2 * qd;
-      qa[ks][0] = gq < p.r ? *reinterpret_cast<const uint32_t*>(qb + gq * D + c0) : 0u;
-      qa[ks][1] = gq + 8 < p.r ? *reinterpret_cast<const uint32_t*>(qb + (gq + 8) * D + c0) : 0u;
-      qa[ks][2] = gq < p.r ? *reinterpret_cast<const uint32_t*>(qb + gq * D + c0 + 8) : 0u;
-      qa[ks][3] =
-          gq + 8 < p.r ? *reinterpret_cast<const uint32_t*>(qb + (gq + 8) * D + c0 + 8) : 0u;
-    }
-  }
+  float m_run[2], l_run[2];
+  float o_acc[NW][4];
 
-  float m_run[2] = {-INFINITY, -INFINITY};   // rows gq, gq+8 (log2 domain)
-  float l_run[2] = {0.f, 0.f};
-  float o_acc[NT][4];
-#pragma unroll
-  for (int nt = 0; nt < NT; ++nt) o_acc[nt][0] = o_acc[nt][1] = o_acc[nt][2] = o_acc[nt][3] = 0.f;
-
-  uint32_t phase = 0;
-  bool ok = true;
-  for (int blk = blk_begin; blk < blk_end && ok; ++blk, phase ^= 1u) {
-    if (threadIdx.x == 0) {
-      mbar_arrive_expect_tx(bar, 2 * kTile);
-#pragma unroll
-      for (int c = 0; c < D / 64; ++c) {
-        tma_load_3d(ks_ + c * 128 * 128, &tm_k, bar, c * 64, blk * 128, bg);
-        tma_load_3d(vs_ + c * 128 * 128, &tm_v, bar, c * 64, blk * 128, bg);
-      }
-    }
-    if (!mbar_wait(bar, phase, &s_abort, p.err)) ok = false;
-    __syncthreads();
-    if (!ok || s_abort) { ok = false; break; }
-    // ---- S = Q K^T for keys kw*16 .. +15 of this block
-    const uint32_t kbase = smem_u32(ks_);
-    float s[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-#pragma unroll
-    for (int nt = 0; nt < 2; ++nt) {
-      const int key = warp * 16 + nt * 8 + gq;
-#pragma unroll
-      for (int ks = 0; ks < KS; ++ks) {
-        uint32_t bb[2];
-        const int col = ks * 16 + 2 * qd;
-        asm volatile("ld.shared.b32 %0, [%1];" : "=r"(bb[0]) : "r"(kbase + sw128_off(key, col)));
-        asm volatile("ld.shared.b32 %0, [%1];"
-                     : "=r"(bb[1])
-                     : "r"(kbase + sw128_off(key, col + 8)));
-        mma16816(s[nt], qa[ks], bb);
-      }
-    }
-    // ---- mask, online softmax (per warp, rows gq / gq+8)
-    float mx[2] = {-INFINITY, -INFINITY};
-#pragma unroll
-    for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int key = blk * 128 + warp * 16 + nt * 8 + 2 * qd + (e & 1);
-        s[nt][e] = key <= pos ? s[nt][e] * p.scale_log2 : -INFINITY;
-        mx[e >> 1] = fmaxf(mx[e >> 1], s[nt][e]);
-      }
+  // Write the (sequence, group) just finished: directly when this CTA holds
+  // all of its items, else as a partial, merged by the last CTA to finish it.
+  auto finish = [&](int bg, long long first, long long end) {
+    const int b = bg / p.G, g = bg % p.G;
+    const int r = p.r;
+    float inv[2], lse2[2];
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
-      mx[h] = fmaxf(mx[h], __shfl_xor_sync(0xffffffffu, mx[h], 1));
-      mx[h] = fmaxf(mx[h], __shfl_xor_sync(0xffffffffu, mx[h], 2));
+      inv[h] = l_run[h] > 0.f ? 1.f / l_run[h] : 0.f;
+      lse2[h] = l_run[h] > 0.f ? m_run[h] + log2f(l_run[h]) : -INFINITY;
     }
-    float corr[2], mnew[2];
+    const long long bfirst = static_cast<long long>(bg) * p.per_bg;
+    if (first == bfirst && end == bfirst + p.per_bg) {
 #pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      mnew[h] = fmaxf(m_run[h], mx[h]);
-      corr[h] = mnew[h] == -INFINITY ? 1.f : exp2f(m_run[h] - mnew[h]);
-      m_run[h] = mnew[h];
-    }
-    float rs[2] = {0.f, 0.f};
+      for (int h = 0; h < 2; ++h) {
+        const int row = gq + 8 * h;
+        if (row >= r) continue;
+        uint16_t* orow = p.o + (static_cast<long long>(b) * p.H + g * r + row) * D;
 #pragma unroll
-    for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const float mh = mnew[e >> 1];
-        const float pv = mh == -INFINITY ? 0.f : exp2f(s[nt][e] - mh);
-        s[nt][e] = pv;
-        rs[e >> 1] += pv;
+        for (int nt = 0; nt < NW; ++nt) {
+          const int col = w * (D / 8) + nt * 8 + 2 * qd;
+          *reinterpret_cast<uint32_t*>(orow + col) =
+              pack_bf16(o_acc[nt][2 * h] * inv[h], o_acc[nt][2 * h + 1] * inv[h]);
+        }
+        if (p.lse && w == 0 && qd == 0)
+          p.lse[static_cast<long long>(b) * p.H + g * r + row] = lse2[h] / kLog2e;
       }
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      rs[h] += __shfl_xor_sync(0xffffffffu, rs[h], 1);
-      rs[h] += __shfl_xor_sync(0xffffffffu, rs[h], 2);
-      l_run[h] = l_run[h] * corr[h] + rs[h];
+      return;
     }
-#pragma unroll
-    for (int nt = 0; nt < NT; ++nt) {
-      o_acc[nt][0] *= corr[0];
-      o_acc[nt][1] *= corr[0];
-      o_acc[nt][2] *= corr[1];
-      o_acc[nt][3] *= corr[1];
-    }
-    // ---- O += P V  (A = P as bf16 from the S accumulators, B = V via ldmatrix.trans)
-    uint32_t pa[4];
-    pa[0] = pack_bf16(s[0][0], s[0][1]);
-    pa[1] = pack_bf16(s[0][2], s[0][3]);
-    pa[2] = pack_bf16(s[1][0], s[1][1]);
-    pa[3] = pack_bf16(s[1][2], s[1][3]);
-    const uint32_t vbase = smem_u32(vs_);
-    const int mi = lane >> 3, ri = lane & 7;
-    const int vkey = warp * 16 + (mi & 1) * 8 + ri;
-#pragma unroll
-    for (int nt = 0; nt < NT; nt += 2) {
-      const int dcol = nt * 8 + (mi >> 1) * 8;
-      uint32_t vb[4];
-      ldsm_x4_trans(vbase + sw128_off(vkey, dcol), vb);
-      mma16816(o_acc[nt], pa, vb);
-      mma16816(o_acc[nt + 1], pa, vb + 2);
-    }
-    __syncthreads();   // every warp is done with this block's K/V tiles
-  }
-
-  // ---- merge the 8 warps (rows < r only)
-  if (lane % 4 == 0) {
-    wm[warp][gq] = m_run[0];
-    wl[warp][gq] = l_run[0];
-    wm[warp][gq + 8] = m_run[1];
-    wl[warp][gq + 8] = l_run[1];
-  }
-  __syncthreads();
-  float wscale[2];
-  float Mrow[2], Lrow[2];
-#pragma unroll
-  for (int h = 0; h < 2; ++h) {
-    const int row = gq + 8 * h;
-    float M = -INFINITY;
-    for (int w = 0; w < 8; ++w) M = fmaxf(M, wm[w][row]);
-    float L = 0.f;
-    for (int w = 0; w < 8; ++w)
-      L += wm[w][row] == -INFINITY ? 0.f : wl[w][row] * exp2f(wm[w][row] - M);
-    Mrow[h] = M;
-    Lrow[h] = L;
-    wscale[h] = (m_run[h] == -INFINITY || L == 0.f) ? 0.f : exp2f(m_run[h] - M) / L;
-  }
-  // red: [8 warps][r rows][D] fp32, reusing the K/V tiles
-  const int r = p.r;
-#pragma unroll
-  for (int nt = 0; nt < NT; ++nt) {
-    const int col = nt * 8 + 2 * qd;
-    if (gq < r) {
-      red[(warp * r + gq) * D + col] = o_acc[nt][0] * wscale[0];
-      red[(warp * r + gq) * D + col + 1] = o_acc[nt][1] * wscale[0];
-    }
-    if (gq + 8 < r) {
-      red[(warp * r + gq + 8) * D + col] = o_acc[nt][2] * wscale[1];
-      red[(warp * r + gq + 8) * D + col + 1] = o_acc[nt][3] * wscale[1];
-    }
-  }
-  __syncthreads();
-  const long long part = static_cast<long long>(bg) * p.nsplit + split;
-  for (int x = threadIdx.x; x < r * D; x += kThreads) {
-    float acc = 0.f;
-#pragma unroll
-    for (int w = 0; w < 8; ++w) acc += red[w * r * D + x];
-    p.part_o[part * r * D + x] = acc;
-  }
-  if (threadIdx.x < 32 && lane % 4 == 0) {
+    const int slot = 2 * static_cast<int>(blockIdx.x) + (first == i0 ? 0 : 1);
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
       const int row = gq + 8 * h;
-      if (row < r)
-        p.part_lse[part * r + row] =
-            (Lrow[h] > 0.f && Mrow[h] != -INFINITY) ? Mrow[h] + log2f(Lrow[h]) : -INFINITY;
+      if (row >= r) continue;
+      float* prow = p.part_o + (static_cast<long long>(slot) * r + row) * D;
+#pragma unroll
+      for (int nt = 0; nt < NW; ++nt) {
+        const int col = w * (D / 8) + nt * 8 + 2 * qd;
+        *reinterpret_cast<float2*>(prow + col) =
+            make_float2(o_acc[nt][2 * h] * inv[h], o_acc[nt][2 * h + 1] * inv[h]);
+      }
+      if (w == 0 && qd == 0) p.part_lse[static_cast<long long>(slot) * r + row] = lse2[h];
     }
-  }
-  // ---- split combine in the last-arriving CTA of this (sequence, group)
-  __threadfence();
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    const uint32_t prev = atomicAdd(&p.counters[bg], 1u);
-    s_last = (prev == static_cast<uint32_t>(p.nsplit - 1)) ? 1 : 0;
-  }
-  __syncthreads();
-  if (!s_last) return;
-  __threadfence();
-  const long long p0 = static_cast<long long>(bg) * p.nsplit;
-  for (int x = threadIdx.x; x < r * D; x += kThreads) {
-    const int row = x / D;
-    float M = -INFINITY;
-    for (int j = 0; j < p.nsplit; ++j) M = fmaxf(M, __ldcg(&p.part_lse[(p0 + j) * r + row]));
-    float den = 0.f, acc = 0.f;
-    for (int j = 0; j < p.nsplit; ++j) {
-      const float lj = __ldcg(&p.part_lse[(p0 + j) * r + row]);
-      if (lj == -INFINITY) continue;
-      const float wj = exp2f(lj - M);
-      den += wj;
-      acc += wj * __ldcg(&p.part_o[(p0 + j) * r * D + x]);
+    __threadfence();
+    named_bar_sync(1, kConsumerThreads);
+    const int cf = cta_of(bfirst, n, grid), cl = cta_of(bfirst + p.per_bg - 1, n, grid);
+    if (threadIdx.x == 0) {
+      const uint32_t prev = atomicAdd(&p.counters[bg], 1u);
+      *s_last = prev == static_cast<uint32_t>(cl - cf) ? 1 : 0;
     }
-    const int h = g * r + row;
-    p.o[(static_cast<long long>(b) * p.H + h) * D + (x % D)] =
-        __bfloat16_as_ushort(__float2bfloat16_rn(acc / den));
-    if (p.lse && (x % D) == 0)
-      p.lse[static_cast<long long>(b) * p.H + h] = (M + log2f(den)) / kLog2e;
-  }
-  if (threadIdx.x == 0) p.counters[bg] = 0u;
-}
+    named_bar_sync(1, kConsumerThreads);
+    if (!*s_last) return;
+    __threadfence();
+    const int sf = 2 * cf + (bfirst == cta_first(cf, n, grid) ? 0 : 1);
+    for (int x = threadIdx.x; x < r * D; x += kConsumerThreads) {
+      const int row = x / D;
+      float M = -INFINITY;
+      for (int c = cf; c <= cl; ++c) {
+        const int sl = c == cf ? sf : 2 * c;
+        M = fmaxf(M, __ldcg(&p.part_lse[static_cast<long long>(sl) * r + row]));
+      }
+      float den = 0.f, acc = 0.f;
+      for (int c = cf; c <= cl; ++c) {
+        const int sl = c == cf ? sf : 2 * c;
+        const float lj = __ldcg(&p.part_lse[static_cast<long long>(sl) * r + row]);
+        if (lj == -INFINITY) continue;
+        const float wj = exp2f(lj - M);
+        den += wj;
+        acc += wj * __ldcg(&p.part_o[static_cast<long long>(sl) * r * D + x]);
+      }
+      const int hh = g * r + row;
+      p.o[(static_cast<long long>(b) * p.H + hh) * D + (x % D)] =
+          __bfloat16_as_ushort(__float2bfloat16_rn(den > 0.f ? acc / den : 0.f));
+      if (p.lse && (x % D) == 0)
+        p.lse[static_cast<long long>(b) * p.H + hh] =
+            den > 0.f ? (M + log2f(den)) / kLog2e : -INFINITY;
+    }
+    if (threadIdx.x == 0) p.counters[bg] = 0u;
+  };
 
-int dense_splits(const msa_shape& s) {
-  const int nb = static_cast<int>(ceil_div(s.seq_kv, 128));
-  return static_cast<int>(ceil_div(nb, kDenseBlocksPerSplit));
+  for (long long base = i0; !failed && base < i1; base += 32) {
+    int bgv = 0;
+    const int blkv = base + lane < i1 ? item_block(p, base + lane, bt, &bgv) : -1;
+    const int nin = static_cast<int>(min(32LL, i1 - base));
+    for (int jj = 0; jj < nin; ++jj) {
+      const int blk = __shfl_sync(0xffffffffu, blkv, jj);
+      const int bg = __shfl_sync(0xffffffffu, bgv, jj);
+      if (bg != cur_bg) {
+        if (cur_bg >= 0) finish(cur_bg, seg_first, base + jj);
+        cur_bg = bg;
+        seg_first = base + jj;
+        const int b = bg / p.G, g = bg % p.G;
+        const uint16_t* qb = p.q + (static_cast<long long>(b) * p.H + g * p.r) * D;
+#pragma unroll
+        for (int ks = 0; ks < KS; ++ks) {
+          const int c0 = ks * 16 + 2 * qd;
+          qa[ks][0] = gq < p.r ? __ldg(reinterpret_cast<const uint32_t*>(qb + gq * D + c0)) : 0u;
+          qa[ks][1] =
+              gq + 8 < p.r ? __ldg(reinterpret_cast<const uint32_t*>(qb + (gq + 8) * D + c0)) : 0u;
+          qa[ks][2] =
+              gq < p.r ? __ldg(reinterpret_cast<const uint32_t*>(qb + gq * D + c0 + 8)) : 0u;
+          qa[ks][3] = gq + 8 < p.r
+                          ? __ldg(reinterpret_cast<const uint32_t*>(qb + (gq + 8) * D + c0 + 8))
+                          : 0u;
+        }
+        m_run[0] = m_run[1] = -INFINITY;
+        l_run[0] = l_run[1] = 0.f;
+#pragma unroll
+        for (int nt = 0; nt < NW; ++nt)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) o_acc[nt][e] = 0.f;
+      }
+      if (blk < 0) continue;
+      const int s = cnt % S;
+      const uint32_t ph = (cnt / S) & 1;
+      ++cnt;
+      const uint32_t kbase = smem_u32(smem + s * 2 * L::kTile);
+      const uint32_t vbase = kbase + L::kTile;
+
+      // ---- S = Q K^T for keys w*16 .. w*16+15 of the block
+      const bool okk = mbar_wait(&kfull[s], ph, abort_flag, p.err);
+      float sv[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt) {
+        const int key = w * 16 + nt * 8 + gq;
+#pragma unroll
+        for (int ks = 0; ks < KS; ++ks) {
+          uint32_t bb[2];
+          const int col = ks * 16 + 2 * qd;
+          asm volatile("ld.shared.b32 %0, [%1];" : "=r"(bb[0]) : "r"(kbase + sw128_off(key, col)));
+          asm volatile("ld.shared.b32 %0, [%1];"
+                       : "=r"(bb[1])
+                       : "r"(kbase + sw128_off(key, col + 8)));
+          mma16816(sv[nt], qa[ks], bb);
+        }
+      }
+      float mx[2] = {-INFINITY, -INFINITY};
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int key = blk * 128 + w * 16 + nt * 8 + 2 * qd + (e & 1);
+          sv[nt][e] = key <= pos ? sv[nt][e] * p.scale_log2 : -INFINITY;
+          mx[e >> 1] = fmaxf(mx[e >> 1], sv[nt][e]);
+        }
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        mx[h] = fmaxf(mx[h], __shfl_xor_sync(0xffffffffu, mx[h], 1));
+        mx[h] = fmaxf(mx[h], __shfl_xor_sync(0xffffffffu, mx[h], 2));
+      }
+      if (qd == 0) {
+        wmax[w * 16 + gq] = mx[0];
+        wmax[w * 16 + gq + 8] = mx[1];
+      }
+      if (named_bar_or(1, kConsumerThreads, !okk || *abort_flag)) {
+        failed = true;
+        *abort_flag = 1;
+        break;
+      }
+      // ---- block row maxima, P = exp2(S - m) in bf16, row sums
+      float corr[2], mnew[2];
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        float bm = -INFINITY;
+#pragma unroll
+        for (int x = 0; x < 8; ++x) bm = fmaxf(bm, wmax[x * 16 + gq + 8 * h]);
+        mnew[h] = fmaxf(m_run[h], bm);
+        corr[h] = mnew[h] == -INFINITY ? 1.f : exp2f(m_run[h] - mnew[h]);
+        m_run[h] = mnew[h];
+      }
+      float rs[2] = {0.f, 0.f};
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float mh = mnew[e >> 1];
+          const float pv = mh == -INFINITY ? 0.f : exp2f(sv[nt][e] - mh);
+          sv[nt][e] = pv;
+          rs[e >> 1] += pv;
+        }
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt) {
+        const int key = w * 16 + nt * 8 + 2 * qd;
+        *reinterpret_cast<uint32_t*>(ps + gq * kPStride + key) = pack_bf16(sv[nt][0], sv[nt][1]);
+        *reinterpret_cast<uint32_t*>(ps + (gq + 8) * kPStride + key) =
+            pack_bf16(sv[nt][2], sv[nt][3]);
+      }
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        rs[h] += __shfl_xor_sync(0xffffffffu, rs[h], 1);
+        rs[h] += __shfl_xor_sync(0xffffffffu, rs[h], 2);
+      }
+      if (qd == 0) {
+        wsum[w * 16 + gq] = rs[0];
+        wsum[w * 16 + gq + 8] = rs[1];
+      }
+      const bool okv = mbar_wait(&vfull[s], ph, abort_flag, p.err);
+      if (named_bar_or(1, kConsumerThreads, !okv || *abort_flag)) {
+        failed = true;
+        *abort_flag = 1;
+        break;
+      }
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        float bs = 0.f;
+#pragma unroll
+        for (int x = 0; x < 8; ++x) bs += wsum[x * 16 + gq + 8 * h];
+        l_run[h] = l_run[h] * corr[h] + bs;
+      }
+#pragma unroll
+      for (int nt = 0; nt < NW; ++nt) {
+        o_acc[nt][0] *= corr[0];
+        o_acc[nt][1] *= corr[0];
+        o_acc[nt][2] *= corr[1];
+        o_acc[nt][3] *= corr[1];
+      }
+      // ---- O[:, w*D/8 ..] += P V over the block's 128 keys
+      const int mi = lane >> 3, ri = lane & 7;
+#pragma unroll
+      for (int ks = 0; ks < 8; ++ks) {
+        uint32_t pa[4];
+        ldsm_x4(pbase + static_cast<uint32_t>(((mi & 1) * 8 + ri) * kPStride * 2 +
+                                              (ks * 16 + (mi >> 1) * 8) * 2),
+                pa);
+        const int vkey = ks * 16 + (mi & 1) * 8 + ri;
+        if constexpr (NW == 2) {
+          uint32_t vb[4];
+          ldsm_x4_trans(vbase + sw128_off(vkey, w * 16 + (mi >> 1) * 8), vb);
+          mma16816(o_acc[0], pa, vb);
+          mma16816(o_acc[1], pa, vb + 2);
+        } else {
+          uint32_t vb[2];
+          ldsm_x2_trans(vbase + sw128_off(vkey, w * 8), vb);
+          mma16816(o_acc[0], pa, vb);
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[s]);
+    }
+  }
+  if (!failed && cur_bg >= 0) finish(cur_bg, seg_first, i1);
 }
 
 }  // namespace
@@ -322,9 +472,11 @@ int dense_splits(const msa_shape& s) {
 size_t decode_workspace_bytes(const msa_shape& s, bool dense) {
   const int r = s.n_q_heads / s.n_kv_heads;
   const size_t bg = static_cast<size_t>(s.batch) * s.n_kv_heads;
-  const size_t ns = dense ? static_cast<size_t>(dense_splits(s)) : static_cast<size_t>(s.topk);
-  return align_up(bg * 4, 256) + align_up(bg * ns * r * 4, 256) +
-         align_up(bg * ns * r * s.head_dim * 4, 256);
+  const size_t per_bg = dense ? static_cast<size_t>(ceil_div(s.seq_kv, 128))
+                              : static_cast<size_t>(s.topk);
+  const size_t slots = 2 * std::min(bg * per_bg, static_cast<size_t>(kMaxGrid));
+  return align_up(bg * 4, 256) + align_up(slots * r * 4, 256) +
+         align_up(slots * r * s.head_dim * 4, 256);
 }
 
 cudaError_t launch_decode(const msa_shape& s, const uint16_t* q, const uint16_t* k,
@@ -334,25 +486,30 @@ cudaError_t launch_decode(const msa_shape& s, const uint16_t* q, const uint16_t*
   if (!ctx) return cudaErrorInitializationError;
   const int r = s.n_q_heads / s.n_kv_heads;
   const size_t bg = static_cast<size_t>(s.batch) * s.n_kv_heads;
-  const int ns = dense ? dense_splits(s) : s.topk;
+  const int per_bg = dense ? static_cast<int>(ceil_div(s.seq_kv, 128)) : s.topk;
+  const long long n_items = static_cast<long long>(bg) * per_bg;
+  const long long grid = std::min<long long>(
+      n_items, std::min<long long>(std::max(ctx->num_sms, 1), kMaxGrid));
+  const size_t slots = 2 * static_cast<size_t>(std::min<long long>(n_items, kMaxGrid));
   DecParams p{};
   char* w = static_cast<char*>(ws);
   p.counters = reinterpret_cast<uint32_t*>(w);
   p.part_lse = reinterpret_cast<float*>(w + align_up(bg * 4, 256));
-  p.part_o = reinterpret_cast<float*>(w + align_up(bg * 4, 256) + align_up(bg * ns * r * 4, 256));
+  p.part_o = reinterpret_cast<float*>(w + align_up(bg * 4, 256) + align_up(slots * r * 4, 256));
   p.q = q;
   p.sel = dense ? nullptr : sel;
   p.o = o;
   p.lse = lse;
   p.err = ctx->err;
+  p.n_items = n_items;
+  p.per_bg = per_bg;
   p.N = s.seq_kv;
   p.H = s.n_q_heads;
   p.G = s.n_kv_heads;
   p.r = r;
   p.k = s.topk;
-  p.nsplit = ns;
-  p.bps = kDenseBlocksPerSplit;
   p.scale_log2 = kLog2e / sqrtf(static_cast<float>(s.head_dim));
+  if (n_items == 0) return cudaSuccess;
 
   CUtensorMap tk, tv;
   const uint64_t dims[3] = {static_cast<uint64_t>(s.head_dim), static_cast<uint64_t>(s.seq_kv),
@@ -368,25 +525,21 @@ cudaError_t launch_decode(const msa_shape& s, const uint16_t* q, const uint16_t*
 
   cudaError_t e = cudaMemsetAsync(p.counters, 0, bg * 4, st);
   if (e != cudaSuccess) return e;
-  const dim3 grid(static_cast<unsigned>(ns), static_cast<unsigned>(s.n_kv_heads),
-                  static_cast<unsigned>(s.batch));
-  const size_t smem = 1024 + 2 * 128 * s.head_dim * 2 + 64;
+  const unsigned g = static_cast<unsigned>(grid);
   if (s.head_dim == 128) {
+    const size_t smem = DecLayout<128>::kBytes;
     e = cudaFuncSetAttribute(decode_attn_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(smem));
     if (e != cudaSuccess) return e;
-    {
     ProfScope ps_("decode_attn", st);
-    decode_attn_kernel<128><<<grid, kThreads, smem, st>>>(tk, tv, p);
-  }
+    decode_attn_kernel<128><<<g, kThreads, smem, st>>>(tk, tv, p);
   } else {
+    const size_t smem = DecLayout<64>::kBytes;
     e = cudaFuncSetAttribute(decode_attn_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(smem));
     if (e != cudaSuccess) return e;
-    {
     ProfScope ps_("decode_attn", st);
-    decode_attn_kernel<64><<<grid, kThreads, smem, st>>>(tk, tv, p);
-  }
+    decode_attn_kernel<64><<<g, kThreads, smem, st>>>(tk, tv, p);
   }
   return cudaGetLastError();
 }

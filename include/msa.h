@@ -134,8 +134,10 @@ msa_status msa_sparse_attn_prefill(const msa_shape* shape, const uint16_t* q,
                                    void* ws, size_t ws_bytes, void* stream);
 
 /* Main branch, decode: same formula with T == 1 and q_offset == N - 1 (the new
- * token is already the last cache row).  Split-K over the selected blocks
- * with an in-kernel combine.  ws >= msa_workspace_size(MSA_OP_SPARSE_DECODE). */
+ * token is already the last cache row).  A persistent grid streams the
+ * selected blocks of every (sequence, group) through a TMA pipeline; a group
+ * whose blocks fall to several CTAs is merged in-kernel by the last of them.
+ * ws >= msa_workspace_size(MSA_OP_SPARSE_DECODE). */
 msa_status msa_sparse_attn_decode(const msa_shape* shape, const uint16_t* q,
                                   const uint16_t* k, const uint16_t* v,
                                   const int32_t* sel, uint16_t* o, float* lse,
@@ -158,8 +160,8 @@ msa_status msa_dense_attn_prefill(const msa_shape* shape, const uint16_t* q,
                                   const uint16_t* k, const uint16_t* v, uint16_t* o,
                                   float* lse, void* ws, size_t ws_bytes, void* stream);
 
-/* Dense causal GQA decode (T == 1): split-K over all causal blocks.
- * ws >= msa_workspace_size(MSA_OP_DENSE_DECODE). */
+/* Dense causal GQA decode (T == 1): the sparse decode kernel over all causal
+ * blocks.  ws >= msa_workspace_size(MSA_OP_DENSE_DECODE). */
 msa_status msa_dense_attn_decode(const msa_shape* shape, const uint16_t* q,
                                  const uint16_t* k, const uint16_t* v, uint16_t* o,
                                  float* lse, void* ws, size_t ws_bytes, void* stream);
@@ -174,9 +176,9 @@ msa_status msa_dense_attn_decode(const msa_shape* shape, const uint16_t* q,
  * static device array of MSA_DECODE_STATIC_SCRATCH_BYTES compiled into the
  * library, which every GPU that loads the library holds until the process
  * exits.  Shapes whose scratch would exceed it (round256(4*B*G) +
- * round256(4*B*G*k*r) + round256(4*B*G*k*r*d) bytes) return
- * MSA_ERR_WORKSPACE_TOO_SMALL before any launch; B=32, G=8, k=16, r=8, d=128
- * fits.  The first call on a device looks up the array's device address with
+ * round256(4*S*r) + round256(4*S*r*d) bytes, S = 2*min(B*G*k, 256)) return
+ * MSA_ERR_WORKSPACE_TOO_SMALL before any launch: only batches with more than
+ * about six million (sequence, group) pairs do.  The first call on a device looks up the array's device address with
  * that device current; make that first call before any stream capture.  All
  * calls share the one array and it keeps the previous call's contents (the
  * counters that must start at zero are cleared by every call): calls that can

@@ -154,7 +154,11 @@ def test_sparse_prefill_spans_token_chunks():
 
 @pytest.mark.parametrize("sp", [spec(3, 1, 3000, 2999, 16, 2, 128, 64, 4, seed=21),
                                 spec(2, 1, 5000, 4999, 8, 2, 64, 32, 16, seed=22),
-                                spec(2, 1, 129, 128, 16, 1, 128, 64, 16, seed=23)])
+                                spec(2, 1, 129, 128, 16, 1, 128, 64, 16, seed=23),
+                                # more (sequence, group, block) items than SMs: each CTA
+                                # streams several blocks, some groups finish inside one CTA
+                                spec(32, 1, 3000, 2999, 16, 8, 64, 32, 4, seed=24),
+                                spec(12, 1, 9000, 8999, 16, 4, 128, 64, 16, seed=25)])
 def test_sparse_decode(sp):
     inp = inputs_cpu(sp)
     sels = [oracle_sel(sp, oracle_pooled(sp, inp, b)) for b in range(sp.batch)]
@@ -167,8 +171,10 @@ def test_sparse_decode(sp):
         assert np.abs(lse[b].double().cpu().numpy() - L_ref).max() < LSE_ABS
 
 
-def test_dense_decode():
-    sp = spec(2, 1, 4000, 3999, 16, 2, 128, 64, 4, seed=31)
+@pytest.mark.parametrize("sp", [spec(2, 1, 4000, 3999, 16, 2, 128, 64, 4, seed=31),
+                                # 2504 blocks: every (sequence, group) spans many CTAs
+                                spec(2, 1, 40000, 39999, 8, 4, 128, 64, 4, seed=36)])
+def test_dense_decode(sp):
     inp = inputs_cpu(sp)
     o, lse = M.dense_attn_decode(M.Shape.of(sp), cuda(inp.q), cuda(inp.k), cuda(inp.v))
     torch.cuda.synchronize()

@@ -54,9 +54,9 @@ def test_static_scratch_decode_matches_workspace_entry_point():
 
 
 def test_static_scratch_rejects_shapes_beyond_its_size():
-    # 64 sequences x 8 groups x 64 slots x 16 heads x 128 dims of fp32 partials
-    # need far more than the static array holds
-    sp = spec(64, 1, 200000, 199999, 128, 8, 128, 64, 64)
+    # 2^20 sequences x 8 groups: the per-(sequence, group) counters alone
+    # need more than the static array holds
+    sp = spec(1 << 20, 1, 255, 254, 16, 8, 128, 64, 2)
     sh = M.Shape.of(sp)
     assert M.workspace_size(sh, M.OP_SPARSE_DECODE) > 24 * 2**20
     dummy = torch.empty(16, dtype=torch.uint8, device="cuda")
