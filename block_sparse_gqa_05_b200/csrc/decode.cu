@@ -55,7 +55,7 @@ struct DecLayout {
   static constexpr uint32_t kOffP = kStages * 2u * kTile;      // P [16][kPStride] bf16
   static constexpr uint32_t kOffRed = kOffP + 16u * kPStride * 2u;   // wmax, wsum [8][16]
   static constexpr uint32_t kOffBar = kOffRed + 2u * 8u * 16u * 4u;
-  static constexpr uint32_t kOffFlag = kOffBar + 3u * kStages * 8u;  // abort, last
+  static constexpr uint32_t kOffFlag = kOffBar + 3u * kStages * 8u;  // abort, last[2]
   static constexpr uint32_t kBytes = kOffFlag + 16u;
 };
 
@@ -133,7 +133,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* vfull = kfull + S;
   uint64_t* empty = vfull + S;
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kOffFlag);
-  volatile int* s_last = abort_flag + 1;
+  volatile int* s_last = abort_flag + 1;   // [2]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const long long n = p.n_items, grid = gridDim.x;
@@ -224,8 +224,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   float m_run[2], l_run[2];
   float o_acc[NW][4];
 
+  // Partials of this CTA still to be announced: the group whose items open
+  // its range (slot 0) and the one whose items close it (slot 1).
+  int pend[2] = {-1, -1};
+
   // Write the (sequence, group) just finished: directly when this CTA holds
-  // all of its items, else as a partial, merged by the last CTA to finish it.
+  // all of its items, else as a normalised partial in this CTA's slot.
   auto finish = [&](int bg, long long first, long long end) {
     const int b = bg / p.G, g = bg % p.G;
     const int r = p.r;
@@ -253,7 +257,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       return;
     }
-    const int slot = 2 * static_cast<int>(blockIdx.x) + (first == i0 ? 0 : 1);
+    const int which = first == i0 ? 0 : 1;
+    pend[which] = bg;
+    const int slot = 2 * static_cast<int>(blockIdx.x) + which;
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
       const int row = gq + 8 * h;
@@ -267,41 +273,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (w == 0 && qd == 0) p.part_lse[static_cast<long long>(slot) * r + row] = lse2[h];
     }
-    __threadfence();
-    named_bar_sync(1, kConsumerThreads);
-    const int cf = cta_of(bfirst, n, grid), cl = cta_of(bfirst + p.per_bg - 1, n, grid);
-    if (threadIdx.x == 0) {
-      const uint32_t prev = atomicAdd(&p.counters[bg], 1u);
-      *s_last = prev == static_cast<uint32_t>(cl - cf) ? 1 : 0;
-    }
-    named_bar_sync(1, kConsumerThreads);
-    if (!*s_last) return;
-    __threadfence();
-    const int sf = 2 * cf + (bfirst == cta_first(cf, n, grid) ? 0 : 1);
-    for (int x = threadIdx.x; x < r * D; x += kConsumerThreads) {
-      const int row = x / D;
-      float M = -INFINITY;
-      for (int c = cf; c <= cl; ++c) {
-        const int sl = c == cf ? sf : 2 * c;
-        M = fmaxf(M, __ldcg(&p.part_lse[static_cast<long long>(sl) * r + row]));
-      }
-      float den = 0.f, acc = 0.f;
-      for (int c = cf; c <= cl; ++c) {
-        const int sl = c == cf ? sf : 2 * c;
-        const float lj = __ldcg(&p.part_lse[static_cast<long long>(sl) * r + row]);
-        if (lj == -INFINITY) continue;
-        const float wj = exp2f(lj - M);
-        den += wj;
-        acc += wj * __ldcg(&p.part_o[static_cast<long long>(sl) * r * D + x]);
-      }
-      const int hh = g * r + row;
-      p.o[(static_cast<long long>(b) * p.H + hh) * D + (x % D)] =
-          __bfloat16_as_ushort(__float2bfloat16_rn(den > 0.f ? acc / den : 0.f));
-      if (p.lse && (x % D) == 0)
-        p.lse[static_cast<long long>(b) * p.H + hh] =
-            den > 0.f ? (M + log2f(den)) / kLog2e : -INFINITY;
-    }
-    if (threadIdx.x == 0) p.counters[bg] = 0u;
   };
 
   for (long long base = i0; !failed && base < i1; base += 32) {
@@ -464,7 +435,93 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (lane == 0) mbar_arrive(&empty[s]);
     }
   }
-  if (!failed && cur_bg >= 0) finish(cur_bg, seg_first, i1);
+  if (failed) return;
+  if (cur_bg >= 0) finish(cur_bg, seg_first, i1);
+  if (pend[0] < 0 && pend[1] < 0) return;
+
+  // Announce the partials; the last CTA to finish a group merges its
+  // partials.  Every load of the ring has been consumed, so the stage memory
+  // holds the merge weights.
+  __threadfence();
+  named_bar_sync(1, kConsumerThreads);
+  if (threadIdx.x == 0) {
+#pragma unroll
+    for (int x = 0; x < 2; ++x) {
+      s_last[x] = 0;
+      if (pend[x] < 0) continue;
+      const long long bfirst = static_cast<long long>(pend[x]) * p.per_bg;
+      const int cf = cta_of(bfirst, n, grid), cl = cta_of(bfirst + p.per_bg - 1, n, grid);
+      const uint32_t prev = atomicAdd(&p.counters[pend[x]], 1u);
+      s_last[x] = prev == static_cast<uint32_t>(cl - cf) ? 1 : 0;
+    }
+  }
+  named_bar_sync(1, kConsumerThreads);
+  const int r = p.r;
+  float* wgt = reinterpret_cast<float*>(smem);   // [CTAs of the group][r]
+#pragma unroll 1
+  for (int x = 0; x < 2; ++x) {
+    if (!s_last[x]) continue;
+    __threadfence();
+    const int bg = pend[x];
+    const int b = bg / p.G, g = bg % p.G;
+    const long long bfirst = static_cast<long long>(bg) * p.per_bg;
+    const int cf = cta_of(bfirst, n, grid), cl = cta_of(bfirst + p.per_bg - 1, n, grid);
+    const int nc = cl - cf + 1;
+    const int sf = 2 * cf + (bfirst == cta_first(cf, n, grid) ? 0 : 1);
+    for (int e = threadIdx.x; e < nc * r; e += kConsumerThreads) {
+      const int c = cf + e / r;
+      const int sl = c == cf ? sf : 2 * c;
+      wgt[e] = __ldcg(&p.part_lse[static_cast<long long>(sl) * r + e % r]);
+    }
+    named_bar_sync(1, kConsumerThreads);
+    // per row: max and sum of the partial weights (warp w: rows w, w + 8)
+    for (int row = w; row < r; row += kConsumerWarps) {
+      float M = -INFINITY;
+      for (int c = lane; c < nc; c += 32) M = fmaxf(M, wgt[c * r + row]);
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+      float den = 0.f;
+      for (int c = lane; c < nc; c += 32) {
+        const float lj = wgt[c * r + row];
+        den += lj == -INFINITY ? 0.f : exp2f(lj - M);
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
+      __syncwarp();
+      const float rden = den > 0.f ? 1.f / den : 0.f;
+      for (int c = lane; c < nc; c += 32) {
+        const float lj = wgt[c * r + row];
+        wgt[c * r + row] = lj == -INFINITY ? 0.f : exp2f(lj - M) * rden;
+      }
+      if (p.lse && lane == 0)
+        p.lse[static_cast<long long>(b) * p.H + g * r + row] =
+            den > 0.f ? (M + log2f(den)) / kLog2e : -INFINITY;
+    }
+    named_bar_sync(1, kConsumerThreads);
+    // outputs, four columns per thread, every partial's load in flight at once
+    for (int e = threadIdx.x; e < r * D / 4; e += kConsumerThreads) {
+      const int row = (e * 4) / D, col = (e * 4) % D;
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 4
+      for (int c = cf; c <= cl; ++c) {
+        const int sl = c == cf ? sf : 2 * c;
+        const float wj = wgt[(c - cf) * r + row];
+        const float4 v4 = __ldcg(reinterpret_cast<const float4*>(
+            p.part_o + (static_cast<long long>(sl) * r + row) * D + col));
+        acc.x += wj * v4.x;
+        acc.y += wj * v4.y;
+        acc.z += wj * v4.z;
+        acc.w += wj * v4.w;
+      }
+      uint2 pk;
+      pk.x = pack_bf16(acc.x, acc.y);
+      pk.y = pack_bf16(acc.z, acc.w);
+      *reinterpret_cast<uint2*>(p.o + (static_cast<long long>(b) * p.H + g * r + row) * D + col) =
+          pk;
+    }
+    if (threadIdx.x == 0) p.counters[bg] = 0u;
+    named_bar_sync(1, kConsumerThreads);
+  }
 }
 
 }  // namespace
