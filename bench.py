@@ -326,6 +326,22 @@ def run_topk_micro(M, args, stream, peaks):
     return res
 
 
+def graph_ms(fn, reps, steps, warmup, pg, stream):
+    """ms per call of fn, replayed from one CUDA graph of ``reps`` calls (a
+    decode loop is replayed this way in serving; eager launches would add the
+    host's per-launch cost between kernels of a ~0.1 ms step)."""
+    fn()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for _ in range(reps):
+            fn()
+    torch.cuda.synchronize()
+    ms = timed_loop(g.replay, steps, warmup, pg, stream) / reps
+    del g
+    return ms
+
+
 def run_decode(M, sp, args, pg, stream, world, peaks, dense):
     inp = synth.make_inputs(sp, "cuda")
     sh = M.Shape.of(sp)
@@ -337,32 +353,39 @@ def run_decode(M, sp, args, pg, stream, world, peaks, dense):
         M.forward(sh, inp.q, inp.k, inp.v, inp.q_idx, inp.k_idx, o=o, lse=None, sel=sel, ws=ws,
                   want_lse=False)
 
-    M.profile_enable(True)
-    ms = timed_loop(step, max(args.steps, 20), args.warmup, pg, stream)
-    prof = M.profile_read()
-    M.profile_enable(False)
-    kernels = {k: v[0] / v[1] for k, v in prof.items()}
+    reps, steps = 10, max(args.steps, 5)
+    ms = graph_ms(step, reps, steps, args.warmup, pg, stream)
+    # the stages one at a time, each replayed from its own graph
+    pooled = torch.empty((sp.batch, 1, sp.n_kv_heads, sp.nb), dtype=torch.float32, device="cuda")
+    aws = M.alloc_workspace(sh, M.OP_SPARSE_DECODE)
+    stages = {
+        "index_scores": lambda: M.index_scores(sh, inp.q_idx, inp.k_idx, pooled),
+        "block_topk": lambda: M.block_topk(sh, pooled, sel),
+        "sparse_attn_decode": lambda: M.sparse_attn_decode(sh, inp.q, inp.k, inp.v, sel, o, None,
+                                                           aws, want_lse=False),
+    }
+    kernels = {k: graph_ms(f, reps, steps, 1, pg, stream) for k, f in stages.items()}
     res = {"workload": f"decode_L{sp.seq_kv}_b{sp.batch}",
            "value": sp.batch * world / (ms / 1e3), "unit": "tokens/s", "ms_per_step": ms,
-           "kernels_ms_per_launch": {k: round(v, 4) for k, v in kernels.items()}}
-    if "decode_attn" in kernels:
-        b = decode_kv_bytes(sp)
-        a = b / (kernels["decode_attn"] / 1e3) / 1e9
-        res["roofline"] = {"kernel": "decode_attn", "bound": "hbm", "achieved": round(a, 1),
-                           "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                           "frac": round(a / peaks["hbm_gbs"], 4),
-                           "algorithmic_per_launch": b}
-    if "index_scores_scan" in kernels:
-        b = float(sp.batch * sp.seq_kv * sp.index_dim * 2)
-        a = b / (kernels["index_scores_scan"] / 1e3) / 1e9
-        res["index_scan"] = {"achieved_gbs": round(a, 1), "frac": round(a / peaks["hbm_gbs"], 4)}
+           "timing": "CUDA graph replay of 10 steps per launch",
+           "stages_ms_per_call": {k: round(v, 4) for k, v in kernels.items()}}
+    b = decode_kv_bytes(sp)
+    a = b / (kernels["sparse_attn_decode"] / 1e3) / 1e9
+    res["roofline"] = {"kernel": "decode_attn", "bound": "hbm", "achieved": round(a, 1),
+                       "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                       "frac": round(a / peaks["hbm_gbs"], 4),
+                       "algorithmic_per_launch": b}
+    b = float(sp.batch * sp.seq_kv * sp.index_dim * 2)
+    a = b / (kernels["index_scores"] / 1e3) / 1e9
+    res["index_scan"] = {"achieved_gbs": round(a, 1), "frac": round(a / peaks["hbm_gbs"], 4)}
+    del pooled, aws
     if dense:
         dws = M.alloc_workspace(sh, M.OP_DENSE_DECODE)
 
         def dstep():
             M.dense_attn_decode(sh, inp.q, inp.k, inp.v, o=o, lse=None, ws=dws, want_lse=False)
 
-        dms = timed_loop(dstep, max(3, args.steps // 2), args.warmup, pg, stream)
+        dms = graph_ms(dstep, 2, max(3, args.steps // 2), 1, pg, stream)
         db = float(sp.batch * sp.n_kv_heads * sp.seq_kv * sp.head_dim * 4)
         res["dense_gqa_decode"] = {"ms_per_step": dms, "value": sp.batch * world / (dms / 1e3),
                                    "achieved_gbs": round(db / (dms / 1e3) / 1e9, 1),

@@ -2,7 +2,8 @@
 // "TopK"; lumi-systems AI news: per-group independent, exponential-free top-k;
 // lefilia.fr: the local block is always included, 16 blocks of 128 tokens).
 //
-// One warp per (sequence, token, group) row.  Candidates are blocks 0..b_t-1;
+// One warp per (sequence, token, group) row, or one CTA per row when there
+// are few long rows (decode).  Candidates are blocks 0..b_t-1;
 // the order is (pooled score descending, block index ascending), encoded as a
 // 64-bit key ((order-preserving score bits) << 32 | ~index) so every compare
 // is exact and ties resolve to the lower block index.  Each chunk of 1024
@@ -110,6 +111,27 @@ __device__ __noinline__ void sort_buffer(const uint64_t* buf, int m, uint64_t& b
   best1 = S > 1 ? x[1 % S] : 0ull;
 }
 
+// The 64 largest of two descending lists of 64 keys (elements lane and
+// 32 + lane of a and of b), descending: pairing a[i] with b[63-i] leaves the
+// 64 largest as one bitonic sequence, which six half-cleaner stages sort.
+MSA_DEV void merge_top64(uint64_t& a0, uint64_t& a1, uint64_t b0, uint64_t b1) {
+  const int lane = threadIdx.x & 31;
+  const uint64_t r0 = shfl64(b1, 31 - lane), r1 = shfl64(b0, 31 - lane);
+  uint64_t c0 = a0 > r0 ? a0 : r0, c1 = a1 > r1 ? a1 : r1;
+  const uint64_t hi = c0 > c1 ? c0 : c1, lo = c0 > c1 ? c1 : c0;
+  c0 = hi;
+  c1 = lo;
+#pragma unroll
+  for (int j = 16; j > 0; j >>= 1) {
+    const bool take_max = (lane & j) == 0;
+    const uint64_t y0 = shfl_xor64(c0, j), y1 = shfl_xor64(c1, j);
+    c0 = take_max ? (c0 > y0 ? c0 : y0) : (c0 > y0 ? y0 : c0);
+    c1 = take_max ? (c1 > y1 ? c1 : y1) : (c1 > y1 ? y1 : c1);
+  }
+  a0 = c0;
+  a1 = c1;
+}
+
 // best0/best1: running list (elements lane, 32+lane, descending); nk: one new
 // key per lane (0 = none).  Keeps the 64 largest of the 96.
 __device__ __noinline__ void merge128(uint64_t& best0, uint64_t& best1, uint64_t nk) {
@@ -119,11 +141,149 @@ __device__ __noinline__ void merge128(uint64_t& best0, uint64_t& best1, uint64_t
   best1 = xk[1];
 }
 
+// Scans chunks c0, c0 + cs, c0 + 2 cs, ... (kChunk candidates each, in
+// increasing order) of one row's n candidates into the running list ``best``
+// (descending; elements lane and 32 + lane; ``have`` valid, at most kk).
+MSA_DEV void scan_chunks(const float* __restrict__ src, int n, int kk, bool vec, int c0, int cs,
+                         uint64_t* buf, uint64_t (&best)[2], int& have) {
+  const int lane = threadIdx.x & 31;
+  for (int base = c0 * kChunk; base < n; base += cs * kChunk) {
+    // this lane's scores: block base + x*128 + lane*4 + e, as order-preserving keys
+    uint32_t uk[kPer];
+#pragma unroll
+    for (int x = 0; x < kPer / 4; ++x) {
+      const int i0 = base + x * 128 + lane * 4;
+      float4 f;
+      if (vec && i0 + 3 < n) {
+        f = __ldg(reinterpret_cast<const float4*>(src + i0));
+      } else {
+        f.x = i0 < n ? __ldg(src + i0) : 0.f;
+        f.y = i0 + 1 < n ? __ldg(src + i0 + 1) : 0.f;
+        f.z = i0 + 2 < n ? __ldg(src + i0 + 2) : 0.f;
+        f.w = i0 + 3 < n ? __ldg(src + i0 + 3) : 0.f;
+      }
+      uk[4 * x] = i0 < n ? float_order_key(f.x) : 0u;
+      uk[4 * x + 1] = i0 + 1 < n ? float_order_key(f.y) : 0u;
+      uk[4 * x + 2] = i0 + 2 < n ? float_order_key(f.z) : 0u;
+      uk[4 * x + 3] = i0 + 3 < n ? float_order_key(f.w) : 0u;
+    }
+    // score threshold that keeps every member of the new top-kk
+    uint32_t tau;
+    if (have >= kk) {
+      // every later block has a larger index than the list's members, so a
+      // score equal to the current kk-th best can no longer enter: strict >
+      const uint32_t kth = static_cast<uint32_t>(shfl64(best[(kk - 1) >> 5], (kk - 1) & 31) >> 32);
+      if (kth == 0xFFFFFFFFu) continue;
+      tau = kth + 1u;
+    } else if (kk <= 32) {
+      uint32_t lmax = 0u;
+#pragma unroll
+      for (int x = 0; x < kPer; ++x) lmax = max(lmax, uk[x]);
+      tau = __shfl_sync(0xffffffffu, warp_sort_desc32(lmax), kk - 1);
+    } else {
+      tau = 0u;
+    }
+    tau = max(tau, 1u);
+    int cnt = 0;
+#pragma unroll
+    for (int x = 0; x < kPer; ++x) cnt += uk[x] >= tau ? 1 : 0;
+    int incl = cnt;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, off);
+      if (lane >= off) incl += y;
+    }
+    const int total = __shfl_sync(0xffffffffu, incl, 31);
+    if (total == 0) continue;
+    const int keep = have < kk ? have : kk;
+    const int m = keep + total;
+    if (m <= kScratch) {
+      // running list and survivors into the warp buffer, one sort of <= 128
+      if (lane < keep) buf[lane] = best[0];
+      if (lane + 32 < keep) buf[32 + lane] = best[1];
+      int slot = keep + incl - cnt;
+#pragma unroll
+      for (int x = 0; x < kPer; ++x) {
+        if (uk[x] >= tau) {
+          const int i = base + (x >> 2) * 128 + lane * 4 + (x & 3);
+          buf[slot++] = make_key(uk[x], i);
+        }
+      }
+      __syncwarp();
+      if (m <= 32) {
+        uint64_t x1[1];
+        x1[0] = lane < m ? buf[lane] : 0ull;
+        warp_sort_desc<1>(x1);
+        best[0] = x1[0];
+        best[1] = 0ull;
+      } else if (m <= 64) {
+        sort_buffer<2>(buf, m, best[0], best[1]);
+      } else {
+        sort_buffer<4>(buf, m, best[0], best[1]);
+      }
+      __syncwarp();
+    } else {
+      // rare: merge the survivors one register slot at a time
+#pragma unroll
+      for (int x = 0; x < kPer; ++x) {
+        const bool take = uk[x] >= tau;
+        const unsigned bal = __ballot_sync(0xffffffffu, take);
+        if (bal != 0u) {
+          const int i = base + (x >> 2) * 128 + lane * 4 + (x & 3);
+          merge128(best[0], best[1], take ? make_key(uk[x], i) : 0ull);
+        }
+      }
+    }
+    have = min(m, kk);
+    if (lane >= kk) best[0] = 0ull;
+    if (lane + 32 >= kk) best[1] = 0ull;
+  }
+}
+
+// Writes a row's selection: the kk chosen blocks (best, descending) plus the
+// local block bt, ascending, then -1 padding up to k.
+MSA_DEV void write_selection(int32_t* out, const uint64_t (&best)[2], int kk, int bt, int k) {
+  const int lane = threadIdx.x & 31;
+  if (kk < 32) {
+    const uint32_t idx = lane < kk ? static_cast<uint32_t>(key_index(best[0]))
+                                   : (lane == kk ? static_cast<uint32_t>(bt) : 0xFFFFFFFFu);
+    const uint32_t sorted = ~warp_sort_desc32(~idx);   // ascending
+    if (lane < k) out[lane] = lane <= kk ? static_cast<int32_t>(sorted) : -1;
+    for (int i = lane + 32; i < k; i += 32) out[i] = -1;
+  } else {
+    const uint32_t i0 = static_cast<uint32_t>(key_index(best[0]));
+    const int e1 = lane + 32;
+    const uint32_t i1 = e1 < kk ? static_cast<uint32_t>(key_index(best[1]))
+                                : (e1 == kk ? static_cast<uint32_t>(bt) : 0xFFFFFFFFu);
+    uint64_t xk[2] = {static_cast<uint64_t>(~i0), static_cast<uint64_t>(~i1)};
+    warp_sort_desc<2>(xk);
+    const uint32_t s0 = ~static_cast<uint32_t>(xk[0]), s1 = ~static_cast<uint32_t>(xk[1]);
+    if (lane < k) out[lane] = lane <= kk ? static_cast<int32_t>(s0) : -1;
+    if (e1 < k) out[e1] = e1 <= kk ? static_cast<int32_t>(s1) : -1;
+  }
+}
+
+// Rows whose selection needs no ranking: every causal block fits (kk == n)
+// or only the local block is asked for (kk == 0).  Returns true if handled.
+MSA_DEV bool write_trivial(int32_t* out, int n, int kk, int bt, int k) {
+  const int lane = threadIdx.x & 31;
+  if (kk == n) {
+    for (int i = lane; i < k; i += 32) out[i] = i <= bt ? i : -1;
+    return true;
+  }
+  if (kk == 0) {
+    for (int i = lane; i < k; i += 32) out[i] = i == 0 ? bt : -1;
+    return true;
+  }
+  return false;
+}
+
+// One warp per row: for many rows (prefill).
 __global__ void __launch_bounds__(kWarps * 32, 3)
     block_topk_kernel(const float* __restrict__ pooled, int32_t* __restrict__ sel,
                       long long rows, int T, int G, int q_off, int nb, int k) {
   __shared__ uint64_t scratch[kWarps][kScratch];
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int warp = threadIdx.x >> 5;
   uint64_t* buf = scratch[warp];
   const long long nwarps = static_cast<long long>(gridDim.x) * kWarps;
   const bool vec = (nb & 3) == 0;
@@ -135,126 +295,55 @@ __global__ void __launch_bounds__(kWarps * 32, 3)
     const int n = bt;                         // candidates 0 .. bt-1
     const int kk = min(k - 1, n);
     int32_t* out = sel + r * k;
-    if (kk == n) {                            // every causal block fits
-      for (int i = lane; i < k; i += 32) out[i] = i <= bt ? i : -1;
-      continue;
+    if (write_trivial(out, n, kk, bt, k)) continue;
+    uint64_t best[2] = {0ull, 0ull};
+    int have = 0;
+    scan_chunks(pooled + r * nb, n, kk, vec, 0, 1, buf, best, have);
+    write_selection(out, best, kk, bt, k);
+  }
+}
+
+// One CTA per row: for few long rows (decode).  Warp w scans chunks w,
+// w + kWarps, ...; the kWarps lists are then merged pairwise in a tree (each
+// merge keeps the 64 best of two sorted lists of at most 63).
+__global__ void __launch_bounds__(kWarps * 32)
+    block_topk_row_cta_kernel(const float* __restrict__ pooled, int32_t* __restrict__ sel,
+                              int T, int G, int q_off, int nb, int k) {
+  __shared__ uint64_t scratch[kWarps][kScratch];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const long long r = blockIdx.x;
+  const int t = static_cast<int>((static_cast<uint32_t>(r) / static_cast<uint32_t>(G)) %
+                                 static_cast<uint32_t>(T));
+  const int bt = (q_off + t) >> 7;
+  const int n = bt;
+  const int kk = min(k - 1, n);
+  int32_t* out = sel + r * k;
+  if (kk == n || kk == 0) {
+    if (warp == 0) write_trivial(out, n, kk, bt, k);
+    return;
+  }
+  uint64_t best[2] = {0ull, 0ull};
+  int have = 0;
+  scan_chunks(pooled + r * nb, n, kk, (nb & 3) == 0, warp, kWarps, scratch[warp], best, have);
+  __syncwarp();
+  scratch[warp][lane] = best[0];
+  scratch[warp][32 + lane] = best[1];
+  __syncthreads();
+#pragma unroll
+  for (int span = 1; span < kWarps; span <<= 1) {
+    if ((warp & (2 * span - 1)) == 0) {
+      uint64_t a0 = scratch[warp][lane], a1 = scratch[warp][32 + lane];
+      merge_top64(a0, a1, scratch[warp + span][lane], scratch[warp + span][32 + lane]);
+      __syncwarp();
+      scratch[warp][lane] = a0;
+      scratch[warp][32 + lane] = a1;
     }
-    if (kk == 0) {
-      for (int i = lane; i < k; i += 32) out[i] = i == 0 ? bt : -1;
-      continue;
-    }
-    const float* src = pooled + r * nb;
-    uint64_t best[2] = {0ull, 0ull};          // sorted descending: element lane / lane+32
-    int have = 0;                             // valid entries in best (<= kk after a chunk)
-    for (int base = 0; base < n; base += kChunk) {
-      // this lane's scores: block base + x*128 + lane*4 + e, as order-preserving keys
-      uint32_t uk[kPer];
-#pragma unroll
-      for (int x = 0; x < kPer / 4; ++x) {
-        const int i0 = base + x * 128 + lane * 4;
-        float4 f;
-        if (vec && i0 + 3 < n) {
-          f = __ldg(reinterpret_cast<const float4*>(src + i0));
-        } else {
-          f.x = i0 < n ? __ldg(src + i0) : 0.f;
-          f.y = i0 + 1 < n ? __ldg(src + i0 + 1) : 0.f;
-          f.z = i0 + 2 < n ? __ldg(src + i0 + 2) : 0.f;
-          f.w = i0 + 3 < n ? __ldg(src + i0 + 3) : 0.f;
-        }
-        uk[4 * x] = i0 < n ? float_order_key(f.x) : 0u;
-        uk[4 * x + 1] = i0 + 1 < n ? float_order_key(f.y) : 0u;
-        uk[4 * x + 2] = i0 + 2 < n ? float_order_key(f.z) : 0u;
-        uk[4 * x + 3] = i0 + 3 < n ? float_order_key(f.w) : 0u;
-      }
-      // score threshold that keeps every member of the new top-kk
-      uint32_t tau;
-      if (have >= kk) {
-        // every later block has a larger index than the list's members, so a
-        // score equal to the current kk-th best can no longer enter: strict >
-        const uint32_t kth = static_cast<uint32_t>(shfl64(best[(kk - 1) >> 5], (kk - 1) & 31) >> 32);
-        if (kth == 0xFFFFFFFFu) continue;
-        tau = kth + 1u;
-      } else if (kk <= 32) {
-        uint32_t lmax = 0u;
-#pragma unroll
-        for (int x = 0; x < kPer; ++x) lmax = max(lmax, uk[x]);
-        tau = __shfl_sync(0xffffffffu, warp_sort_desc32(lmax), kk - 1);
-      } else {
-        tau = 0u;
-      }
-      tau = max(tau, 1u);
-      int cnt = 0;
-#pragma unroll
-      for (int x = 0; x < kPer; ++x) cnt += uk[x] >= tau ? 1 : 0;
-      int incl = cnt;
-#pragma unroll
-      for (int off = 1; off < 32; off <<= 1) {
-        const int y = __shfl_up_sync(0xffffffffu, incl, off);
-        if (lane >= off) incl += y;
-      }
-      const int total = __shfl_sync(0xffffffffu, incl, 31);
-      if (total == 0) continue;
-      const int keep = have < kk ? have : kk;
-      const int m = keep + total;
-      if (m <= kScratch) {
-        // running list and survivors into the warp buffer, one sort of <= 128
-        if (lane < keep) buf[lane] = best[0];
-        if (lane + 32 < keep) buf[32 + lane] = best[1];
-        int slot = keep + incl - cnt;
-#pragma unroll
-        for (int x = 0; x < kPer; ++x) {
-          if (uk[x] >= tau) {
-            const int i = base + (x >> 2) * 128 + lane * 4 + (x & 3);
-            buf[slot++] = make_key(uk[x], i);
-          }
-        }
-        __syncwarp();
-        if (m <= 32) {
-          uint64_t x1[1];
-          x1[0] = lane < m ? buf[lane] : 0ull;
-          warp_sort_desc<1>(x1);
-          best[0] = x1[0];
-          best[1] = 0ull;
-        } else if (m <= 64) {
-          sort_buffer<2>(buf, m, best[0], best[1]);
-        } else {
-          sort_buffer<4>(buf, m, best[0], best[1]);
-        }
-        __syncwarp();
-      } else {
-        // rare: merge the survivors one register slot at a time
-#pragma unroll
-        for (int x = 0; x < kPer; ++x) {
-          const bool take = uk[x] >= tau;
-          const unsigned bal = __ballot_sync(0xffffffffu, take);
-          if (bal != 0u) {
-            const int i = base + (x >> 2) * 128 + lane * 4 + (x & 3);
-            merge128(best[0], best[1], take ? make_key(uk[x], i) : 0ull);
-          }
-        }
-      }
-      have = min(m, kk);
-      if (lane >= kk) best[0] = 0ull;
-      if (lane + 32 >= kk) best[1] = 0ull;
-    }
-    // output: the kk chosen blocks plus bt, ascending, then -1 padding
-    if (kk < 32) {
-      const uint32_t idx = lane < kk ? static_cast<uint32_t>(key_index(best[0]))
-                                     : (lane == kk ? static_cast<uint32_t>(bt) : 0xFFFFFFFFu);
-      const uint32_t sorted = ~warp_sort_desc32(~idx);   // ascending
-      if (lane < k) out[lane] = lane <= kk ? static_cast<int32_t>(sorted) : -1;
-      for (int i = lane + 32; i < k; i += 32) out[i] = -1;
-    } else {
-      const uint32_t i0 = static_cast<uint32_t>(key_index(best[0]));
-      const int e1 = lane + 32;
-      const uint32_t i1 = e1 < kk ? static_cast<uint32_t>(key_index(best[1]))
-                                  : (e1 == kk ? static_cast<uint32_t>(bt) : 0xFFFFFFFFu);
-      uint64_t xk[2] = {static_cast<uint64_t>(~i0), static_cast<uint64_t>(~i1)};
-      warp_sort_desc<2>(xk);
-      const uint32_t s0 = ~static_cast<uint32_t>(xk[0]), s1 = ~static_cast<uint32_t>(xk[1]);
-      if (lane < k) out[lane] = lane <= kk ? static_cast<int32_t>(s0) : -1;
-      if (e1 < k) out[e1] = e1 <= kk ? static_cast<int32_t>(s1) : -1;
-    }
+    __syncthreads();
+  }
+  if (warp == 0) {
+    best[0] = lane < kk ? scratch[0][lane] : 0ull;
+    best[1] = lane + 32 < kk ? scratch[0][32 + lane] : 0ull;
+    write_selection(out, best, kk, bt, k);
   }
 }
 
@@ -266,6 +355,14 @@ cudaError_t launch_block_topk(const msa_shape& s, const float* pooled, int32_t* 
   if (!ctx) return cudaErrorInitializationError;
   const long long rows = static_cast<long long>(s.batch) * s.seq_q * s.n_kv_heads;
   const int nb = static_cast<int>(ceil_div(s.seq_kv, 128));
+  // Few long rows (decode) leave most warps of the one-warp-per-row kernel
+  // idle: give each row a CTA instead.
+  if (rows <= 4LL * ctx->num_sms && nb > kChunk) {
+    ProfScope ps_("block_topk", st);
+    block_topk_row_cta_kernel<<<static_cast<unsigned>(rows), kWarps * 32, 0, st>>>(
+        pooled, sel, s.seq_q, s.n_kv_heads, s.q_offset, nb, s.topk);
+    return cudaGetLastError();
+  }
   long long blocks = (rows + kWarps - 1) / kWarps;
   const long long cap = static_cast<long long>(ctx->num_sms) * 32;
   if (blocks > cap) blocks = cap;

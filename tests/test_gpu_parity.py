@@ -91,6 +91,11 @@ def _random_pooled(sp, gen, lo, hi, integer=True):
     (spec(64, 1, 300000, 299999, 64, 8, 64, 64, 16), -50, 50),          # 2344 blocks: 3 chunks
     (spec(16, 1, 300000, 299999, 64, 8, 64, 64, 16), 0, 0),             # all equal, long rows
     (spec(1, 1500, 1500, 0, 8, 8, 64, 64, 1), -3, 3),                   # k = 1: local only
+    # few long rows: one CTA per row, lists merged across its warps
+    (spec(4, 1, 300000, 299999, 16, 8, 64, 64, 64), -5, 5),             # k = 64, heavy ties
+    (spec(3, 1, 300000, 299999, 16, 8, 64, 64, 33), -1000, 1000),       # k-1 = 32
+    (spec(2, 1, 1 << 20, (1 << 20) - 1, 64, 8, 64, 64, 16), -50, 50),   # 8192 blocks
+    (spec(8, 1, 140000, 139999, 64, 8, 64, 64, 16), -50, 50),           # 1094 blocks: 3 warps busy
 ])
 def test_topk_random_scores(sp, lo, hi):
     gen = torch.Generator().manual_seed(sp.seq_q + sp.topk)
