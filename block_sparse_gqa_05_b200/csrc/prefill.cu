@@ -212,6 +212,7 @@ struct AttnParams {
   PrefillWs w;
   uint32_t* err;
   int T, N, H, G, r, k, nb, q_off, tpt;
+  int q3d;   // r = 8, d = 128: one 3-D TMA load per token ([half][head][64] in smem)
   float scale_log2;
 };
 
@@ -339,33 +340,42 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           tma_prefetch_desc(&tm_k);
           tma_prefetch_desc(&tm_v);
         }
+        // running counters only: no division on this path
         int prev_col = -1;
-        long long u = -1;   // column ordinal
+        int u = -1;                    // column ordinal
+        int ib = 0, ms = 0;            // tile within its metadata batch, batch slot
+        uint32_t mph = 0;              // parity of that slot's barriers
+        int qb = 0;                    // query buffer
+        uint32_t qph = 0;              // its parity
+        const int nx = (tpt + 31) >> 5;
         for (long long i = 0; i < n; ++i) {
-          const long long bi = i / kmb;
-          const int ms = static_cast<int>(bi & 1);
-          const int slot = ms * kmb + static_cast<int>(i % kmb);
           int ok = 1;
-          if (i % kmb == 0) {
-            ok = mbar_wait(&mfull[ms], (bi >> 1) & 1, abort_flag, p.err) ? 1 : 0;
+          if (ib == 0) {
+            ok = mbar_wait(&mfull[ms], mph, abort_flag, p.err) ? 1 : 0;
             ok = __shfl_sync(0xffffffffu, ok, 0);
             if (!ok) break;
           }
-          const int col = tcol[ms * kMBMax + static_cast<int>(i % kmb)];
-          const bool last = tlast[ms * kMBMax + static_cast<int>(i % kmb)] != 0;
+          const int col = tcol[ms * kMBMax + ib];
+          const bool last = tlast[ms * kMBMax + ib] != 0;
+          const uint32_t* te = tent + (ms * kmb + ib) * tpt;
           uint32_t ent[4];
 #pragma unroll
           for (int x = 0; x < 4; ++x)
-            ent[x] = lane + 32 * x < tpt ? tent[slot * tpt + lane + 32 * x] : 0xFFFFFFFFu;
+            ent[x] = x < nx && lane + 32 * x < tpt ? te[lane + 32 * x] : 0xFFFFFFFFu;
           __syncwarp();
-          if (lane == 0 && (i % kmb == kmb - 1 || i + 1 == n)) mbar_arrive(&mempty[ms]);
-          const int bg = static_cast<int>(col / p.nb);
-          const int blk = static_cast<int>(col - static_cast<long long>(bg) * p.nb);
+          if (++ib == kmb || i + 1 == n) {
+            if (lane == 0) mbar_arrive(&mempty[ms]);
+            ib = 0;
+            ms ^= 1;
+            if (ms == 0) mph ^= 1u;
+          }
+          const int bg = col / p.nb;
+          const int blk = col - bg * p.nb;
           const bool newcol = col != prev_col;
           if (newcol) {
             prev_col = col;
             ++u;
-            const int st = static_cast<int>(u & 1);
+            const int st = u & 1;
             if (lane == 0) {
               ok = mbar_wait(&kempty[st], ((u >> 1) & 1) ^ 1, abort_flag, p.err) ? 1 : 0;
               if (ok) {
@@ -382,12 +392,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           int cnt = 0;
 #pragma unroll
           for (int x = 0; x < 4; ++x)
-            cnt += __popc(__ballot_sync(0xffffffffu, ent[x] != 0xFFFFFFFFu));
-          const int qb = static_cast<int>(i % kNQ);
+            if (x < nx) cnt += __popc(__ballot_sync(0xffffffffu, ent[x] != 0xFFFFFFFFu));
           if (lane == 0) {
-            ok = mbar_wait(&qempty[qb], ((i / kNQ) & 1) ^ 1, abort_flag, p.err) ? 1 : 0;
+            ok = mbar_wait(&qempty[qb], qph ^ 1u, abort_flag, p.err) ? 1 : 0;
             if (ok) {
-              meta[qb * 4 + 0] = static_cast<int>(u & 1);
+              meta[qb * 4 + 0] = u & 1;
               meta[qb * 4 + 1] = newcol ? 1 : 0;
               meta[qb * 4 + 2] = last ? 1 : 0;
               mbar_arrive_expect_tx(&qfull[qb], static_cast<uint32_t>(cnt * p.r * D * 2));
@@ -395,17 +404,28 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           }
           ok = __shfl_sync(0xffffffffu, ok, 0);
           if (!ok) break;
-          const int b = bg / p.G, g = bg % p.G;
+          const int b = bg / p.G, g = bg - b * p.G;
+          const int row0 = b * p.T * p.H + g * p.r;
+          uint8_t* qdst = smem + L::kOffQ + qb * L::kQ;
 #pragma unroll
           for (int x = 0; x < 4; ++x) {
             const int j = lane + 32 * x;
-            if (ent[x] != 0xFFFFFFFFu) {
-              const int row = (b * p.T + static_cast<int>(ent[x] >> 6)) * p.H + g * p.r;
+            if (x < nx && ent[x] != 0xFFFFFFFFu) {
+              const int row = row0 + static_cast<int>(ent[x] >> 6) * p.H;
+              if (p.q3d) {
+                // token j's 8 heads x 128 columns as [half][head][64]: two 1 KB
+                // swizzle atoms, 8-row groups 2 KB apart
+                tma_load_3d(qdst + j * 2048, &tm_q, &qfull[qb], 0, row, 0);
+              } else {
 #pragma unroll
-              for (int c = 0; c < D / 64; ++c)
-                tma_load_2d(smem + L::kOffQ + qb * L::kQ + c * 16384 + j * p.r * 128, &tm_q,
-                            &qfull[qb], c * 64, row);
+                for (int c = 0; c < D / 64; ++c)
+                  tma_load_2d(qdst + c * 16384 + j * p.r * 128, &tm_q, &qfull[qb], c * 64, row);
+              }
             }
+          }
+          if (++qb == kNQ) {
+            qb = 0;
+            qph ^= 1u;
           }
         }
       }
@@ -489,6 +509,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       // buffer of tile j-2, so it is issued only after PV(j-2); tcgen05 MMAs of
       // one thread execute in issue order, which makes that reuse safe.
       if (lane == 0 && n > 0) {
+        const bool q3d = p.q3d != 0;
         long long ns = 0, np = 0;   // next S, next PV
         long long u = -1;           // K column ordinal (S side)
         long long uv = -1;          // V column ordinal (PV side)
@@ -524,7 +545,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 #pragma unroll
               for (int ks = 0; ks < D / 16; ++ks) {
                 const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
-                tc_mma_ss(tS + sb * 128, smem_desc(qa + off, 16, 1024, 2),
+                const uint32_t qoff = q3d ? (ks >> 2) * 1024 + (ks & 3) * 32 : off;
+                tc_mma_ss(tS + sb * 128, smem_desc(qa + qoff, 16, q3d ? 2048 : 1024, 2),
                           smem_desc(ka + off, 16, 1024, 2), kIdescS, ks > 0 ? 1u : 0u);
               }
               tc_commit(&sfull[sb]);
@@ -649,15 +671,19 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     }
   } else {
     // ------------------------------------------------------------- epilogue
-    // O row (scaled by 1/l, bf16) -> swizzled staging tile -> one TMA store
-    // per token of r rows (the rows of a token's heads are contiguous).
+    // O row (scaled by 1/l, bf16) -> swizzled staging tile -> TMA stores of
+    // each token's r rows (the rows of a token's heads are contiguous): one
+    // 3-D store per token from a [token][half][head][64] staging layout when
+    // r = 8 and d = 128, else one 2-D store per 64-column half.
     regs_dec<96>();
     const int quarter = warp & 3;
     const int row = quarter * 32 + lane;
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
     const int tok = row / p.r, head = row % p.r;
+    const bool q3d = p.q3d != 0;
     uint8_t* stage = smem + L::kOffStage;
-    uint8_t* srow = stage + row * 128;
+    uint8_t* srow = q3d ? stage + tok * 2048 + head * 128 : stage + row * 128;
+    const uint32_t half_stride = q3d ? 1024u : 16384u;
     bool stored = false;   // this thread has bulk stores in flight
     for (long long i = 0; i < n; ++i) {
       const long long ti = t_begin + i;
@@ -692,7 +718,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           __nv_bfloat162 h2 = __floats2bfloat162_rn(ov[8 * x + 4] * il, ov[8 * x + 5] * il);
           __nv_bfloat162 h3 = __floats2bfloat162_rn(ov[8 * x + 6] * il, ov[8 * x + 7] * il);
           const int u = (c * 32 + 8 * x) >> 3;            // 16-byte unit of the row
-          uint4* dst = reinterpret_cast<uint4*>(srow + (u >> 3) * 16384 + (((u & 7) ^ (row & 7)) << 4));
+          uint4* dst = reinterpret_cast<uint4*>(srow + (u >> 3) * half_stride +
+                                                (((u & 7) ^ (row & 7)) << 4));
           *dst = make_uint4(*reinterpret_cast<uint32_t*>(&h0), *reinterpret_cast<uint32_t*>(&h1),
                             *reinterpret_cast<uint32_t*>(&h2), *reinterpret_cast<uint32_t*>(&h3));
         }
@@ -704,9 +731,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         const int b = bg / p.G, g = bg % p.G;
         const int t = static_cast<int>(e >> 6), slot = static_cast<int>(e & 63u);
         const int orow = ((b * p.T + t) * p.k + slot) * p.H + g * p.r;
+        if (q3d) {
+          tma_store_3d(&tm_o, stage + tok * 2048, 0, orow, 0);
+        } else {
 #pragma unroll
-        for (int c = 0; c < D / 64; ++c)
-          tma_store_2d(&tm_o, stage + c * 16384 + tok * p.r * 128, c * 64, orow);
+          for (int c = 0; c < D / 64; ++c)
+            tma_store_2d(&tm_o, stage + c * 16384 + tok * p.r * 128, c * 64, orow);
+        }
         bulk_commit_group();
         stored = true;
       }
@@ -783,8 +814,12 @@ cudaError_t launch_attn(const msa_shape& s, const uint16_t* q, const uint16_t* k
                         const uint16_t* v, const AttnParams& p, const DevCtx* ctx,
                         cudaStream_t st) {
   CUtensorMap tq, tk, tv, to;
-  const uint64_t dq[2] = {static_cast<uint64_t>(D),
-                          static_cast<uint64_t>(s.batch) * s.seq_q * s.n_q_heads};
+  const uint64_t rows = static_cast<uint64_t>(s.batch) * s.seq_q * s.n_q_heads;
+  const uint64_t dq[2] = {static_cast<uint64_t>(D), rows};
+  // [half of the row (stride 128 B)][row (stride 256 B)][64 columns]
+  const uint64_t dq3[3] = {64, rows, 2};
+  const uint64_t sq3[2] = {static_cast<uint64_t>(D) * 2, 128};
+  const uint32_t bq3[3] = {64, 8, 2};
   const uint64_t sq[1] = {static_cast<uint64_t>(D) * 2};
   const uint32_t bq[2] = {64, static_cast<uint32_t>(p.r)};
   const uint64_t dk[3] = {static_cast<uint64_t>(D), static_cast<uint64_t>(s.seq_kv),
@@ -792,16 +827,22 @@ cudaError_t launch_attn(const msa_shape& s, const uint16_t* q, const uint16_t* k
   const uint64_t sk[2] = {static_cast<uint64_t>(D) * 2,
                           static_cast<uint64_t>(s.seq_kv) * D * 2};
   const uint32_t bk[3] = {64, 128, 1};
-  const uint64_t dpo[2] = {static_cast<uint64_t>(D),
-                           static_cast<uint64_t>(s.batch) * s.seq_q * s.topk * s.n_q_heads};
-  if (!encode_tmap(&tq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, q, dq, sq, bq,
-                   CU_TENSOR_MAP_SWIZZLE_128B) ||
+  const uint64_t prow = static_cast<uint64_t>(s.batch) * s.seq_q * s.topk * s.n_q_heads;
+  const uint64_t dpo[2] = {static_cast<uint64_t>(D), prow};
+  const uint64_t dpo3[3] = {64, prow, 2};
+  const bool qmap = p.q3d ? encode_tmap(&tq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, q, dq3, sq3,
+                                        bq3, CU_TENSOR_MAP_SWIZZLE_128B)
+                           : encode_tmap(&tq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, q, dq, sq, bq,
+                                         CU_TENSOR_MAP_SWIZZLE_128B);
+  if (!qmap ||
       !encode_tmap(&tk, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, k, dk, sk, bk,
                    CU_TENSOR_MAP_SWIZZLE_128B) ||
       !encode_tmap(&tv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, v, dk, sk, bk,
                    CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !encode_tmap(&to, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, p.w.part_o, dpo, sq, bq,
-                   CU_TENSOR_MAP_SWIZZLE_128B))
+      !(p.q3d ? encode_tmap(&to, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, p.w.part_o, dpo3, sq3, bq3,
+                            CU_TENSOR_MAP_SWIZZLE_128B)
+              : encode_tmap(&to, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, p.w.part_o, dpo, sq, bq,
+                            CU_TENSOR_MAP_SWIZZLE_128B)))
     return cudaErrorInvalidValue;
   const size_t smem = AttnSmem<D>::kBytes;
   cudaError_t e = cudaFuncSetAttribute(kvouter_attn_kernel<D>,
@@ -868,6 +909,7 @@ cudaError_t launch_sparse_prefill(const msa_shape& s, const uint16_t* q, const u
   p.nb = nb;
   p.q_off = s.q_offset;
   p.tpt = tpt;
+  p.q3d = (r == 8 && s.head_dim == 128) ? 1 : 0;
   p.scale_log2 = kLog2e / sqrtf(static_cast<float>(s.head_dim));
   e = s.head_dim == 128 ? launch_attn<128>(s, q, k, v, p, ctx, st)
                         : launch_attn<64>(s, q, k, v, p, ctx, st);
