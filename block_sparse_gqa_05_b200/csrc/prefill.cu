@@ -12,8 +12,11 @@
 //     CTA that works on it and reused by every tile of its column; for a tile,
 //     S = Q K^T (TMEM), softmax over the block (causal mask on the local
 //     block), P (bf16, written back into TMEM), O_part = P V (TMEM) -> bf16
-//     partial plus its (max, sum) per (token, slot, head);
-//  4. combine the k partials of every (token, head).
+//     partial plus its (max, sum) per (token, slot, head), stored in the order
+//     of the column-sorted entry list, so a full tile's partials are one
+//     contiguous block (two TMA stores);
+//  4. combine the k partials of every (token, head), found through the
+//     position of each (token, group, slot) in the entry list.
 #include <math.h>
 
 #include "internal.h"
@@ -31,11 +34,12 @@ struct PrefillWs {
   uint32_t* col_fill;    // [ncol]
   uint32_t* col_off;     // [ncol + 1]
   uint32_t* tile_off;    // [ncol + 1]
-  uint32_t* entries;     // [B*T*G*k]   (t << 6) | slot
+  uint32_t* entries;     // [B*T*G*k]   (t << 6) | slot, sorted by column
+  uint32_t* inv;         // [B*T*G*k]   position in entries of each selected (t, g, slot)
   int4* tiles;           // [max_tiles] (column, entry start, count, 0)
   uint32_t* tile_ent;    // [max_tiles * tpt] entries of each tile, 0xFFFFFFFF past its count
-  uint16_t* part_o;      // [B, T, k, H, d] bf16 partial outputs, normalised by their own l
-  float* part_ml;        // [B, T, k, H, 2] (running max m, sum l) of each partial, log2 units
+  uint16_t* part_o;      // [entry, r, d] bf16 partial outputs, normalised by their own l
+  float* part_ml;        // [entry, r, 2] (running max m, sum l) of each partial, log2 units
   long long ncol, max_tiles;
 };
 
@@ -59,6 +63,7 @@ PrefillWs carve(const msa_shape& s, void* base) {
   w.col_off = reinterpret_cast<uint32_t*>(take(4 * (w.ncol + 1)));
   w.tile_off = reinterpret_cast<uint32_t*>(take(4 * (w.ncol + 1)));
   w.entries = reinterpret_cast<uint32_t*>(take(4 * nent));
+  w.inv = reinterpret_cast<uint32_t*>(take(4 * nent));
   w.tiles = reinterpret_cast<int4*>(take(16 * w.max_tiles));
   w.tile_ent = reinterpret_cast<uint32_t*>(take(4ull * w.max_tiles * tpt));
   w.part_o = reinterpret_cast<uint16_t*>(take(2ull * s.batch * s.seq_q * s.n_q_heads *
@@ -77,7 +82,7 @@ size_t carve_bytes(const msa_shape& s) {
   size_t b = 0;
   b += align_up(4 * ncol, 256) * 2;
   b += align_up(4 * (ncol + 1), 256) * 2;
-  b += align_up(4 * nent, 256);
+  b += align_up(4 * nent, 256) * 2;
   b += align_up(16 * max_tiles, 256);
   b += align_up(4ull * max_tiles * tpt, 256);
   b += align_up(2ull * s.batch * s.seq_q * s.n_q_heads * s.topk * s.head_dim, 256);
@@ -122,6 +127,7 @@ __global__ void __launch_bounds__(256) sel_invert_kernel(const int32_t* __restri
     if (c >= 0) {
       const uint32_t pos = base[c] + atomicAdd(&hist[c], 1u);
       w.entries[pos] = (static_cast<uint32_t>(t) << 6) | static_cast<uint32_t>(slot);
+      w.inv[((static_cast<long long>(b) * T + t) * G + g) * k + slot] = pos;
     }
   }
 }
@@ -230,10 +236,11 @@ struct AttnSmem {
   static constexpr uint32_t kOffStage = kOffQ + kNQ * kQ;   // epilogue staging (128 rows x D)
   static constexpr uint32_t kOffLinv = kOffStage + kQ;      // float [2][128]
   static constexpr uint32_t kOffMeta = kOffLinv + 1024;     // int [kNQ][4]
-  static constexpr uint32_t kOffTcol = kOffMeta + 64;       // int [2*kMBMax] column of each tile
-  static constexpr uint32_t kOffTlast = kOffTcol + 128;     // int [2*kMBMax] last tile of its column
-  static constexpr uint32_t kOffTent = kOffTlast + 128;     // uint [kTentWords] entries (tpt per tile)
-  static constexpr uint32_t kOffBar = kOffTent + kTentWords * 4;
+  // int4 [2*kMBMax] per tile: group (b*G+g), block, entries, flags (1: first
+  // tile of its column here, 2: last)
+  static constexpr uint32_t kOffThdr = kOffMeta + 64;
+  static constexpr uint32_t kOffTrow = kOffThdr + 2 * kMBMax * 16;   // int [kTentWords] query row
+  static constexpr uint32_t kOffBar = kOffTrow + kTentWords * 4;
   static constexpr uint32_t kBytes = kOffBar + 256;
 };
 
@@ -249,7 +256,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     kvouter_attn_kernel(const __grid_constant__ CUtensorMap tm_q,
                         const __grid_constant__ CUtensorMap tm_k,
                         const __grid_constant__ CUtensorMap tm_v,
-                        const __grid_constant__ CUtensorMap tm_o, const AttnParams p) {
+                        const __grid_constant__ CUtensorMap tm_o,
+                        const __grid_constant__ CUtensorMap tm_ot, const AttnParams p) {
   using L = AttnSmem<D>;
   constexpr uint32_t kIdescS = idesc_bf16(128, 128, 0, 0);   // Q (K-major) x K (K-major)
   constexpr uint32_t kIdescO = idesc_bf16(128, D, 0, 1);     // P (TMEM) x V (MN-major)
@@ -279,9 +287,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   uint64_t* lempty = sfull + 10;        // [2]
   uint64_t* mfull = sfull + 12;         // [2] metadata batch ready
   uint64_t* mempty = sfull + 14;        // [2] metadata batch consumed
-  int* tcol = reinterpret_cast<int*>(smem + L::kOffTcol);
-  int* tlast = reinterpret_cast<int*>(smem + L::kOffTlast);
-  uint32_t* tent = reinterpret_cast<uint32_t*>(smem + L::kOffTent);
+  int4* thdr = reinterpret_cast<int4*>(smem + L::kOffThdr);
+  int* trow = reinterpret_cast<int*>(smem + L::kOffTrow);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sfull + 16);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -340,8 +347,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           tma_prefetch_desc(&tm_k);
           tma_prefetch_desc(&tm_v);
         }
-        // running counters only: no division on this path
-        int prev_col = -1;
+        // running counters only, and every per-tile value prepared by the
+        // metadata warp: this loop is the pacing stage of the kernel
         int u = -1;                    // column ordinal
         int ib = 0, ms = 0;            // tile within its metadata batch, batch slot
         uint32_t mph = 0;              // parity of that slot's barriers
@@ -355,13 +362,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             ok = __shfl_sync(0xffffffffu, ok, 0);
             if (!ok) break;
           }
-          const int col = tcol[ms * kMBMax + ib];
-          const bool last = tlast[ms * kMBMax + ib] != 0;
-          const uint32_t* te = tent + (ms * kmb + ib) * tpt;
-          uint32_t ent[4];
+          const int4 hd = thdr[ms * kMBMax + ib];
+          const int* tr = trow + (ms * kmb + ib) * tpt;
+          int rows[4];
 #pragma unroll
-          for (int x = 0; x < 4; ++x)
-            ent[x] = x < nx && lane + 32 * x < tpt ? te[lane + 32 * x] : 0xFFFFFFFFu;
+          for (int x = 0; x < 4; ++x) rows[x] = x < nx && lane + 32 * x < tpt ? tr[lane + 32 * x] : -1;
           __syncwarp();
           if (++ib == kmb || i + 1 == n) {
             if (lane == 0) mbar_arrive(&mempty[ms]);
@@ -369,11 +374,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             ms ^= 1;
             if (ms == 0) mph ^= 1u;
           }
-          const int bg = col / p.nb;
-          const int blk = col - bg * p.nb;
-          const bool newcol = col != prev_col;
+          const bool newcol = (hd.w & 1) != 0;
           if (newcol) {
-            prev_col = col;
             ++u;
             const int st = u & 1;
             if (lane == 0) {
@@ -383,43 +385,37 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 #pragma unroll
                 for (int c = 0; c < D / 64; ++c)
                   tma_load_3d(smem + L::kOffK + st * L::kKV + c * 16384, &tm_k, &kfull[st],
-                              c * 64, blk * 128, bg);
+                              c * 64, hd.y * 128, hd.x);
               }
             }
             ok = __shfl_sync(0xffffffffu, ok, 0);
             if (!ok) break;
           }
-          int cnt = 0;
-#pragma unroll
-          for (int x = 0; x < 4; ++x)
-            if (x < nx) cnt += __popc(__ballot_sync(0xffffffffu, ent[x] != 0xFFFFFFFFu));
           if (lane == 0) {
             ok = mbar_wait(&qempty[qb], qph ^ 1u, abort_flag, p.err) ? 1 : 0;
             if (ok) {
               meta[qb * 4 + 0] = u & 1;
               meta[qb * 4 + 1] = newcol ? 1 : 0;
-              meta[qb * 4 + 2] = last ? 1 : 0;
-              mbar_arrive_expect_tx(&qfull[qb], static_cast<uint32_t>(cnt * p.r * D * 2));
+              meta[qb * 4 + 2] = (hd.w & 2) != 0 ? 1 : 0;
+              mbar_arrive_expect_tx(&qfull[qb], static_cast<uint32_t>(hd.z * p.r * D * 2));
             }
           }
           ok = __shfl_sync(0xffffffffu, ok, 0);
           if (!ok) break;
-          const int b = bg / p.G, g = bg - b * p.G;
-          const int row0 = b * p.T * p.H + g * p.r;
           uint8_t* qdst = smem + L::kOffQ + qb * L::kQ;
 #pragma unroll
           for (int x = 0; x < 4; ++x) {
             const int j = lane + 32 * x;
-            if (x < nx && ent[x] != 0xFFFFFFFFu) {
-              const int row = row0 + static_cast<int>(ent[x] >> 6) * p.H;
+            if (rows[x] >= 0) {
               if (p.q3d) {
                 // token j's 8 heads x 128 columns as [half][head][64]: two 1 KB
                 // swizzle atoms, 8-row groups 2 KB apart
-                tma_load_3d(qdst + j * 2048, &tm_q, &qfull[qb], 0, row, 0);
+                tma_load_3d(qdst + j * 2048, &tm_q, &qfull[qb], 0, rows[x], 0);
               } else {
 #pragma unroll
                 for (int c = 0; c < D / 64; ++c)
-                  tma_load_2d(qdst + c * 16384 + j * p.r * 128, &tm_q, &qfull[qb], c * 64, row);
+                  tma_load_2d(qdst + c * 16384 + j * p.r * 128, &tm_q, &qfull[qb], c * 64,
+                              rows[x]);
               }
             }
           }
@@ -432,16 +428,31 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       __syncwarp();
     } else if (warp == 2) {
       // ---------------------------------------------------------- metadata
-      // Batches of kmb tiles: descriptors and entries into the shared ring,
-      // all loads of a batch in flight together.
+      // Batches of kmb tiles into the shared ring: a header per tile (group,
+      // block, entries, first/last tile of its column) and the query row of
+      // every token, all loads of a batch in flight together.
+      const int tshift = __ffs(tpt) - 1;   // tpt = 128 / r is a power of two
+      int pcol = -1;                       // column of the previous batch's last tile
       for (long long bi = 0; bi * kmb < n; ++bi) {
         const int ms = static_cast<int>(bi & 1);
         if (!mbar_wait(&mempty[ms], ((bi >> 1) & 1) ^ 1, abort_flag, p.err)) break;
         const long long a = t_begin + bi * kmb;
         const int nt = static_cast<int>(min(static_cast<long long>(kmb), t_end - a));
-        // columns of the batch's tiles and of the tile after it
-        const int mycol = lane <= nt && a + lane < ntiles ? p.w.tiles[a + lane].x : -1;
-        const int nextcol = __shfl_down_sync(0xffffffffu, mycol, 1);
+        // the batch's tiles and, in lane nt, the tile after it (for its column)
+        int4 td = make_int4(-1, 0, 0, 0);
+        if (lane <= nt && a + lane < ntiles) td = p.w.tiles[a + lane];
+        const int col = td.x;
+        const int nextcol = __shfl_down_sync(0xffffffffu, col, 1);
+        int prvcol = __shfl_up_sync(0xffffffffu, col, 1);
+        if (lane == 0) prvcol = pcol;
+        const int bg = col >= 0 ? col / p.nb : 0;
+        const int b = bg / p.G, g = bg - b * p.G;
+        const int rowbase = b * p.T * p.H + g * p.r;
+        if (lane < nt) {
+          const int flags = (col != prvcol ? 1 : 0) |
+                            ((a + lane + 1 >= t_end || nextcol != col) ? 2 : 0);
+          thdr[ms * kMBMax + lane] = make_int4(bg, col - bg * p.nb, td.z, flags);
+        }
         // entries of tiles a .. a+nt-1 are contiguous: nt * tpt words
         const int nent = nt * tpt;
         for (int base = 0; base < nent; base += 8 * 32) {
@@ -454,13 +465,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 #pragma unroll
           for (int x = 0; x < 8; ++x) {
             const int idx = base + lane + 32 * x;
-            if (idx < nent) tent[(ms * kmb) * tpt + idx] = ev[x];
+            const int rb = __shfl_sync(0xffffffffu, rowbase, min(idx >> tshift, 31));
+            if (idx < nent)
+              trow[(ms * kmb) * tpt + idx] =
+                  ev[x] != 0xFFFFFFFFu ? rb + static_cast<int>(ev[x] >> 6) * p.H : -1;
           }
         }
-        if (lane < nt) {
-          tcol[ms * kMBMax + lane] = mycol;
-          tlast[ms * kMBMax + lane] = (a + lane + 1 >= t_end || nextcol != mycol) ? 1 : 0;
-        }
+        pcol = __shfl_sync(0xffffffffu, col, nt - 1);
         __syncwarp();
         mbar_arrive(&mfull[ms]);
       }
@@ -605,24 +616,22 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     const int tok = row / p.r, head = row % p.r;
     for (long long i = wg; i < n; i += 2) {
       const long long ti = t_begin + i;
-      const int col = p.w.tiles[ti].x;
+      const int2 cs = *reinterpret_cast<const int2*>(&p.w.tiles[ti]);   // column, entry start
+      const int col = cs.x;
       const uint32_t e = tok < tpt ? p.w.tile_ent[ti * tpt + tok] : 0xFFFFFFFFu;
       if (!mbar_wait(&sfull[wg], (i >> 1) & 1, abort_flag, p.err)) break;
       tc_fence_after();
       float sv[128];
 #pragma unroll
       for (int c = 0; c < 4; ++c) tmem_ld32(sbuf + c * 32, sv + c * 32);
-      const int bg = static_cast<int>(col / p.nb);
-      const int blk = static_cast<int>(col - static_cast<long long>(bg) * p.nb);
-      const int b = bg / p.G, g = bg % p.G;
+      const int blk = col - (col / p.nb) * p.nb;
       const bool valid = e != 0xFFFFFFFFu;
       int lim = 127;
-      long long prow = 0;
+      // partial row: entry (start + token) of the column-sorted list, head
+      const long long prow = (static_cast<long long>(cs.y) + tok) * p.r + head;
       if (valid) {
-        const int t = static_cast<int>(e >> 6), slot = static_cast<int>(e & 63u);
-        const int pos = p.q_off + t;
+        const int pos = p.q_off + static_cast<int>(e >> 6);
         if ((pos >> 7) == blk) lim = pos & 127;
-        prow = ((static_cast<long long>(b) * p.T + t) * p.k + slot) * p.H + g * p.r + head;
       }
       tc_wait_ld();
       // Only rows of the local block need the causal mask; the branch is
@@ -671,24 +680,21 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     }
   } else {
     // ------------------------------------------------------------- epilogue
-    // O row (scaled by 1/l, bf16) -> swizzled staging tile -> TMA stores of
-    // each token's r rows (the rows of a token's heads are contiguous): one
-    // 3-D store per token from a [token][half][head][64] staging layout when
-    // r = 8 and d = 128, else one 2-D store per 64-column half.
+    // O row (scaled by 1/l, bf16) -> swizzled staging tile -> TMA stores.
+    // Partials are stored in entry order, so the 128 rows of a full tile are
+    // one contiguous block: one store per 64-column half.  The last, partial
+    // tile of a column stores its tokens' r rows one token at a time.
     regs_dec<96>();
     const int quarter = warp & 3;
     const int row = quarter * 32 + lane;
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
     const int tok = row / p.r, head = row % p.r;
-    const bool q3d = p.q3d != 0;
     uint8_t* stage = smem + L::kOffStage;
-    uint8_t* srow = q3d ? stage + tok * 2048 + head * 128 : stage + row * 128;
-    const uint32_t half_stride = q3d ? 1024u : 16384u;
+    uint8_t* srow = stage + row * 128;
     bool stored = false;   // this thread has bulk stores in flight
     for (long long i = 0; i < n; ++i) {
       const long long ti = t_begin + i;
-      const int col = p.w.tiles[ti].x;
-      const uint32_t e = tok < tpt ? p.w.tile_ent[ti * tpt + tok] : 0xFFFFFFFFu;
+      const int4 td = p.w.tiles[ti];   // column, entry start, entries
       const int ob = static_cast<int>(i & 1);
       if (!mbar_wait(&ofull[ob], (i >> 1) & 1, abort_flag, p.err)) break;
       if (!mbar_wait(&lfull[ob], (i >> 1) & 1, abort_flag, p.err)) break;
@@ -718,7 +724,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           __nv_bfloat162 h2 = __floats2bfloat162_rn(ov[8 * x + 4] * il, ov[8 * x + 5] * il);
           __nv_bfloat162 h3 = __floats2bfloat162_rn(ov[8 * x + 6] * il, ov[8 * x + 7] * il);
           const int u = (c * 32 + 8 * x) >> 3;            // 16-byte unit of the row
-          uint4* dst = reinterpret_cast<uint4*>(srow + (u >> 3) * half_stride +
+          uint4* dst = reinterpret_cast<uint4*>(srow + (u >> 3) * 16384 +
                                                 (((u & 7) ^ (row & 7)) << 4));
           *dst = make_uint4(*reinterpret_cast<uint32_t*>(&h0), *reinterpret_cast<uint32_t*>(&h1),
                             *reinterpret_cast<uint32_t*>(&h2), *reinterpret_cast<uint32_t*>(&h3));
@@ -726,18 +732,17 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       }
       fence_proxy_async_smem();
       named_bar_sync(1, 128);
-      if (head == 0 && e != 0xFFFFFFFFu) {
-        const int bg = static_cast<int>(col / p.nb);
-        const int b = bg / p.G, g = bg % p.G;
-        const int t = static_cast<int>(e >> 6), slot = static_cast<int>(e & 63u);
-        const int orow = ((b * p.T + t) * p.k + slot) * p.H + g * p.r;
-        if (q3d) {
-          tma_store_3d(&tm_o, stage + tok * 2048, 0, orow, 0);
-        } else {
+      if (td.z == tpt) {
+        if (row == 0) {
 #pragma unroll
-          for (int c = 0; c < D / 64; ++c)
-            tma_store_2d(&tm_o, stage + c * 16384 + tok * p.r * 128, c * 64, orow);
+          for (int c = 0; c < D / 64; ++c) tma_store_2d(&tm_ot, stage + c * 16384, c * 64, td.y * p.r);
+          bulk_commit_group();
+          stored = true;
         }
+      } else if (head == 0 && tok < td.z) {
+#pragma unroll
+        for (int c = 0; c < D / 64; ++c)
+          tma_store_2d(&tm_o, stage + c * 16384 + tok * p.r * 128, c * 64, (td.y + tok) * p.r);
         bulk_commit_group();
         stored = true;
       }
@@ -757,7 +762,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 // One CTA per (sequence, token): merge the k partials of each of the H heads.
 // Partial s of a row holds the normalised output O_s (bf16), its running max
 // m_s and sum l_s = sum_j 2^(x_j - m_s) (x in log2 units).  With M = max_s m_s
-// and w_s = 2^(m_s - M) l_s:  o = sum_s w_s O_s / sum_s w_s.
+// and w_s = 2^(m_s - M) l_s:  o = sum_s w_s O_s / sum_s w_s.  The partial of
+// (group g, slot s) sits at entry inv[t, g, s] of the column-sorted list.
 template <int D>
 __global__ void __launch_bounds__(256) combine_kernel(const int32_t* __restrict__ sel,
                                                       const PrefillWs w, uint16_t* __restrict__ o,
@@ -765,17 +771,24 @@ __global__ void __launch_bounds__(256) combine_kernel(const int32_t* __restrict_
                                                       int r, int k) {
   constexpr int CH = D / 8;                  // 16-byte chunks per head row
   extern __shared__ float2 sm_ml[];          // [k][H] (m, l), m = -inf for unused slots
+  uint32_t* sm_pos = reinterpret_cast<uint32_t*>(sm_ml + k * H);   // [G][k] entry of each slot
   const long long bt = blockIdx.x;           // b*T + t
-  const float2* msrc = reinterpret_cast<const float2*>(w.part_ml) + bt * k * H;
+  const float2* ml_all = reinterpret_cast<const float2*>(w.part_ml);
   const int32_t* srow = sel + bt * G * k;
+  const uint32_t* irow = w.inv + bt * G * k;
+  for (int x = threadIdx.x; x < G * k; x += blockDim.x)
+    sm_pos[x] = srow[x] >= 0 ? irow[x] : 0xFFFFFFFFu;
+  __syncthreads();
   for (int x = threadIdx.x; x < k * H; x += blockDim.x) {
-    const int s = x / H, h = x % H;
-    sm_ml[x] = srow[(h / r) * k + s] >= 0 ? msrc[x] : make_float2(-INFINITY, 0.f);
+    const int s = x / H, h = x % H, g = h / r;
+    const uint32_t pos = sm_pos[g * k + s];
+    sm_ml[x] = pos != 0xFFFFFFFFu ? ml_all[static_cast<long long>(pos) * r + (h - g * r)]
+                                  : make_float2(-INFINITY, 0.f);
   }
   __syncthreads();
-  const uint16_t* osrc = w.part_o + bt * k * H * D;
   for (int item = threadIdx.x; item < H * CH; item += blockDim.x) {
     const int h = item / CH, c = item % CH;
+    const int g = h / r, hh = h - g * r;
     float M = -INFINITY;
     for (int s = 0; s < k; ++s) M = fmaxf(M, sm_ml[s * H + h].x);
     float acc[8];
@@ -788,7 +801,8 @@ __global__ void __launch_bounds__(256) combine_kernel(const int32_t* __restrict_
       if (ml.x == -INFINITY) continue;
       const float ws = exp2f(ml.x - M) * ml.y;
       den += ws;
-      const uint4 u = __ldcs(reinterpret_cast<const uint4*>(osrc + (static_cast<long long>(s) * H + h) * D) + c);
+      const long long prow = static_cast<long long>(sm_pos[g * k + s]) * r + hh;
+      const uint4 u = __ldcs(reinterpret_cast<const uint4*>(w.part_o + prow * D) + c);
       const uint32_t wds[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
@@ -813,7 +827,7 @@ template <int D>
 cudaError_t launch_attn(const msa_shape& s, const uint16_t* q, const uint16_t* k,
                         const uint16_t* v, const AttnParams& p, const DevCtx* ctx,
                         cudaStream_t st) {
-  CUtensorMap tq, tk, tv, to;
+  CUtensorMap tq, tk, tv, to, tot;
   const uint64_t rows = static_cast<uint64_t>(s.batch) * s.seq_q * s.n_q_heads;
   const uint64_t dq[2] = {static_cast<uint64_t>(D), rows};
   // [half of the row (stride 128 B)][row (stride 256 B)][64 columns]
@@ -827,9 +841,10 @@ cudaError_t launch_attn(const msa_shape& s, const uint16_t* q, const uint16_t* k
   const uint64_t sk[2] = {static_cast<uint64_t>(D) * 2,
                           static_cast<uint64_t>(s.seq_kv) * D * 2};
   const uint32_t bk[3] = {64, 128, 1};
+  // partial rows: (entry, head) with entries in column order
   const uint64_t prow = static_cast<uint64_t>(s.batch) * s.seq_q * s.topk * s.n_q_heads;
   const uint64_t dpo[2] = {static_cast<uint64_t>(D), prow};
-  const uint64_t dpo3[3] = {64, prow, 2};
+  const uint32_t bpt[2] = {64, 128};
   const bool qmap = p.q3d ? encode_tmap(&tq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, q, dq3, sq3,
                                         bq3, CU_TENSOR_MAP_SWIZZLE_128B)
                            : encode_tmap(&tq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, q, dq, sq, bq,
@@ -839,10 +854,10 @@ cudaError_t launch_attn(const msa_shape& s, const uint16_t* q, const uint16_t* k
                    CU_TENSOR_MAP_SWIZZLE_128B) ||
       !encode_tmap(&tv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, v, dk, sk, bk,
                    CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !(p.q3d ? encode_tmap(&to, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, p.w.part_o, dpo3, sq3, bq3,
-                            CU_TENSOR_MAP_SWIZZLE_128B)
-              : encode_tmap(&to, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, p.w.part_o, dpo, sq, bq,
-                            CU_TENSOR_MAP_SWIZZLE_128B)))
+      !encode_tmap(&to, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, p.w.part_o, dpo, sq, bq,
+                   CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !encode_tmap(&tot, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, p.w.part_o, dpo, sq, bpt,
+                   CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorInvalidValue;
   const size_t smem = AttnSmem<D>::kBytes;
   cudaError_t e = cudaFuncSetAttribute(kvouter_attn_kernel<D>,
@@ -851,7 +866,7 @@ cudaError_t launch_attn(const msa_shape& s, const uint16_t* q, const uint16_t* k
   if (e != cudaSuccess) return e;
   {
     ProfScope ps_("kvouter_attn", st);
-    kvouter_attn_kernel<D><<<ctx->num_sms, kAttnThreads, smem, st>>>(tq, tk, tv, to, p);
+    kvouter_attn_kernel<D><<<ctx->num_sms, kAttnThreads, smem, st>>>(tq, tk, tv, to, tot, p);
   }
   return cudaGetLastError();
 }
@@ -915,7 +930,7 @@ cudaError_t launch_sparse_prefill(const msa_shape& s, const uint16_t* q, const u
                         : launch_attn<64>(s, q, k, v, p, ctx, st);
   if (e != cudaSuccess) return e;
   const unsigned ntok = static_cast<unsigned>(static_cast<long long>(s.batch) * s.seq_q);
-  const size_t csmem = sizeof(float2) * s.topk * s.n_q_heads;
+  const size_t csmem = sizeof(float2) * s.topk * s.n_q_heads + 4u * s.n_kv_heads * s.topk;
   {
     ProfScope ps_("combine", st);
     if (s.head_dim == 128)

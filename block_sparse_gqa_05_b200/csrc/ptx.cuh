@@ -178,6 +178,20 @@ MSA_DEV void bulk_load(void* smem_dst, const void* gsrc, uint32_t bytes, uint64_
       : "memory");
 }
 
+// 16-byte asynchronous copy global -> shared through L2 (cp.async, LSU path).
+MSA_DEV void cp_async16(void* smem_dst, const void* gsrc) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;"
+               ::"r"(smem_u32(smem_dst)), "l"(reinterpret_cast<uint64_t>(gsrc))
+               : "memory");
+}
+
+// Arrive on ``bar`` once every cp.async this thread issued so far has landed
+// (the arrival is one of the barrier's expected arrivals).
+MSA_DEV void cp_async_arrive_noinc(uint64_t* bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar))
+               : "memory");
+}
+
 // Generic-proxy shared-memory writes -> visible to the async proxy (tensor core).
 MSA_DEV void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
