@@ -223,6 +223,7 @@ struct AttnParams {
 };
 
 constexpr int kNQ = 3;        // query tile buffers
+constexpr int kNS = 3;        // S/P buffers in TMEM (128 columns each)
 constexpr int kMBMax = 16;    // most tiles per metadata batch (two batches in flight)
 constexpr int kTentWords = 256; // entry words in the metadata ring (both batches)
 
@@ -248,9 +249,11 @@ struct AttnSmem {
 // idle), WG1 and WG2 = softmax of alternate tiles, WG3 = epilogue.  Register
 // budget per thread is moved from WG0/WG3 to the softmax warpgroups so that a
 // softmax thread holds its whole 128-score row.
-// TMEM: S/P buffers at columns [0,128) and [128,256) (P is written over the
-// first 64 columns of its tile's S as packed bf16 and consumed from there by
-// the PV MMA), O buffers at [256, 256+D) and [256+D, 256+2D).
+// TMEM: three S/P buffers at columns [0,384) (P is written over the first 64
+// columns of its tile's S as packed bf16 and consumed from there by the PV
+// MMA), so S(j+1) and S(j+2) can be computed while tile j's softmax runs;
+// then the O buffers: one of 128 columns for d = 128 (the epilogue drains it
+// long before the next PV completes), two of 64 for d = 64.
 template <int D>
 __global__ void __launch_bounds__(kAttnThreads, 1)
     kvouter_attn_kernel(const __grid_constant__ CUtensorMap tm_q,
@@ -262,6 +265,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   constexpr uint32_t kIdescS = idesc_bf16(128, 128, 0, 0);   // Q (K-major) x K (K-major)
   constexpr uint32_t kIdescO = idesc_bf16(128, D, 0, 1);     // P (TMEM) x V (MN-major)
   constexpr uint32_t kTmemCols = 512;
+  constexpr int kNO = D == 128 ? 1 : 2;    // O buffers: kNS*128 + kNO*D = 512 columns
+  static_assert(kNS * 128 + kNO * D <= static_cast<int>(kTmemCols), "TMEM columns");
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   // the swizzled operand tiles need 1024-byte alignment; the launch reserves no slack
   if ((smem_u32(smem_raw) & 1023u) != 0) {
@@ -279,17 +284,17 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   uint64_t* vempty = bars + 5;          // V tile free (last PV of its column done)
   uint64_t* qfull = bars + 6;           // [kNQ]
   uint64_t* qempty = bars + 6 + kNQ;    // [kNQ]
-  uint64_t* sfull = bars + 6 + 2 * kNQ; // [2]
-  uint64_t* pfull = sfull + 2;          // [2]
-  uint64_t* ofull = sfull + 4;          // [2]
-  uint64_t* ofree = sfull + 6;          // [2]
-  uint64_t* lfull = sfull + 8;          // [2]
-  uint64_t* lempty = sfull + 10;        // [2]
-  uint64_t* mfull = sfull + 12;         // [2] metadata batch ready
-  uint64_t* mempty = sfull + 14;        // [2] metadata batch consumed
+  uint64_t* sfull = bars + 6 + 2 * kNQ; // [kNS]
+  uint64_t* pfull = sfull + kNS;        // [kNS]
+  uint64_t* ofull = pfull + kNS;        // [kNO]
+  uint64_t* ofree = ofull + 2;          // [kNO]
+  uint64_t* lfull = ofree + 2;          // [2]
+  uint64_t* lempty = lfull + 2;         // [2]
+  uint64_t* mfull = lempty + 2;         // [2] metadata batch ready
+  uint64_t* mempty = mfull + 2;         // [2] metadata batch consumed
   int4* thdr = reinterpret_cast<int4*>(smem + L::kOffThdr);
   int* trow = reinterpret_cast<int*>(smem + L::kOffTrow);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sfull + 16);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mempty + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -301,11 +306,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   const int tpt = p.tpt;
 
   if (threadIdx.x == 0) {
+    for (int i = 0; i < kNS; ++i) {
+      mbar_init(&sfull[i], 1);
+      mbar_init(&pfull[i], 128);
+    }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&kfull[i], 1);
       mbar_init(&kempty[i], 1);
-      mbar_init(&sfull[i], 1);
-      mbar_init(&pfull[i], 128);
       mbar_init(&ofull[i], 1);
       mbar_init(&ofree[i], 128);
       mbar_init(&lfull[i], 128);
@@ -331,8 +338,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t tS = tmem;          // S/P buffers
-  const uint32_t tO = tmem + 256;    // O buffers
+  const uint32_t tS = tmem;                // kNS S/P buffers of 128 columns
+  const uint32_t tO = tmem + kNS * 128;    // kNO O buffers of D columns
 
   if (wgid == 0) {
     regs_dec<56>();
@@ -517,8 +524,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       // Two in-order streams, S(j) = Q K^T and PV(i) = P V, issued by one
       // thread as soon as each is ready (polling), so a query gather that is
       // late never holds back the PV of an earlier tile.  S(j) reuses the S/P
-      // buffer of tile j-2, so it is issued only after PV(j-2); tcgen05 MMAs of
-      // one thread execute in issue order, which makes that reuse safe.
+      // buffer of tile j-kNS, so it is issued only after PV(j-kNS); tcgen05 MMAs
+      // of one thread execute in issue order, which makes that reuse safe.
       if (lane == 0 && n > 0) {
         const bool q3d = p.q3d != 0;
         long long ns = 0, np = 0;   // next S, next PV
@@ -534,7 +541,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         while (np < n) {
           bool progress = false;
           // ---- S(ns)
-          if (ns < n && ns < np + 2) {
+          if (ns < n && ns < np + kNS) {
             const int qb = static_cast<int>(ns % kNQ);
             if (!s_meta && mbar_test(&qfull[qb], (ns / kNQ) & 1)) {
               s_st = meta[qb * 4 + 0];
@@ -552,7 +559,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
               tc_fence_after();
               const uint32_t qa = smem_u32(smem + L::kOffQ + qb * L::kQ);
               const uint32_t ka = smem_u32(smem + L::kOffK + st * L::kKV);
-              const int sb = static_cast<int>(ns & 1);
+              const int sb = static_cast<int>(ns % kNS);
 #pragma unroll
               for (int ks = 0; ks < D / 16; ++ks) {
                 const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
@@ -570,20 +577,21 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           }
           // ---- PV(np)
           if (np < ns) {
-            const int sb = static_cast<int>(np & 1);
+            const int sb = static_cast<int>(np % kNS);
+            const int ob = static_cast<int>(np % kNO);
             const bool need_v = first_of_col[np & 3];
             if ((!need_v || mbar_test(vfull, (uv + 1) & 1)) &&
-                mbar_test(&pfull[sb], (np >> 1) & 1) &&
-                mbar_test(&ofree[sb], ((np >> 1) & 1) ^ 1)) {
+                mbar_test(&pfull[sb], (np / kNS) & 1) &&
+                mbar_test(&ofree[ob], ((np / kNO) & 1) ^ 1)) {
               if (need_v) ++uv;
               tc_fence_after();
               const uint32_t va = smem_u32(smem + L::kOffV);
 #pragma unroll
               for (int ks = 0; ks < 8; ++ks) {   // 128 keys in steps of 16 (8 packed columns)
                 const uint64_t bd = smem_desc(va + ks * 16 * 128, 16384, 1024, 2);
-                tc_mma_ts(tO + sb * D, tS + sb * 128 + ks * 8, bd, kIdescO, ks > 0 ? 1u : 0u);
+                tc_mma_ts(tO + ob * D, tS + sb * 128 + ks * 8, bd, kIdescO, ks > 0 ? 1u : 0u);
               }
-              tc_commit(&ofull[sb]);
+              tc_commit(&ofull[ob]);
               if (last_of_col[np & 3]) tc_commit(vempty);
               ++np;
               progress = true;
@@ -612,14 +620,16 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     const int quarter = warp & 3;
     const int row = quarter * 32 + lane;
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
-    const uint32_t sbuf = tS + wg * 128 + lane_off;
+    const uint32_t sbase = tS + lane_off;
     const int tok = row / p.r, head = row % p.r;
     for (long long i = wg; i < n; i += 2) {
       const long long ti = t_begin + i;
       const int2 cs = *reinterpret_cast<const int2*>(&p.w.tiles[ti]);   // column, entry start
       const int col = cs.x;
       const uint32_t e = tok < tpt ? p.w.tile_ent[ti * tpt + tok] : 0xFFFFFFFFu;
-      if (!mbar_wait(&sfull[wg], (i >> 1) & 1, abort_flag, p.err)) break;
+      const int sb = static_cast<int>(i % kNS);
+      const uint32_t sbuf = sbase + sb * 128;
+      if (!mbar_wait(&sfull[sb], (i / kNS) & 1, abort_flag, p.err)) break;
       tc_fence_after();
       float sv[128];
 #pragma unroll
@@ -671,7 +681,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       const float l = ((l8[0] + l8[1]) + (l8[2] + l8[3])) + ((l8[4] + l8[5]) + (l8[6] + l8[7]));
       tc_wait_st();
       tc_fence_before();
-      mbar_arrive(&pfull[wg]);
+      mbar_arrive(&pfull[sb]);
       if (valid) reinterpret_cast<float2*>(p.w.part_ml)[prow] = make_float2(mxs, l);
       // 1/l for the epilogue of this tile
       if (!mbar_wait(&lempty[wg], ((i >> 1) & 1) ^ 1, abort_flag, p.err)) break;
@@ -695,12 +705,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     for (long long i = 0; i < n; ++i) {
       const long long ti = t_begin + i;
       const int4 td = p.w.tiles[ti];   // column, entry start, entries
-      const int ob = static_cast<int>(i & 1);
-      if (!mbar_wait(&ofull[ob], (i >> 1) & 1, abort_flag, p.err)) break;
-      if (!mbar_wait(&lfull[ob], (i >> 1) & 1, abort_flag, p.err)) break;
+      const int ob = static_cast<int>(i % kNO);
+      const int lb = static_cast<int>(i & 1);   // softmax warpgroup of this tile
+      if (!mbar_wait(&ofull[ob], (i / kNO) & 1, abort_flag, p.err)) break;
+      if (!mbar_wait(&lfull[lb], (i >> 1) & 1, abort_flag, p.err)) break;
       tc_fence_after();
-      const float il = linv[ob * 128 + row];
-      mbar_arrive(&lempty[ob]);
+      const float il = linv[lb * 128 + row];
+      mbar_arrive(&lempty[lb]);
       // the staging tile must be free: own stores read out, then everyone's
       if (stored) {
         bulk_wait_read0();
