@@ -265,6 +265,15 @@ def run_msa(args, world, rank, pg):
                             "frac": round(a / pk, 4)}
     out["stages"] = stages
 
+    # ---- the same workload through the dense causal GQA kernel (the baseline
+    # the pages compare MSA against)
+    if not args.skip_dense:
+        def dstep():
+            M.dense_attn_prefill(sh, inp.q, inp.k, inp.v, o=o, lse=None, want_lse=False)
+        dms = timed_loop(dstep, 2, 1, pg, stream)
+        out["dense_gqa_prefill"] = {"ms_per_step": dms, "value": tokens * world / (dms / 1e3),
+                                    "speedup_msa_vs_dense": round(dms / ms, 2)}
+
     # ---- end to end through the public API with host buffers
     if not args.skip_e2e:
         host = {n: getattr(inp, n).cpu().pin_memory() for n in ("q", "k", "v", "q_idx", "k_idx")}
@@ -546,6 +555,7 @@ def main():
     ap.add_argument("--skip-cpu", action="store_true")
     ap.add_argument("--skip-e2e", action="store_true")
     ap.add_argument("--skip-topk-micro", action="store_true")
+    ap.add_argument("--skip-dense", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--ref-step-s", type=float, default=4.0)
     args = ap.parse_args()
