@@ -583,7 +583,7 @@ def main():
                 "gpu_launches": res["gpu_launches"], "roofline": res["roofline"],
                 "stages": res["stages"], "kernels_ms_per_launch": res["kernels_ms_per_launch"],
                 "clocks": res["clocks"]}
-        for key in ("e2e", "topk_microbench", "decode", "ctx_1m"):
+        for key in ("e2e", "dense_gqa_prefill", "topk_microbench", "decode", "ctx_1m"):
             if key in res:
                 line[key] = res[key]
         if world == 1 and not args.skip_cpu:
