@@ -27,9 +27,6 @@ MSA_DEV uint64_t globaltimer() {
   return t;
 }
 
-MSA_DEV uint32_t lane_id() { return threadIdx.x & 31u; }
-MSA_DEV uint32_t warp_id() { return threadIdx.x >> 5; }
-
 // ------------------------------------------------------------------ mbarrier
 MSA_DEV void mbar_init(uint64_t* bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count)
@@ -118,25 +115,11 @@ MSA_DEV void tma_load_3d(void* smem_dst, const CUtensorMap* m, uint64_t* bar, in
       : "memory");
 }
 
-// Prefetch a 2D box into L2 (no shared-memory destination).
-MSA_DEV void tma_prefetch_l2_2d(const CUtensorMap* m, int x, int y) {
-  asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];"
-               ::"l"(reinterpret_cast<uint64_t>(m)), "r"(x), "r"(y)
-               : "memory");
-}
-
 // 2D tensor store shared -> global (bulk-group completion).
 MSA_DEV void tma_store_2d(const CUtensorMap* m, const void* smem_src, int x, int y) {
   asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];"
                ::"l"(reinterpret_cast<uint64_t>(m)), "r"(smem_u32(smem_src)), "r"(x), "r"(y)
                : "memory");
-}
-// 3D tensor store shared -> global (bulk-group completion).
-MSA_DEV void tma_store_3d(const CUtensorMap* m, const void* smem_src, int x, int y, int z) {
-  asm volatile(
-      "cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%2, %3, %4}], [%1];"
-      ::"l"(reinterpret_cast<uint64_t>(m)), "r"(smem_u32(smem_src)), "r"(x), "r"(y), "r"(z)
-      : "memory");
 }
 MSA_DEV void bulk_commit_group() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 // Wait until every committed bulk store of this thread has finished reading shared memory.
@@ -168,29 +151,6 @@ template <uint32_t N>
 MSA_DEV void regs_dec() { asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N)); }
 template <uint32_t N>
 MSA_DEV void regs_inc() { asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N)); }
-
-// Untiled bulk copy global -> shared (both 16-byte aligned, bytes % 16 == 0).
-MSA_DEV void bulk_load(void* smem_dst, const void* gsrc, uint32_t bytes, uint64_t* bar) {
-  asm volatile(
-      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
-      ::"r"(smem_u32(smem_dst)), "l"(reinterpret_cast<uint64_t>(gsrc)), "r"(bytes),
-        "r"(smem_u32(bar))
-      : "memory");
-}
-
-// 16-byte asynchronous copy global -> shared through L2 (cp.async, LSU path).
-MSA_DEV void cp_async16(void* smem_dst, const void* gsrc) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;"
-               ::"r"(smem_u32(smem_dst)), "l"(reinterpret_cast<uint64_t>(gsrc))
-               : "memory");
-}
-
-// Arrive on ``bar`` once every cp.async this thread issued so far has landed
-// (the arrival is one of the barrier's expected arrivals).
-MSA_DEV void cp_async_arrive_noinc(uint64_t* bar) {
-  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar))
-               : "memory");
-}
 
 // Generic-proxy shared-memory writes -> visible to the async proxy (tensor core).
 MSA_DEV void fence_proxy_async_smem() {
