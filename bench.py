@@ -45,10 +45,11 @@ def load_peaks():
     return dict(PEAKS_FALLBACK), "fallback"
 
 
-def src_hash():
+def src_hash(files=None):
+    """Hash of the library sources a kernel is built from (all of them by default)."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "block_sparse_gqa_05_b200", "csrc")
-    for f in sorted(os.listdir(csrc)):
+    for f in sorted(files or os.listdir(csrc)):
         h.update(open(os.path.join(csrc, f), "rb").read())
     return h.hexdigest()[:16]
 
@@ -59,10 +60,10 @@ def ncu_traffic(kernel):
     if not os.path.exists(p):
         return None
     d = json.load(open(p))
-    if d.get("src_sha") != src_hash():
-        return None
     e = d.get("kernels", {}).get(kernel)
-    return None if e is None else e.get("bytes_per_launch_full")
+    if e is None or e.get("src_sha") != src_hash(e.get("sources")):
+        return None   # the kernel changed since the counters were taken
+    return e.get("bytes_per_launch_full")
 
 
 class ClockSampler:
