@@ -127,11 +127,15 @@ def dist_setup(args):
     if world > 1:
         import datetime
         import torch.distributed as dist
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(minutes=10),
-                                device_id=torch.device("cuda", local))
+        # NCCL between the GPUs; gloo on a host without GPUs (the CPU tests)
+        if torch.cuda.is_available():
+            torch.cuda.set_device(local)
+            dist.init_process_group("nccl", timeout=datetime.timedelta(minutes=10),
+                                    device_id=torch.device("cuda", local))
+        else:
+            dist.init_process_group("gloo", timeout=datetime.timedelta(minutes=2))
         pg = dist
-    else:
+    elif torch.cuda.is_available():
         torch.cuda.set_device(0)
     return world, rank, local, pg
 
@@ -139,9 +143,17 @@ def dist_setup(args):
 def max_over_ranks(x, pg):
     if pg is None:
         return x
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if pg.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     pg.all_reduce(t, op=pg.ReduceOp.MAX)
     return float(t.item())
+
+
+def rank_workload(name, rank):
+    """The named workload with its seed offset by rank: every rank runs an
+    independent sequence (weak scaling, no exchange inside the layer)."""
+    sp = synth.workload(name)
+    return synth.workload(name, seed=sp.seed + 1000 * rank)
 
 
 def barrier(pg):
@@ -199,8 +211,7 @@ def run_msa(args, world, rank, pg):
     peaks, peak_src = load_peaks()
     stream = torch.cuda.current_stream()
     out = {}
-    sp = synth.workload(args.workload)
-    sp = synth.workload(args.workload, seed=sp.seed + 1000 * rank)   # independent per rank
+    sp = rank_workload(args.workload, rank)
     inp = synth.make_inputs(sp, "cuda")
     sh = M.Shape.of(sp)
     ws = M.alloc_workspace(sh, M.OP_FORWARD)
@@ -345,9 +356,8 @@ def run_msa(args, world, rank, pg):
         out["topk_microbench"] = run_topk_micro(M, args, stream, peaks)
     # ---- decode at 128K, batch 32
     if not args.skip_decode:
-        dw = synth.workload(args.decode_workload)
-        out["decode"] = run_decode(M, synth.workload(args.decode_workload, seed=dw.seed + 1000 * rank),
-                                   args, pg, stream, world, peaks, dense=False)
+        out["decode"] = run_decode(M, rank_workload(args.decode_workload, rank), args, pg, stream,
+                                   world, peaks, dense=False)
     # ---- 1M context: prefill chunk + decode, against the dense kernels
     if not args.skip_long:
         out["ctx_1m"] = run_long(M, args, pg, stream, world, rank, peaks)
@@ -449,7 +459,7 @@ def run_decode(M, sp, args, pg, stream, world, peaks, dense):
 
 def run_long(M, args, pg, stream, world, rank, peaks):
     res = {}
-    sp = synth.workload("prefill_1m_chunk8k", seed=5 + 1000 * rank)
+    sp = rank_workload("prefill_1m_chunk8k", rank)
     inp = synth.make_inputs(sp, "cuda")
     sh = M.Shape.of(sp)
     ws = M.alloc_workspace(sh, M.OP_FORWARD)
@@ -486,7 +496,7 @@ def run_long(M, args, pg, stream, world, rank, peaks):
     res["prefill"] = pre
     del inp, ws, o, sel
     torch.cuda.empty_cache()
-    res["decode"] = run_decode(M, synth.workload("decode_1m_b4", seed=6 + 1000 * rank), args, pg,
+    res["decode"] = run_decode(M, rank_workload("decode_1m_b4", rank), args, pg,
                                stream, world, peaks, dense=True)
     return res
 
