@@ -36,6 +36,7 @@ constexpr float kLog2e = 1.4426950408889634f;
 struct DecParams {
   const uint16_t* q;      // [B, 1, H, d]
   const int32_t* sel;     // [B, 1, G, k] (sparse) or nullptr (dense)
+  const int32_t* lens;    // [B] cache lengths (ragged decode) or nullptr: all N
   uint16_t* o;            // [B, 1, H, d]
   float* lse;             // [B, 1, H] or nullptr
   uint32_t* counters;     // [B*G] CTAs done with a (sequence, group)
@@ -99,12 +100,18 @@ __device__ __forceinline__ uint32_t sw128_off(int row, int col) {
   return static_cast<uint32_t>(chunk * (128 * 128) + row * 128 + unit * 16 + (c & 7) * 2);
 }
 
+// Query position of sequence b: the last row of its cache.
+__device__ __forceinline__ int query_pos(const DecParams& p, int b) {
+  return p.lens ? ragged_len(p.lens, b, p.N, p.err) - 1 : p.N - 1;
+}
+
 // Block of item i (-1 when it has nothing to attend to: an empty selection
 // slot or a block past the query), and its (sequence, group) in *bg.
-__device__ __forceinline__ int item_block(const DecParams& p, long long i, int bt, int* bg) {
+__device__ __forceinline__ int item_block(const DecParams& p, long long i, int* bg) {
   const int g = static_cast<int>(i / p.per_bg);
   const int j = static_cast<int>(i - static_cast<long long>(g) * p.per_bg);
   *bg = g;
+  const int bt = query_pos(p, g / p.G) >> 7;
   const int blk = p.sel ? __ldg(p.sel + static_cast<long long>(g) * p.k + j) : j;
   return (blk >= 0 && blk <= bt) ? blk : -1;
 }
@@ -139,8 +146,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   const long long n = p.n_items, grid = gridDim.x;
   const long long i0 = cta_first(blockIdx.x, n, grid);
   const long long i1 = cta_first(blockIdx.x + 1, n, grid);
-  const int pos = p.N - 1;
-  const int bt = pos >> 7;
 
   // the swizzled K/V tiles need 1024-byte alignment; the launch reserves no slack
   if ((smem_u32(smem) & 1023u) != 0u) {
@@ -168,7 +173,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool ok = true;
     for (long long base = i0; ok && base < i1; base += 32) {
       int bgv = 0;
-      const int blk = base + lane < i1 ? item_block(p, base + lane, bt, &bgv) : -1;
+      const int blk = base + lane < i1 ? item_block(p, base + lane, &bgv) : -1;
       unsigned m = __ballot_sync(0xffffffffu, blk >= 0);
       while (m) {
         const int src = __ffs(m) - 1;
@@ -218,6 +223,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t pbase = smem_u32(ps);
   int cnt = 0;
   int cur_bg = -1;
+  int pos = 0;                     // query position of the current sequence
   long long seg_first = 0;
   bool failed = false;
   uint32_t qa[KS][4];
@@ -277,7 +283,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   for (long long base = i0; !failed && base < i1; base += 32) {
     int bgv = 0;
-    const int blkv = base + lane < i1 ? item_block(p, base + lane, bt, &bgv) : -1;
+    const int blkv = base + lane < i1 ? item_block(p, base + lane, &bgv) : -1;
     const int nin = static_cast<int>(min(32LL, i1 - base));
     for (int jj = 0; jj < nin; ++jj) {
       const int blk = __shfl_sync(0xffffffffu, blkv, jj);
@@ -285,6 +291,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (bg != cur_bg) {
         if (cur_bg >= 0) finish(cur_bg, seg_first, base + jj);
         cur_bg = bg;
+        pos = query_pos(p, bg / p.G);
         seg_first = base + jj;
         const int b = bg / p.G, g = bg % p.G;
         const uint16_t* qb = p.q + (static_cast<long long>(b) * p.H + g * p.r) * D;
@@ -538,7 +545,7 @@ size_t decode_workspace_bytes(const msa_shape& s, bool dense) {
 
 cudaError_t launch_decode(const msa_shape& s, const uint16_t* q, const uint16_t* k,
                           const uint16_t* v, const int32_t* sel, uint16_t* o, float* lse,
-                          void* ws, bool dense, cudaStream_t st) {
+                          void* ws, bool dense, cudaStream_t st, const int32_t* lens) {
   const DevCtx* ctx = device_ctx();
   if (!ctx) return cudaErrorInitializationError;
   const int r = s.n_q_heads / s.n_kv_heads;
@@ -555,6 +562,7 @@ cudaError_t launch_decode(const msa_shape& s, const uint16_t* q, const uint16_t*
   p.part_o = reinterpret_cast<float*>(w + align_up(bg * 4, 256) + align_up(slots * r * 4, 256));
   p.q = q;
   p.sel = dense ? nullptr : sel;
+  p.lens = lens;
   p.o = o;
   p.lse = lse;
   p.err = ctx->err;

@@ -284,13 +284,16 @@ template <int DI>
 __global__ void __launch_bounds__(256) index_scores_scan_kernel(const uint16_t* __restrict__ q_idx,
                                                                 const uint16_t* __restrict__ k_idx,
                                                                 float* __restrict__ pooled, int T,
-                                                                int N, int G, int q_off, int nb) {
+                                                                int N, int G, int q_off, int nb,
+                                                                const int32_t* __restrict__ lens,
+                                                                uint32_t* err) {
   constexpr int KS = DI / 16;          // k-steps
   constexpr int W = KS * 2;            // 32-bit words per thread per row
   const int row_bt = blockIdx.y;       // seq * T + t
   const int seq = row_bt / T;
   const int t = row_bt - seq * T;
-  const int pos = q_off + t;
+  // ragged decode: the query sits at the end of its own cache
+  const int pos = lens ? ragged_len(lens, seq, N, err) - 1 : q_off + t;
   const int bt = pos >> 7;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int blk = blockIdx.x * 8 + warp;
@@ -419,14 +422,16 @@ cudaError_t launch_tc(const msa_shape& s, const uint16_t* q_idx, const uint16_t*
 }  // namespace
 
 cudaError_t launch_index_scores(const msa_shape& s, const uint16_t* q_idx, const uint16_t* k_idx,
-                                float* pooled, bool fill_upper, cudaStream_t st) {
+                                float* pooled, bool fill_upper, cudaStream_t st,
+                                const int32_t* lens) {
   const DevCtx* ctx = device_ctx();
   if (!ctx) return cudaErrorInitializationError;
   const int nb = static_cast<int>(ceil_div(s.seq_kv, 128));
   const long long rows = static_cast<long long>(s.batch) * s.seq_q * s.n_kv_heads;
   cudaError_t e;
-  // the tensor-core path needs a full 128-row query tile and a 256-key box
-  if (static_cast<long long>(s.seq_q) * s.n_kv_heads < 128 ||
+  // the tensor-core path needs a full 128-row query tile and a 256-key box;
+  // ragged decode always scans
+  if (lens || static_cast<long long>(s.seq_q) * s.n_kv_heads < 128 ||
       static_cast<long long>(s.batch) * s.seq_kv < 256) {
     const int last_bt = (s.q_offset + s.seq_q - 1) / 128;
     dim3 grid(static_cast<unsigned>(ceil_div(last_bt + 1, 8)),
@@ -435,13 +440,15 @@ cudaError_t launch_index_scores(const msa_shape& s, const uint16_t* q_idx, const
       {
     ProfScope ps_("index_scores_scan", st);
     index_scores_scan_kernel<64><<<grid, 256, 0, st>>>(q_idx, k_idx, pooled, s.seq_q, s.seq_kv,
-                                                         s.n_kv_heads, s.q_offset, nb);
+                                                         s.n_kv_heads, s.q_offset, nb, lens,
+                                                         ctx->err);
   }
     else
       {
     ProfScope ps_("index_scores_scan", st);
     index_scores_scan_kernel<32><<<grid, 256, 0, st>>>(q_idx, k_idx, pooled, s.seq_q, s.seq_kv,
-                                                         s.n_kv_heads, s.q_offset, nb);
+                                                         s.n_kv_heads, s.q_offset, nb, lens,
+                                                         ctx->err);
   }
     e = cudaGetLastError();
   } else {

@@ -14,11 +14,21 @@ namespace msa {
 
 // Device error word bits.
 constexpr uint32_t kErrTimeout = 1u;
+constexpr uint32_t kErrBadLength = 2u;   // a ragged-decode cache length outside [1, N]
 // Bound of every mbarrier wait, in nanoseconds of %globaltimer.
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 
 MSA_DEV uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+// Cache length of sequence b in ragged decode: lens[b] clamped into [1, N];
+// a length outside that range also sets kErrBadLength in the error word.
+MSA_DEV int ragged_len(const int32_t* lens, int b, int N, uint32_t* err) {
+  const int len = lens[b];
+  if (len >= 1 && len <= N) return len;
+  atomicOr(err, kErrBadLength);
+  return len < 1 ? 1 : N;
 }
 
 MSA_DEV uint64_t globaltimer() {

@@ -281,7 +281,8 @@ MSA_DEV bool write_trivial(int32_t* out, int n, int kk, int bt, int k) {
 // One warp per row: for many rows (prefill).
 __global__ void __launch_bounds__(kWarps * 32, 3)
     block_topk_kernel(const float* __restrict__ pooled, int32_t* __restrict__ sel,
-                      long long rows, int T, int G, int q_off, int nb, int k) {
+                      long long rows, int T, int G, int q_off, int nb, int k,
+                      const int32_t* __restrict__ lens, int N, uint32_t* err) {
   __shared__ uint64_t scratch[kWarps][kScratch];
   const int warp = threadIdx.x >> 5;
   uint64_t* buf = scratch[warp];
@@ -289,9 +290,11 @@ __global__ void __launch_bounds__(kWarps * 32, 3)
   const bool vec = (nb & 3) == 0;
   for (long long r = static_cast<long long>(blockIdx.x) * kWarps + warp; r < rows; r += nwarps) {
     // rows < 2^31 (checked by the API): 32-bit index math
-    const int t = static_cast<int>((static_cast<uint32_t>(r) / static_cast<uint32_t>(G)) %
-                                   static_cast<uint32_t>(T));
-    const int bt = (q_off + t) >> 7;
+    const uint32_t tg = static_cast<uint32_t>(r) / static_cast<uint32_t>(G);
+    const int t = static_cast<int>(tg % static_cast<uint32_t>(T));
+    const int pos = lens ? ragged_len(lens, static_cast<int>(tg / static_cast<uint32_t>(T)), N, err) - 1
+                         : q_off + t;
+    const int bt = pos >> 7;
     const int n = bt;                         // candidates 0 .. bt-1
     const int kk = min(k - 1, n);
     int32_t* out = sel + r * k;
@@ -308,13 +311,16 @@ __global__ void __launch_bounds__(kWarps * 32, 3)
 // merge keeps the 64 best of two sorted lists of at most 63).
 __global__ void __launch_bounds__(kWarps * 32)
     block_topk_row_cta_kernel(const float* __restrict__ pooled, int32_t* __restrict__ sel,
-                              int T, int G, int q_off, int nb, int k) {
+                              int T, int G, int q_off, int nb, int k,
+                              const int32_t* __restrict__ lens, int N, uint32_t* err) {
   __shared__ uint64_t scratch[kWarps][kScratch];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const long long r = blockIdx.x;
-  const int t = static_cast<int>((static_cast<uint32_t>(r) / static_cast<uint32_t>(G)) %
-                                 static_cast<uint32_t>(T));
-  const int bt = (q_off + t) >> 7;
+  const uint32_t tg = static_cast<uint32_t>(r) / static_cast<uint32_t>(G);
+  const int t = static_cast<int>(tg % static_cast<uint32_t>(T));
+  const int pos = lens ? ragged_len(lens, static_cast<int>(tg / static_cast<uint32_t>(T)), N, err) - 1
+                       : q_off + t;
+  const int bt = pos >> 7;
   const int n = bt;
   const int kk = min(k - 1, n);
   int32_t* out = sel + r * k;
@@ -350,7 +356,7 @@ __global__ void __launch_bounds__(kWarps * 32)
 }  // namespace
 
 cudaError_t launch_block_topk(const msa_shape& s, const float* pooled, int32_t* sel,
-                              cudaStream_t st) {
+                              cudaStream_t st, const int32_t* lens) {
   const DevCtx* ctx = device_ctx();
   if (!ctx) return cudaErrorInitializationError;
   const long long rows = static_cast<long long>(s.batch) * s.seq_q * s.n_kv_heads;
@@ -360,7 +366,7 @@ cudaError_t launch_block_topk(const msa_shape& s, const float* pooled, int32_t* 
   if (rows <= 4LL * ctx->num_sms && nb > kChunk) {
     ProfScope ps_("block_topk", st);
     block_topk_row_cta_kernel<<<static_cast<unsigned>(rows), kWarps * 32, 0, st>>>(
-        pooled, sel, s.seq_q, s.n_kv_heads, s.q_offset, nb, s.topk);
+        pooled, sel, s.seq_q, s.n_kv_heads, s.q_offset, nb, s.topk, lens, s.seq_kv, ctx->err);
     return cudaGetLastError();
   }
   long long blocks = (rows + kWarps - 1) / kWarps;
@@ -369,7 +375,8 @@ cudaError_t launch_block_topk(const msa_shape& s, const float* pooled, int32_t* 
   {
     ProfScope ps_("block_topk", st);
     block_topk_kernel<<<static_cast<unsigned>(blocks), kWarps * 32, 0, st>>>(
-      pooled, sel, rows, s.seq_q, s.n_kv_heads, s.q_offset, nb, s.topk);
+      pooled, sel, rows, s.seq_q, s.n_kv_heads, s.q_offset, nb, s.topk, lens, s.seq_kv,
+      ctx->err);
   }
   return cudaGetLastError();
 }

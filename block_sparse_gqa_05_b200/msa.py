@@ -62,6 +62,8 @@ _SIGS = {
                                       ctypes.c_int),
     "msa_forward": ([ctypes.POINTER(Shape), _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
                      ctypes.c_size_t, _vp], ctypes.c_int),
+    "msa_forward_decode_ragged": ([ctypes.POINTER(Shape), _vp, _vp, _vp, _vp, _vp, _vp, _vp,
+                                   _vp, _vp, _vp, ctypes.c_size_t, _vp], ctypes.c_int),
     "msa_dense_attn_prefill": ([ctypes.POINTER(Shape), _vp, _vp, _vp, _vp, _vp, _vp,
                                 ctypes.c_size_t, _vp], ctypes.c_int),
     "msa_dense_attn_decode": ([ctypes.POINTER(Shape), _vp, _vp, _vp, _vp, _vp, _vp,
@@ -202,6 +204,23 @@ def forward(shape: Shape, q, k, v, q_idx, k_idx, o=None, lse=None, sel=None, ws=
     return o, lse, sel
 
 
+def forward_decode_ragged(shape: Shape, q, k, v, q_idx, k_idx, seq_lens, o=None, lse=None,
+                          sel=None, ws=None, want_lse=True, want_sel=True, stream=None):
+    """msa_forward_decode_ragged: one decode step over caches of different
+    lengths.  seq_lens: int32 CUDA tensor [B], each in [1, shape.seq_kv]
+    (shape.seq_kv is the cache capacity)."""
+    o, lse = _attn_out(shape, q, o, lse, want_lse)
+    if sel is None and want_sel:
+        sel = torch.empty((shape.batch, 1, shape.n_kv_heads, shape.topk), dtype=torch.int32,
+                          device=q.device)
+    ws = alloc_workspace(shape, OP_FORWARD, q.device) if ws is None else ws
+    _check(lib().msa_forward_decode_ragged(ctypes.byref(shape), _ptr(seq_lens), _ptr(q), _ptr(k),
+                                           _ptr(v), _ptr(q_idx), _ptr(k_idx), _ptr(o), _ptr(lse),
+                                           _ptr(sel), _ptr(ws), ws.numel(), _stream(stream)),
+           "msa_forward_decode_ragged")
+    return o, lse, sel
+
+
 def dense_attn_prefill(shape: Shape, q, k, v, o=None, lse=None, want_lse=True, stream=None):
     o, lse = _attn_out(shape, q, o, lse, want_lse)
     _check(lib().msa_dense_attn_prefill(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(o),
@@ -242,7 +261,8 @@ def profile_read() -> dict:
 
 
 def device_status() -> int:
-    """Raw device error word (0 = no bounded wait expired); clears it."""
+    """Raw device error word (bit 0: a bounded wait expired; bit 1: a ragged-decode
+    cache length was out of range); clears it."""
     f = ctypes.c_uint32(0)
     st = lib().msa_device_status(ctypes.byref(f))
     if st not in (0, 7):

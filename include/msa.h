@@ -153,6 +153,23 @@ msa_status msa_forward(const msa_shape* shape, const uint16_t* q, const uint16_t
                        uint16_t* o, float* lse, int32_t* sel_out, void* ws,
                        size_t ws_bytes, void* stream);
 
+/* Whole layer for one decode step over caches of different lengths (the
+ * pages' decode step, batched for serving; no other counterpart on them):
+ * as msa_forward with T == 1, except that sequence b's caches hold
+ * seq_lens[b] valid rows and its query sits at position seq_lens[b] - 1, so
+ * its local block is (seq_lens[b] - 1) / 128 and only its causal blocks are
+ * scored and selected.  seq_lens: device int32 [B], 4-byte aligned, each in
+ * [1, seq_kv]; shape.seq_kv is the cache capacity (row stride of k, v,
+ * k_idx) and shape.q_offset is ignored.  A length outside [1, seq_kv] is
+ * clamped into it and sets bit 1 of the device error word.  Same layouts,
+ * outputs and workspace (msa_workspace_size(MSA_OP_FORWARD) with T == 1) as
+ * msa_forward. */
+msa_status msa_forward_decode_ragged(const msa_shape* shape, const int32_t* seq_lens,
+                                     const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                                     const uint16_t* q_idx, const uint16_t* k_idx, uint16_t* o,
+                                     float* lse, int32_t* sel_out, void* ws, size_t ws_bytes,
+                                     void* stream);
+
 /* Dense causal GQA attention (every key x <= p_t), the baseline the pages
  * compare MSA against ([P1] GQA definition; [P2], [P4] speed-ups vs GQA).
  * Prefill: q-outer flash attention, no workspace needed (pass NULL/0). */
@@ -191,7 +208,8 @@ msa_status msa_sparse_attn_decode_static(const msa_shape* shape, const uint16_t*
                                          void* stream);
 
 /* Reads and clears the device error word of the current device (bit 0: a
- * bounded wait timed out).  Synchronises the current device.  Returns
+ * bounded wait timed out; bit 1: a ragged-decode cache length was out of
+ * range).  Synchronises the current device.  Returns
  * MSA_ERR_DEVICE_TIMEOUT if any bit was set, MSA_OK otherwise; *flags (may be
  * NULL) receives the raw word. */
 msa_status msa_device_status(uint32_t* flags);

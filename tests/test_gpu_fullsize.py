@@ -123,6 +123,33 @@ def run_case(name, n_pool_rows, n_attn_rows):
     torch.cuda.empty_cache()
 
 
+def test_ragged_decode_full_size():
+    """32 sequences in a 128K-capacity cache with seeded lengths in [1, 131072]
+    (both ends included): whole selection against the host re-sort, every
+    output against the oracle."""
+    sp = synth.workload("decode_128k_b32")
+    inp = synth.make_inputs(sp, "cuda")
+    sh = M.Shape.of(sp)
+    rng = np.random.default_rng(7)
+    lens = rng.integers(1, sp.seq_kv + 1, size=sp.batch)
+    lens[:3] = [1, 128, sp.seq_kv]
+    seq_lens = torch.tensor(lens, dtype=torch.int32, device="cuda")
+    o, _, sel = M.forward_decode_ragged(sh, inp.q, inp.k, inp.v, inp.q_idx, inp.k_idx, seq_lens,
+                                        want_lse=False)
+    torch.cuda.synchronize()
+    assert M.device_status() == 0
+    for b in range(sp.batch):
+        pos = np.array([int(lens[b]) - 1])
+        pooled = O.index_pooled(inp.q_idx[b].cpu(), inp.k_idx[b].cpu(), pos, sp.block)
+        ref = host_resort(torch.from_numpy(pooled).float(), pos, sp.block, sp.topk)
+        assert torch.equal(sel[b].cpu(), ref), f"b={b} len={lens[b]}"
+        assert np.array_equal(ref.numpy(), O.block_topk(pooled, pos, sp.block, sp.topk))
+        ref_o = compact_attention_ref(sp, inp.q[b, 0].cpu(), inp.k[b], inp.v[b],
+                                      sel[b, 0].cpu().numpy(), int(pos[0]))
+        err = np.abs(ref_o - o[b, 0].double().cpu().numpy())
+        assert err.max() <= MAX_ABS and err.mean() <= MEAN_ABS, (b, err.max(), err.mean())
+
+
 @pytest.mark.parametrize("name,n_pool,n_attn", [
     ("prefill_32k", 48, 48),
     ("prefill_128k", 48, 48),

@@ -243,3 +243,52 @@ def test_forward_decode():
 
 def test_device_status_clean():
     assert M.device_status() == 0
+
+
+# ------------------------------------------------- ragged batched decode
+def _ragged_case(sp, lens):
+    inp = inputs_cpu(sp)
+    sh = M.Shape.of(sp)
+    seq_lens = cuda(torch.tensor(lens, dtype=torch.int32))
+    o, lse, sel = M.forward_decode_ragged(sh, cuda(inp.q), cuda(inp.k), cuda(inp.v),
+                                          cuda(inp.q_idx), cuda(inp.k_idx), seq_lens)
+    torch.cuda.synchronize()
+    return inp, o, lse, sel
+
+
+@pytest.mark.parametrize("sp,lens", [
+    (spec(6, 1, 9000, 8999, 16, 4, 128, 64, 16, seed=51, planted=4),
+     [1, 127, 128, 129, 5000, 9000]),
+    (spec(5, 1, 3000, 2999, 8, 4, 64, 32, 4, seed=52), [2, 300, 640, 2999, 3000]),
+])
+def test_forward_decode_ragged(sp, lens):
+    inp, o, lse, sel = _ragged_case(sp, lens)
+    assert M.device_status() == 0
+    o_ref, l_ref = [], []
+    for b, n in enumerate(lens):
+        pos = np.array([n - 1])
+        pooled = O.index_pooled(inp.q_idx[b], inp.k_idx[b], pos, sp.block)
+        sref = O.block_topk(pooled, pos, sp.block, sp.topk)
+        assert np.array_equal(sel[b].cpu().numpy(), sref), f"sel b={b} len={n}"
+        ob, lb = O.sparse_attention(inp.q[b], inp.k[b], inp.v[b], sref, pos, sp.block)
+        o_ref.append(ob)
+        l_ref.append(lb)
+    # the tolerance applies to the call's whole output (a sequence with two
+    # keys alone has too few values for a mean)
+    check_attn(o, np.stack(o_ref), "ragged decode")
+    assert np.abs(lse.double().cpu().numpy() - np.stack(l_ref)).max() < LSE_ABS
+
+
+def test_forward_decode_ragged_length_out_of_range():
+    # lengths 0 and capacity+5 are clamped to 1 and capacity; the kernels flag them
+    sp = spec(2, 1, 1000, 999, 8, 2, 64, 32, 4, seed=53)
+    inp, o, lse, sel = _ragged_case(sp, [0, 1005])
+    flags = M.device_status()
+    assert flags & 2, flags
+    for b, n in enumerate([1, 1000]):
+        pos = np.array([n - 1])
+        sref = O.block_topk(O.index_pooled(inp.q_idx[b], inp.k_idx[b], pos, sp.block), pos,
+                            sp.block, sp.topk)
+        assert np.array_equal(sel[b].cpu().numpy(), sref)
+        O_ref, _ = O.sparse_attention(inp.q[b], inp.k[b], inp.v[b], sref, pos, sp.block)
+        check_attn(o[b], O_ref, f"clamped ragged decode b={b}")
