@@ -24,6 +24,10 @@ Attention (MSA) : attention block-sparse à deux branches…"):
    group's selection (P3: Q1/Q2/Q3 share I1, Q4/Q5/Q6 share I2).
 4. ``dense_attention`` -- causal GQA (P1, GQA definition) for the
    "k >= number of causal blocks" invariant and the dense baseline.
+5. ``index_alignment_kl`` -- the divergence P1 (bullet "KL Loss Alignment")
+   trains the index branch on, computed forward-only as a diagnostic: the
+   main branch's attention distribution over the selected blocks against the
+   index branch's distribution over the same blocks.
 
 Readings where the pages are silent (each listed in the design notes):
   * index score: raw dot product, no scale / activation (P3 names only Q_idx.K_idx;
@@ -38,6 +42,11 @@ Readings where the pages are silent (each listed in the design notes):
   * selection is decided on the pooled scores rounded to float32 (the
     kernel's precision); with the integer-valued index inputs of the workloads
     every score is an exact integer, so this rounding is the identity.
+
+  * alignment (P1 gives no formula): per (query, group), P_main(b) = the
+    attention mass of selected block b averaged over the group's heads,
+    P_index(b) = softmax over the selected blocks of the raw pooled index
+    scores (no temperature), KL(P_main || P_index) in natural log.
 
 Precision: float64 throughout.  Parity of the attention outputs is unpinned
 beyond the special cases the tests check (dense equivalence, closed forms).
@@ -194,6 +203,33 @@ def msa_forward(q, k, v, q_idx, k_idx, positions, block: int, topk: int):
     sel = block_topk(pooled, positions, block, topk)
     O, L = sparse_attention(q, k, v, sel, positions, block)
     return O, L, sel, pooled
+
+
+def index_alignment_kl(q, k, v, sel, pooled, positions, block: int,
+                       scale: float | None = None) -> np.ndarray:
+    """KL(P_main || P_index) per (query row, group), float64 [R, G].
+
+    P_main(b): for each head of group g, the sum of its attention weights
+    (``sparse_attention``'s normalised weights) over the keys of selected
+    block b, averaged over the group's heads.  P_index(b): softmax over the
+    selected blocks of pooled[r, g, b].  Terms with P_main(b) = 0 contribute 0.
+    """
+    sl = np.asarray(sel)
+    pl = _f64(pooled)
+    R, G, _ = sl.shape
+    _, _, weights = sparse_attention(q, k, v, sel, positions, block, scale, return_weights=True)
+    out = np.zeros((R, G))
+    for i in range(R):
+        for g in range(G):
+            keys, w = weights[i][g]                       # w [r, n] rows sum to 1
+            blocks = [int(b) for b in sl[i, g] if b >= 0]
+            p_main = np.array([w[:, (keys // block) == b].sum(axis=1).mean() for b in blocks])
+            logits = np.array([pl[i, g, b] for b in blocks])
+            p_idx = np.exp(logits - logits.max())
+            p_idx /= p_idx.sum()
+            nz = p_main > 0
+            out[i, g] = float(np.sum(p_main[nz] * (np.log(p_main[nz]) - np.log(p_idx[nz]))))
+    return out
 
 
 def attention_flops_ratio(n_ctx: int, H: int, d: int, G: int, d_idx: int,

@@ -259,3 +259,51 @@ def test_topk_selection_on_planted_synthetic_block():
     sel = O.block_topk(O.index_pooled(qi, ki, pos, B), pos, B, k=2)
     assert np.all(sel[:, 0, 0] == 3)
     assert np.all(sel[:, 0, 1] == pos // B)
+
+
+# ------------------------------------------------------- alignment diagnostic
+
+def test_alignment_single_block_is_zero():
+    # k = 1: both distributions sit on the local block alone
+    rng = np.random.default_rng(3)
+    q = rng.standard_normal((1, 4, 8))
+    k = rng.standard_normal((2, 40, 8))
+    v = rng.standard_normal((2, 40, 8))
+    sel = np.array([[[3], [3]]], dtype=np.int32)
+    pooled = rng.standard_normal((1, 2, 5))
+    kl = O.index_alignment_kl(q, k, v, sel, pooled, np.array([29]), 8)
+    assert np.all(kl == 0.0)
+
+
+def test_alignment_uniform_keys_closed_form():
+    # identical keys -> uniform attention over the attended keys: block masses
+    # are key counts (8, 8, and the 6 causal keys 24..29 of local block 3);
+    # equal pooled scores -> uniform index distribution over the 3 blocks
+    B, N, d = 8, 40, 4
+    rng = np.random.default_rng(4)
+    q = rng.standard_normal((1, 2, d))
+    k = np.tile(rng.standard_normal((1, 1, d)), (1, N, 1))
+    v = rng.standard_normal((1, N, d))
+    sel = np.array([[[0, 2, 3]]], dtype=np.int32)
+    pooled = np.full((1, 1, 5), 7.0)
+    kl = O.index_alignment_kl(q, k, v, sel, pooled, np.array([29]), B)
+    p = np.array([8, 8, 6]) / 22.0
+    assert kl[0, 0] == pytest.approx(float(np.sum(p * np.log(p * 3.0))), rel=1e-12)
+
+
+def test_alignment_averages_heads_and_direction():
+    # head 0 sees only block 0, head 1 only block 1 -> P_main = (1/2, 1/2);
+    # index logits (log 3, 0) -> P_index = (3/4, 1/4);
+    # KL(P_main || P_index) = 1/2 log(4/3) (the reverse direction differs)
+    B, N, d = 8, 16, 2
+    k = np.zeros((1, N, d))
+    k[0, :8, 0] = 50.0
+    k[0, 8:, 1] = 50.0
+    q = np.array([[[20.0, 0.0], [0.0, 20.0]]])
+    v = np.zeros((1, N, d))
+    sel = np.array([[[0, 1]]], dtype=np.int32)
+    pooled = np.array([[[math.log(3.0), 0.0]]])
+    kl = O.index_alignment_kl(q, k, v, sel, pooled, np.array([15]), B)
+    assert kl[0, 0] == pytest.approx(0.5 * math.log(4.0 / 3.0), abs=1e-12)
+    reverse = 0.75 * math.log(1.5) + 0.25 * math.log(0.5)
+    assert abs(kl[0, 0] - reverse) > 1e-3
