@@ -240,6 +240,10 @@ msa_status msa_workspace_size(const msa_shape* s, msa_op op, size_t* bytes) {
       return MSA_OK;
     case MSA_OP_DENSE_PREFILL:
       return check_shape(s, true, false);
+    case MSA_OP_FORWARD_ALIGNMENT:
+      if ((st = check_shape(s, true, true)) != MSA_OK) return st;
+      *bytes = pooled_bytes(*s) + sel_bytes(*s) + prefill_workspace_bytes(*s);
+      return MSA_OK;
   }
   return MSA_ERR_UNSUPPORTED;
 }
@@ -350,6 +354,34 @@ msa_status msa_forward(const msa_shape* s, const uint16_t* q, const uint16_t* k,
     else
       e = launch_sparse_prefill(*s, q, k, v, sel, o, lse, rest, cs);
   }
+  return from_cuda(e);
+}
+
+msa_status msa_forward_alignment(const msa_shape* s, const uint16_t* q, const uint16_t* k,
+                                 const uint16_t* v, const uint16_t* q_idx,
+                                 const uint16_t* k_idx, uint16_t* o, float* lse,
+                                 int32_t* sel_out, float* kl, void* ws, size_t ws_bytes,
+                                 void* stream) {
+  msa_status st = check_shape(s, true, true);
+  if (st != MSA_OK) return st;
+  if ((st = check_attn_ptrs(q, k, v, nullptr, false, o, lse)) != MSA_OK) return st;
+  if (!q_idx || !k_idx || !kl) return MSA_ERR_NULL_PTR;
+  if (!aligned16(q_idx) || !aligned16(k_idx) || (sel_out && !aligned16(sel_out)) || !aligned4(kl))
+    return MSA_ERR_MISALIGNED;
+  size_t need = 0;
+  if ((st = msa_workspace_size(s, MSA_OP_FORWARD_ALIGNMENT, &need)) != MSA_OK) return st;
+  if (!ws) return MSA_ERR_NULL_PTR;
+  if (ws_bytes < need) return MSA_ERR_WORKSPACE_TOO_SMALL;
+  if (!aligned16(ws)) return MSA_ERR_MISALIGNED;
+  if (!device_ctx()) return MSA_ERR_CUDA;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  char* w = static_cast<char*>(ws);
+  float* pooled = reinterpret_cast<float*>(w);
+  int32_t* sel = sel_out ? sel_out : reinterpret_cast<int32_t*>(w + pooled_bytes(*s));
+  void* rest = w + pooled_bytes(*s) + sel_bytes(*s);
+  cudaError_t e = launch_index_scores(*s, q_idx, k_idx, pooled, false, cs);
+  if (e == cudaSuccess) e = launch_block_topk(*s, pooled, sel, cs);
+  if (e == cudaSuccess) e = launch_sparse_prefill(*s, q, k, v, sel, o, lse, rest, cs, pooled, kl);
   return from_cuda(e);
 }
 

@@ -53,7 +53,8 @@ cudaError_t launch_block_topk(const msa_shape& s, const float* pooled, int32_t* 
 size_t prefill_workspace_bytes(const msa_shape& s);
 cudaError_t launch_sparse_prefill(const msa_shape& s, const uint16_t* q, const uint16_t* k,
                                   const uint16_t* v, const int32_t* sel, uint16_t* o,
-                                  float* lse, void* ws, cudaStream_t st);
+                                  float* lse, void* ws, cudaStream_t st,
+                                  const float* pooled = nullptr, float* kl = nullptr);
 size_t decode_workspace_bytes(const msa_shape& s, bool dense);
 cudaError_t launch_decode(const msa_shape& s, const uint16_t* q, const uint16_t* k,
                           const uint16_t* v, const int32_t* sel, uint16_t* o, float* lse,

@@ -775,14 +775,24 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 // m_s and sum l_s = sum_j 2^(x_j - m_s) (x in log2 units).  With M = max_s m_s
 // and w_s = 2^(m_s - M) l_s:  o = sum_s w_s O_s / sum_s w_s.  The partial of
 // (group g, slot s) sits at entry inv[t, g, s] of the column-sorted list.
-template <int D>
+//
+// KL (index-alignment diagnostic, MiniMax Sparse Attention pages, "KL Loss
+// Alignment"): w_s / sum_s w_s is the attention mass head h puts on selected
+// block s, so the same (m, l) pairs also give, per group g,
+//   P_main(s)  = mean over the group's heads of w_s / sum w
+//   P_index(s) = softmax over the selected slots of pooled[t, g, sel[s]]
+//   kl[t, g]   = sum_s P_main(s) (log P_main(s) - log P_index(s)).
+template <int D, bool KL>
 __global__ void __launch_bounds__(256) combine_kernel(const int32_t* __restrict__ sel,
                                                       const PrefillWs w, uint16_t* __restrict__ o,
                                                       float* __restrict__ lse, int H, int G,
-                                                      int r, int k) {
+                                                      int r, int k,
+                                                      const float* __restrict__ pooled,
+                                                      float* __restrict__ kl, int nb) {
   constexpr int CH = D / 8;                  // 16-byte chunks per head row
   extern __shared__ float2 sm_ml[];          // [k][H] (m, l), m = -inf for unused slots
-  uint32_t* sm_pos = reinterpret_cast<uint32_t*>(sm_ml + k * H);   // [G][k] entry of each slot
+  float2* sm_hd = sm_ml + k * H;             // [H] (M, 1 / den), KL only
+  uint32_t* sm_pos = reinterpret_cast<uint32_t*>(sm_hd + (KL ? H : 0));   // [G][k] entries
   const long long bt = blockIdx.x;           // b*T + t
   const float2* ml_all = reinterpret_cast<const float2*>(w.part_ml);
   const int32_t* srow = sel + bt * G * k;
@@ -797,6 +807,46 @@ __global__ void __launch_bounds__(256) combine_kernel(const int32_t* __restrict_
                                   : make_float2(-INFINITY, 0.f);
   }
   __syncthreads();
+  if constexpr (KL) {
+    for (int h = threadIdx.x; h < H; h += blockDim.x) {
+      float M = -INFINITY, den = 0.f;
+      for (int s = 0; s < k; ++s) M = fmaxf(M, sm_ml[s * H + h].x);
+      for (int s = 0; s < k; ++s) {
+        const float2 ml = sm_ml[s * H + h];
+        if (ml.x != -INFINITY) den += exp2f(ml.x - M) * ml.y;
+      }
+      sm_hd[h] = make_float2(M, 1.f / den);
+    }
+    __syncthreads();
+    const int lane = threadIdx.x & 31;
+    for (int g = threadIdx.x >> 5; g < G; g += blockDim.x >> 5) {
+      const float* prow = pooled + (bt * G + g) * nb;
+      float zmax = -INFINITY;
+      for (int s = lane; s < k; s += 32)
+        if (srow[g * k + s] >= 0) zmax = fmaxf(zmax, prow[srow[g * k + s]]);
+      for (int off = 16; off; off >>= 1) zmax = fmaxf(zmax, __shfl_xor_sync(~0u, zmax, off));
+      float zsum = 0.f;
+      for (int s = lane; s < k; s += 32)
+        if (srow[g * k + s] >= 0) zsum += expf(prow[srow[g * k + s]] - zmax);
+      for (int off = 16; off; off >>= 1) zsum += __shfl_xor_sync(~0u, zsum, off);
+      const float log_z = logf(zsum);        // log P_index(s) = z_s - zmax - log_z
+      float acc = 0.f;
+      for (int s = lane; s < k; s += 32) {
+        if (srow[g * k + s] < 0) continue;
+        float pm = 0.f;
+        for (int hh = 0; hh < r; ++hh) {
+          const int h = g * r + hh;
+          const float2 ml = sm_ml[s * H + h];
+          const float2 hd = sm_hd[h];
+          if (ml.x != -INFINITY) pm += exp2f(ml.x - hd.x) * ml.y * hd.y;
+        }
+        pm /= static_cast<float>(r);
+        if (pm > 0.f) acc += pm * (logf(pm) - (prow[srow[g * k + s]] - zmax - log_z));
+      }
+      for (int off = 16; off; off >>= 1) acc += __shfl_xor_sync(~0u, acc, off);
+      if (lane == 0) kl[bt * G + g] = acc;
+    }
+  }
   for (int item = threadIdx.x; item < H * CH; item += blockDim.x) {
     const int h = item / CH, c = item % CH;
     const int g = h / r, hh = h - g * r;
@@ -888,7 +938,8 @@ size_t prefill_workspace_bytes(const msa_shape& s) { return carve_bytes(s); }
 
 cudaError_t launch_sparse_prefill(const msa_shape& s, const uint16_t* q, const uint16_t* k,
                                   const uint16_t* v, const int32_t* sel, uint16_t* o,
-                                  float* lse, void* ws, cudaStream_t st) {
+                                  float* lse, void* ws, cudaStream_t st, const float* pooled,
+                                  float* kl) {
   const DevCtx* ctx = device_ctx();
   if (!ctx) return cudaErrorInitializationError;
   PrefillWs w = carve(s, ws);
@@ -941,15 +992,24 @@ cudaError_t launch_sparse_prefill(const msa_shape& s, const uint16_t* q, const u
                         : launch_attn<64>(s, q, k, v, p, ctx, st);
   if (e != cudaSuccess) return e;
   const unsigned ntok = static_cast<unsigned>(static_cast<long long>(s.batch) * s.seq_q);
-  const size_t csmem = sizeof(float2) * s.topk * s.n_q_heads + 4u * s.n_kv_heads * s.topk;
+  const bool with_kl = kl != nullptr;
+  const size_t csmem = sizeof(float2) * s.topk * s.n_q_heads +
+                       (with_kl ? sizeof(float2) * s.n_q_heads : 0) + 4u * s.n_kv_heads * s.topk;
   {
-    ProfScope ps_("combine", st);
-    if (s.head_dim == 128)
-      combine_kernel<128><<<ntok, 256, csmem, st>>>(sel, w, o, lse, s.n_q_heads, s.n_kv_heads, r,
-                                                    s.topk);
+    ProfScope ps_(with_kl ? "combine_kl" : "combine", st);
+    const int H = s.n_q_heads, G = s.n_kv_heads, kk = s.topk;
+    if (s.head_dim == 128 && with_kl)
+      combine_kernel<128, true><<<ntok, 256, csmem, st>>>(sel, w, o, lse, H, G, r, kk, pooled, kl,
+                                                          nb);
+    else if (s.head_dim == 128)
+      combine_kernel<128, false><<<ntok, 256, csmem, st>>>(sel, w, o, lse, H, G, r, kk, nullptr,
+                                                           nullptr, nb);
+    else if (with_kl)
+      combine_kernel<64, true><<<ntok, 256, csmem, st>>>(sel, w, o, lse, H, G, r, kk, pooled, kl,
+                                                         nb);
     else
-      combine_kernel<64><<<ntok, 256, csmem, st>>>(sel, w, o, lse, s.n_q_heads, s.n_kv_heads, r,
-                                                   s.topk);
+      combine_kernel<64, false><<<ntok, 256, csmem, st>>>(sel, w, o, lse, H, G, r, kk, nullptr,
+                                                          nullptr, nb);
   }
   return cudaGetLastError();
 }

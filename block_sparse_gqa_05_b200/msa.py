@@ -19,7 +19,7 @@ LIB_PATH = os.path.join(_PKG, "libmsa.so")
 HEADER_PATH = os.path.join(os.path.dirname(_PKG), "include", "msa.h")
 
 OP_INDEX_SCORES, OP_BLOCK_TOPK, OP_SPARSE_PREFILL, OP_SPARSE_DECODE, OP_FORWARD, \
-    OP_DENSE_PREFILL, OP_DENSE_DECODE = range(7)
+    OP_DENSE_PREFILL, OP_DENSE_DECODE, OP_FORWARD_ALIGNMENT = range(8)
 
 STATUS = {0: "MSA_OK", 1: "MSA_ERR_INVALID_SHAPE", 2: "MSA_ERR_NULL_PTR", 3: "MSA_ERR_MISALIGNED",
           4: "MSA_ERR_WORKSPACE_TOO_SMALL", 5: "MSA_ERR_UNSUPPORTED", 6: "MSA_ERR_CUDA",
@@ -62,6 +62,8 @@ _SIGS = {
                                       ctypes.c_int),
     "msa_forward": ([ctypes.POINTER(Shape), _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
                      ctypes.c_size_t, _vp], ctypes.c_int),
+    "msa_forward_alignment": ([ctypes.POINTER(Shape), _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
+                               _vp, _vp, ctypes.c_size_t, _vp], ctypes.c_int),
     "msa_forward_decode_ragged": ([ctypes.POINTER(Shape), _vp, _vp, _vp, _vp, _vp, _vp, _vp,
                                    _vp, _vp, _vp, ctypes.c_size_t, _vp], ctypes.c_int),
     "msa_dense_attn_prefill": ([ctypes.POINTER(Shape), _vp, _vp, _vp, _vp, _vp, _vp,
@@ -202,6 +204,26 @@ def forward(shape: Shape, q, k, v, q_idx, k_idx, o=None, lse=None, sel=None, ws=
                              _ptr(k_idx), _ptr(o), _ptr(lse), _ptr(sel), _ptr(ws), ws.numel(),
                              _stream(stream)), "msa_forward")
     return o, lse, sel
+
+
+def forward_alignment(shape: Shape, q, k, v, q_idx, k_idx, o=None, lse=None, sel=None,
+                      kl=None, ws=None, want_lse=True, want_sel=True, stream=None):
+    """msa_forward_alignment: the whole layer plus kl [B, T, G] float32, the
+    divergence of the index branch's block distribution from the main
+    branch's (forward only).  Returns (o, lse, sel, kl)."""
+    o, lse = _attn_out(shape, q, o, lse, want_lse)
+    if sel is None and want_sel:
+        sel = torch.empty((shape.batch, shape.seq_q, shape.n_kv_heads, shape.topk),
+                          dtype=torch.int32, device=q.device)
+    if kl is None:
+        kl = torch.empty((shape.batch, shape.seq_q, shape.n_kv_heads), dtype=torch.float32,
+                         device=q.device)
+    ws = alloc_workspace(shape, OP_FORWARD_ALIGNMENT, q.device) if ws is None else ws
+    _check(lib().msa_forward_alignment(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v),
+                                       _ptr(q_idx), _ptr(k_idx), _ptr(o), _ptr(lse), _ptr(sel),
+                                       _ptr(kl), _ptr(ws), ws.numel(), _stream(stream)),
+           "msa_forward_alignment")
+    return o, lse, sel, kl
 
 
 def forward_decode_ragged(shape: Shape, q, k, v, q_idx, k_idx, seq_lens, o=None, lse=None,

@@ -5,6 +5,8 @@
  * real K/V of the selected blocks, shared by every query head of a group).
  *
  * Sources of the definitions (web pages on the method):
+ *   [P1] Notion note "Minimax sparse Attention" (GQA definition; the index
+ *        branch is aligned to the main branch with a KL loss).
  *   [P2] hamidun.com, "MiniMax lança MSA: atenção esparsa acelera em 28 vezes…",
  *        section "Como o MSA funciona" (index branch picks top-k KV blocks per
  *        query and per GQA group; main branch runs exact attention on them).
@@ -90,7 +92,8 @@ typedef enum msa_op {
   MSA_OP_SPARSE_DECODE = 3,
   MSA_OP_FORWARD = 4,
   MSA_OP_DENSE_PREFILL = 5,
-  MSA_OP_DENSE_DECODE = 6
+  MSA_OP_DENSE_DECODE = 6,
+  MSA_OP_FORWARD_ALIGNMENT = 7
 } msa_op;
 
 /* Human-readable name of a status code (static string, never NULL). */
@@ -152,6 +155,28 @@ msa_status msa_forward(const msa_shape* shape, const uint16_t* q, const uint16_t
                        const uint16_t* v, const uint16_t* q_idx, const uint16_t* k_idx,
                        uint16_t* o, float* lse, int32_t* sel_out, void* ws,
                        size_t ws_bytes, void* stream);
+
+/* Whole layer plus the index-alignment divergence, forward only ([P1] bullet
+ * "KL Loss Alignment": the index branch is trained towards the main branch's
+ * attention distribution; the pages give no formula, so this call computes
+ * the plainest reading of it as a diagnostic and trains nothing):
+ *   P_main[b,t,g](j)  = attention mass the heads of group g put on selected
+ *                       block j (sum of softmax weights over its keys),
+ *                       averaged over the group's r heads;
+ *   P_index[b,t,g](j) = softmax over the selected blocks j of pooled[b,t,g,j]
+ *                       (raw scores, no temperature);
+ *   kl[b,t,g]         = sum_j P_main(j) (ln P_main(j) - ln P_index(j)),
+ *                       terms with P_main(j) == 0 count 0.
+ * kl: device float32 [B, T, G], 4-byte aligned, required.  o, lse and
+ * sel_out are as in msa_forward.  Every shape (T == 1 included) runs the
+ * prefill path (KV-outer attention, then a combine that also reduces the
+ * per-block masses into kl); ws >= msa_workspace_size(
+ * MSA_OP_FORWARD_ALIGNMENT). */
+msa_status msa_forward_alignment(const msa_shape* shape, const uint16_t* q,
+                                 const uint16_t* k, const uint16_t* v,
+                                 const uint16_t* q_idx, const uint16_t* k_idx,
+                                 uint16_t* o, float* lse, int32_t* sel_out, float* kl,
+                                 void* ws, size_t ws_bytes, void* stream);
 
 /* Whole layer for one decode step over caches of different lengths (the
  * pages' decode step, batched for serving; no other counterpart on them):

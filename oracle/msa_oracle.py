@@ -15,8 +15,8 @@ Attention (MSA) : attention block-sparse à deux branches…"):
    heads, token score = raw dot product q_idx . k_idx over causal keys, then a
    max over each B-token block.  Blocks with no causal key are -inf.
 2. ``select_blocks`` / ``block_topk`` -- per query and per group, keep the top
-   scoring blocks (P3 第一步 "TopK"; P4 "pro GQA-Gruppe unabhängig ein
-   Top-k-Subset"), with the local block always included (P5, paragraph on the
+   scoring blocks (P3 第一步 "TopK"; P4, passage on one independent top-k
+   subset per GQA group), with the local block always included (P5, paragraph on the
    local block) in a budget of k blocks of B tokens (P5: 16 x 128 = 2048).
 3. ``sparse_attention`` -- main branch (P3, section 第二步 "sparse branch"; P2
    "Como o MSA funciona"): exact softmax attention of every query head over

@@ -13,6 +13,13 @@ MEAN_ABS = 1e-3
 # row normaliser l, so |d lse| = |d l| / l <= 2^-9 from that rounding alone,
 # plus fp32 accumulation; 4e-3 leaves a 2x margin.
 LSE_ABS = 4e-3
+# Index-alignment KL.  P_main(j) is built from the same l sums, so each block
+# mass has relative error eps <= 2 * 2^-9 (numerator and normaliser).  With
+# sum_j dP_main(j) = 0, dKL = sum_j dP_main(j) ln(P_main(j) / P_index(j)), and
+# sum_j P_main |ln(P_main / P_index)| <= KL + 2 (the terms with P_main < P_index
+# add at most sum P_index <= 1 in absolute value), so |dKL| <= eps (KL + 2);
+# the tolerance doubles eps.
+KL_REL = 8e-3
 
 
 def spec(batch, seq_q, seq_kv, q_offset, H, G, d, di, topk, seed=7, planted=0):

@@ -53,6 +53,13 @@ def test_workspace_sizes_and_validation():
     assert st == 0 and n >= 3 * 8 * 4 * 64 * 4
     st, nd = ws(dec, M.OP_DENSE_DECODE)
     assert st == 0 and nd > 0
+    # the alignment forward runs the prefill path for every T, decode shapes too
+    st, al = ws(tiny(), M.OP_FORWARD_ALIGNMENT)
+    assert st == 0 and al == fwd
+    st, ald = ws(dec, M.OP_FORWARD_ALIGNMENT)
+    st2, fd = ws(dec, M.OP_FORWARD)
+    st3, pd = ws(dec, M.OP_SPARSE_PREFILL)
+    assert st == st2 == st3 == 0 and ald >= pd and ald != fd
     # decode needs T == 1 and q_offset == N - 1
     assert ws(tiny(batch=3, seq_q=1, seq_kv=5000, q_offset=10), M.OP_SPARSE_DECODE)[0] == 1
     assert ws(tiny(), M.OP_SPARSE_DECODE)[0] == 1
@@ -80,6 +87,13 @@ def test_pointer_checks_precede_device_use(L):
     bad = tiny(block=256)
     assert L.msa_forward(ctypes.byref(bad), ok, ok, ok, ok, ok, ok, None, None, ok, 1 << 40,
                          None) == 5
+    # kl is required, 4-byte aligned, checked before the workspace
+    assert L.msa_forward_alignment(ctypes.byref(s), ok, ok, ok, ok, ok, ok, None, None, None,
+                                   ok, 1 << 40, None) == 2
+    assert L.msa_forward_alignment(ctypes.byref(s), ok, ok, ok, ok, ok, ok, None, None,
+                                   ctypes.c_void_p((1 << 20) + 2), ok, 1 << 40, None) == 3
+    assert L.msa_forward_alignment(ctypes.byref(s), ok, ok, ok, ok, ok, ok, None, None, ok,
+                                   ok, 16, None) == 4
     dec = tiny(seq_q=1, seq_kv=4096, q_offset=4095)
     assert L.msa_sparse_attn_decode(ctypes.byref(dec), ok, ok, ok, ok, ok, None, ok, 8, None) == 4
     assert L.msa_dense_attn_decode(ctypes.byref(s), ok, ok, ok, ok, None, ok, 1 << 30, None) == 1

@@ -13,7 +13,8 @@ import block_sparse_gqa_05_b200 as M
 import oracle as O
 import synth
 from tests.gpu_helpers import (spec, inputs_cpu, positions, oracle_pooled, oracle_sel,
-                               check_pooled, check_attn, oracle_attention, cuda, LSE_ABS)
+                               check_pooled, check_attn, oracle_attention, cuda, LSE_ABS,
+                               KL_REL)
 
 pytestmark = pytest.mark.gpu
 
@@ -239,6 +240,40 @@ def test_forward_decode():
         assert np.array_equal(sel[b].cpu().numpy(), sref)
         O_ref, _ = oracle_attention(sp, inp, sref, b)
         check_attn(o[b], O_ref, f"forward decode b={b}")
+
+
+@pytest.mark.parametrize("sp", [
+    RAGGED,                                                          # r = 4, d = 64, k = 5
+    spec(1, 640, 9000, 8000, 8, 8, 128, 64, 16, seed=62),            # r = 1
+    spec(1, 400, 3000, 2600, 16, 2, 128, 64, 16, seed=63, planted=2),  # r = 8, d = 128
+    spec(2, 1, 3000, 2999, 16, 2, 128, 64, 4, seed=64),              # T = 1 on the prefill path
+    spec(1, 200, 1000, 800, 8, 2, 64, 32, 1, seed=65),               # k = 1: KL = 0
+])
+def test_forward_alignment_kl(sp):
+    """kl against the oracle's alignment KL on the oracle's pooled scores and
+    selection; o and sel as msa_forward returns them."""
+    inp = inputs_cpu(sp)
+    sh = M.Shape.of(sp)
+    o, lse, sel, kl = M.forward_alignment(sh, cuda(inp.q), cuda(inp.k), cuda(inp.v),
+                                          cuda(inp.q_idx), cuda(inp.k_idx))
+    torch.cuda.synchronize()
+    assert M.device_status() == 0
+    for b in range(sp.batch):
+        pooled = oracle_pooled(sp, inp, b)
+        sref = oracle_sel(sp, pooled)
+        assert np.array_equal(sel[b].cpu().numpy(), sref)
+        O_ref, _ = oracle_attention(sp, inp, sref, b)
+        check_attn(o[b], O_ref, f"alignment forward b={b}")
+        kl_ref = O.index_alignment_kl(inp.q[b], inp.k[b], inp.v[b], sref, pooled, positions(sp),
+                                      sp.block)
+        got = kl[b].double().cpu().numpy()
+        assert np.all(np.isfinite(got))
+        err = np.abs(got - kl_ref)
+        bad = np.argwhere(err > KL_REL * (kl_ref + 2.0))
+        assert bad.size == 0, f"b={b}: {len(bad)} kl mismatches, first {bad[:3].tolist()}: " \
+            f"gpu {got[tuple(bad[0])]} ref {kl_ref[tuple(bad[0])]}"
+        if sp.topk == 1:
+            assert np.all(kl_ref == 0.0)
 
 
 def test_device_status_clean():
