@@ -782,8 +782,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 //   P_main(s)  = mean over the group's heads of w_s / sum w
 //   P_index(s) = softmax over the selected slots of pooled[t, g, sel[s]]
 //   kl[t, g]   = sum_s P_main(s) (log P_main(s) - log P_index(s)).
+// Six CTAs per SM (<= 40 registers): the kernel waits on scattered partial
+// reads, and the KL variant at its natural 46 registers fits only five, which
+// cost it a fifth of its speed.
 template <int D, bool KL>
-__global__ void __launch_bounds__(256) combine_kernel(const int32_t* __restrict__ sel,
+__global__ void __launch_bounds__(256, 8) combine_kernel(const int32_t* __restrict__ sel,
                                                       const PrefillWs w, uint16_t* __restrict__ o,
                                                       float* __restrict__ lse, int H, int G,
                                                       int r, int k,
@@ -791,14 +794,18 @@ __global__ void __launch_bounds__(256) combine_kernel(const int32_t* __restrict_
                                                       float* __restrict__ kl, int nb) {
   constexpr int CH = D / 8;                  // 16-byte chunks per head row
   extern __shared__ float2 sm_ml[];          // [k][H] (m, l), m = -inf for unused slots
-  float2* sm_hd = sm_ml + k * H;             // [H] (M, 1 / den), KL only
-  uint32_t* sm_pos = reinterpret_cast<uint32_t*>(sm_hd + (KL ? H : 0));   // [G][k] entries
+  float2* sm_hd = sm_ml + k * H;             // KL only: [H] (M, 1 / den)
+  float* sm_z = reinterpret_cast<float*>(sm_hd + (KL ? H : 0));   // KL only: [G][k] pooled
+  uint32_t* sm_pos = reinterpret_cast<uint32_t*>(sm_z + (KL ? G * k : 0));   // [G][k] entries
   const long long bt = blockIdx.x;           // b*T + t
   const float2* ml_all = reinterpret_cast<const float2*>(w.part_ml);
   const int32_t* srow = sel + bt * G * k;
   const uint32_t* irow = w.inv + bt * G * k;
-  for (int x = threadIdx.x; x < G * k; x += blockDim.x)
-    sm_pos[x] = srow[x] >= 0 ? irow[x] : 0xFFFFFFFFu;
+  for (int x = threadIdx.x; x < G * k; x += blockDim.x) {
+    const int j = srow[x];
+    sm_pos[x] = j >= 0 ? irow[x] : 0xFFFFFFFFu;
+    if constexpr (KL) sm_z[x] = j >= 0 ? pooled[(bt * G + x / k) * nb + j] : -INFINITY;
+  }
   __syncthreads();
   for (int x = threadIdx.x; x < k * H; x += blockDim.x) {
     const int s = x / H, h = x % H, g = h / r;
@@ -807,46 +814,6 @@ __global__ void __launch_bounds__(256) combine_kernel(const int32_t* __restrict_
                                   : make_float2(-INFINITY, 0.f);
   }
   __syncthreads();
-  if constexpr (KL) {
-    for (int h = threadIdx.x; h < H; h += blockDim.x) {
-      float M = -INFINITY, den = 0.f;
-      for (int s = 0; s < k; ++s) M = fmaxf(M, sm_ml[s * H + h].x);
-      for (int s = 0; s < k; ++s) {
-        const float2 ml = sm_ml[s * H + h];
-        if (ml.x != -INFINITY) den += exp2f(ml.x - M) * ml.y;
-      }
-      sm_hd[h] = make_float2(M, 1.f / den);
-    }
-    __syncthreads();
-    const int lane = threadIdx.x & 31;
-    for (int g = threadIdx.x >> 5; g < G; g += blockDim.x >> 5) {
-      const float* prow = pooled + (bt * G + g) * nb;
-      float zmax = -INFINITY;
-      for (int s = lane; s < k; s += 32)
-        if (srow[g * k + s] >= 0) zmax = fmaxf(zmax, prow[srow[g * k + s]]);
-      for (int off = 16; off; off >>= 1) zmax = fmaxf(zmax, __shfl_xor_sync(~0u, zmax, off));
-      float zsum = 0.f;
-      for (int s = lane; s < k; s += 32)
-        if (srow[g * k + s] >= 0) zsum += expf(prow[srow[g * k + s]] - zmax);
-      for (int off = 16; off; off >>= 1) zsum += __shfl_xor_sync(~0u, zsum, off);
-      const float log_z = logf(zsum);        // log P_index(s) = z_s - zmax - log_z
-      float acc = 0.f;
-      for (int s = lane; s < k; s += 32) {
-        if (srow[g * k + s] < 0) continue;
-        float pm = 0.f;
-        for (int hh = 0; hh < r; ++hh) {
-          const int h = g * r + hh;
-          const float2 ml = sm_ml[s * H + h];
-          const float2 hd = sm_hd[h];
-          if (ml.x != -INFINITY) pm += exp2f(ml.x - hd.x) * ml.y * hd.y;
-        }
-        pm /= static_cast<float>(r);
-        if (pm > 0.f) acc += pm * (logf(pm) - (prow[srow[g * k + s]] - zmax - log_z));
-      }
-      for (int off = 16; off; off >>= 1) acc += __shfl_xor_sync(~0u, acc, off);
-      if (lane == 0) kl[bt * G + g] = acc;
-    }
-  }
   for (int item = threadIdx.x; item < H * CH; item += blockDim.x) {
     const int h = item / CH, c = item % CH;
     const int g = h / r, hh = h - g * r;
@@ -881,6 +848,39 @@ __global__ void __launch_bounds__(256) combine_kernel(const int32_t* __restrict_
     }
     *(reinterpret_cast<uint4*>(o + (bt * H + h) * D) + c) = make_uint4(out[0], out[1], out[2], out[3]);
     if (lse && c == 0) lse[bt * H + h] = (M + log2f(den)) / kLog2e;
+    if constexpr (KL) {
+      if (c == 0) sm_hd[h] = make_float2(M, inv);
+    }
+  }
+  if constexpr (KL) {
+    __syncthreads();
+    const int lane = threadIdx.x & 31;
+    for (int g = threadIdx.x >> 5; g < G; g += blockDim.x >> 5) {
+      const float* zg = sm_z + g * k;
+      float zmax = -INFINITY;
+      for (int s = lane; s < k; s += 32) zmax = fmaxf(zmax, zg[s]);
+      for (int off = 16; off; off >>= 1) zmax = fmaxf(zmax, __shfl_xor_sync(~0u, zmax, off));
+      float zsum = 0.f;
+      for (int s = lane; s < k; s += 32)
+        if (zg[s] != -INFINITY) zsum += expf(zg[s] - zmax);
+      for (int off = 16; off; off >>= 1) zsum += __shfl_xor_sync(~0u, zsum, off);
+      const float log_z = logf(zsum);        // ln P_index(s) = z_s - zmax - log_z
+      float acc = 0.f;
+      for (int s = lane; s < k; s += 32) {
+        if (zg[s] == -INFINITY) continue;
+        float pm = 0.f;
+        for (int hh = 0; hh < r; ++hh) {
+          const int h = g * r + hh;
+          const float2 ml = sm_ml[s * H + h];
+          const float2 hd = sm_hd[h];
+          if (ml.x != -INFINITY) pm += exp2f(ml.x - hd.x) * ml.y * hd.y;
+        }
+        pm /= static_cast<float>(r);
+        if (pm > 0.f) acc += pm * (logf(pm) - (zg[s] - zmax - log_z));
+      }
+      for (int off = 16; off; off >>= 1) acc += __shfl_xor_sync(~0u, acc, off);
+      if (lane == 0) kl[bt * G + g] = acc;
+    }
   }
 }
 
@@ -994,7 +994,8 @@ cudaError_t launch_sparse_prefill(const msa_shape& s, const uint16_t* q, const u
   const unsigned ntok = static_cast<unsigned>(static_cast<long long>(s.batch) * s.seq_q);
   const bool with_kl = kl != nullptr;
   const size_t csmem = sizeof(float2) * s.topk * s.n_q_heads +
-                       (with_kl ? sizeof(float2) * s.n_q_heads : 0) + 4u * s.n_kv_heads * s.topk;
+                       (with_kl ? sizeof(float2) * s.n_q_heads + 4u * s.n_kv_heads * s.topk : 0) +
+                       4u * s.n_kv_heads * s.topk;
   {
     ProfScope ps_(with_kl ? "combine_kl" : "combine", st);
     const int H = s.n_q_heads, G = s.n_kv_heads, kk = s.topk;

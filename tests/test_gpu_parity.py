@@ -272,8 +272,8 @@ def test_forward_alignment_kl(sp):
         bad = np.argwhere(err > KL_REL * (kl_ref + 2.0))
         assert bad.size == 0, f"b={b}: {len(bad)} kl mismatches, first {bad[:3].tolist()}: " \
             f"gpu {got[tuple(bad[0])]} ref {kl_ref[tuple(bad[0])]}"
-        if sp.topk == 1:
-            assert np.all(kl_ref == 0.0)
+        if sp.topk == 1:                     # one block: both distributions are (1)
+            assert np.abs(kl_ref).max() <= 1e-12 and np.abs(got).max() <= 1e-5
 
 
 def test_device_status_clean():

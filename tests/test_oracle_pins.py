@@ -272,7 +272,7 @@ def test_alignment_single_block_is_zero():
     sel = np.array([[[3], [3]]], dtype=np.int32)
     pooled = rng.standard_normal((1, 2, 5))
     kl = O.index_alignment_kl(q, k, v, sel, pooled, np.array([29]), 8)
-    assert np.all(kl == 0.0)
+    assert np.abs(kl).max() <= 1e-12          # the head weights sum to 1 up to rounding
 
 
 def test_alignment_uniform_keys_closed_form():
