@@ -2,19 +2,24 @@
 """Throughput of the MSA hot path on B200 (one JSON line on rank 0).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl msa|reference]
-                    [--workload prefill_128k] [--skip-long] [--skip-cpu]
+                    [--workload prefill_128k] [--shard sequence|group]
+                    [--skip-long] [--skip-cpu]
 
 Headline step: one MSA forward (index scores -> block top-k -> KV-outer sparse
 attention) over one 131072-token sequence per GPU, inputs resident in HBM.
 In the same run, and reported in their own objects: batched decode (32
 sequences x 128K cache), and the 1M-token context (last 8192-query prefill
-chunk, batch-4 decode) beside the in-repo dense causal GQA kernels.  Every
-GPU runs an independent sequence (weak scaling, no collective on the data
-path); the time is the max over ranks.
+chunk, batch-4 decode) beside the in-repo dense causal GQA kernels.  By
+default every GPU runs an independent sequence (weak scaling, no collective on
+the data path); with --shard group the GPUs split the KV groups of the one
+headline sequence instead (strong scaling: each owns G/N groups' K/V, query
+heads and index queries plus a replica of the index keys; no exchange inside
+the layer).  The time is the max over ranks.
 """
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import hashlib
 import json
 import math
@@ -23,6 +28,7 @@ import statistics
 import subprocess
 import sys
 import time
+import types
 
 import numpy as np
 import torch
@@ -156,6 +162,18 @@ def rank_workload(name, rank):
     return synth.workload(name, seed=sp.seed + 1000 * rank)
 
 
+def group_shard_inputs(sp, rank, world, device):
+    """This rank's group shard of workload ``sp`` (the same sequence on every
+    rank): (GroupShard, (q, k, v, q_idx, k_idx)), contiguous, on ``device``."""
+    from block_sparse_gqa_05_b200 import shard as S
+    from block_sparse_gqa_05_b200.msa import Shape
+    gs = S.group_shard(Shape.of(sp), rank, world)
+    full = synth.make_inputs(sp, device)
+    parts = S.shard_inputs(gs, full.q, full.k, full.v, full.q_idx, full.k_idx)
+    del full
+    return gs, parts
+
+
 def barrier(pg):
     if pg is not None:
         pg.barrier()
@@ -211,8 +229,20 @@ def run_msa(args, world, rank, pg):
     peaks, peak_src = load_peaks()
     stream = torch.cuda.current_stream()
     out = {}
-    sp = rank_workload(args.workload, rank)
-    inp = synth.make_inputs(sp, "cuda")
+    if args.shard == "group":
+        # one sequence, G/world groups per rank: every rank's step covers all
+        # of the sequence's tokens for its share of the heads
+        sp_full = synth.workload(args.workload)
+        gs, parts = group_shard_inputs(sp_full, rank, world, "cuda")
+        inp = types.SimpleNamespace(**dict(zip(("q", "k", "v", "q_idx", "k_idx"), parts)))
+        sp = dataclasses.replace(sp_full, n_q_heads=gs.shape.n_q_heads,
+                                 n_kv_heads=gs.shape.n_kv_heads)
+        token_ranks = 1
+        torch.cuda.empty_cache()
+    else:
+        sp = rank_workload(args.workload, rank)
+        inp = synth.make_inputs(sp, "cuda")
+        token_ranks = world
     sh = M.Shape.of(sp)
     ws = M.alloc_workspace(sh, M.OP_FORWARD)
     o = torch.empty_like(inp.q)
@@ -239,7 +269,7 @@ def run_msa(args, world, rank, pg):
     kernels = {k: v[0] / v[1] for k, v in prof.items()}   # ms per launch
     launches_per_step = sum(v[1] for v in prof.values()) / nsteps
     tokens = sp.batch * sp.seq_q
-    out["value"] = tokens * world / (ms / 1e3)
+    out["value"] = tokens * token_ranks / (ms / 1e3)
     out["ms_per_step"] = ms
     out["gpu_launches"] = int(round(launches_per_step * args.steps))
     out["kernels_ms_per_launch"] = {k: round(v, 4) for k, v in kernels.items()}
@@ -283,7 +313,7 @@ def run_msa(args, world, rank, pg):
         def dstep():
             M.dense_attn_prefill(sh, inp.q, inp.k, inp.v, o=o, lse=None, want_lse=False)
         dms = timed_loop(dstep, 2, 1, pg, stream)
-        out["dense_gqa_prefill"] = {"ms_per_step": dms, "value": tokens * world / (dms / 1e3),
+        out["dense_gqa_prefill"] = {"ms_per_step": dms, "value": tokens * token_ranks / (dms / 1e3),
                                     "speedup_msa_vs_dense": round(dms / ms, 2)}
 
     # ---- end to end through the public API with host buffers.  Each step
@@ -343,7 +373,7 @@ def run_msa(args, world, rank, pg):
         torch.cuda.synchronize()
         ems = max_over_ranks(t0.elapsed_time(t1), pg) / e2e_n
         barrier(pg)
-        out["e2e"] = {"value": tokens * world / (ems / 1e3), "unit": "tokens/s",
+        out["e2e"] = {"value": tokens * token_ranks / (ems / 1e3), "unit": "tokens/s",
                       "ms_per_step": ems, "pipelined": "upload / compute / download streams, 2 buffer sets",
                       "h2d_bytes_per_step": int(sum(t.numel() * t.element_size() for t in host.values())),
                       "d2h_bytes_per_step": int(o_host[0].numel() * o_host[0].element_size())}
@@ -602,6 +632,9 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="msa", choices=["msa", "reference"])
     ap.add_argument("--workload", default="prefill_128k")
+    ap.add_argument("--shard", default="sequence", choices=["sequence", "group"],
+                    help="sequence: one independent sequence per GPU (weak scaling); "
+                         "group: the GPUs split the KV groups of one sequence (strong)")
     ap.add_argument("--decode-workload", default="decode_128k_b32")
     ap.add_argument("--skip-long", action="store_true")
     ap.add_argument("--skip-decode", action="store_true")
@@ -623,15 +656,24 @@ def main():
         return
     world, rank, local, pg = dist_setup(args)
     res, sp = run_msa(args, world, rank, pg)
+    grouped = args.shard == "group"
+    if grouped:
+        sp = synth.workload(args.workload)
+        parallelism = (f"group-sharded over {world} GPU(s): {sp.n_kv_heads // world} KV groups "
+                       f"each, index keys replicated; decode and 1M sections: independent "
+                       f"sequences per GPU")
+    else:
+        parallelism = f"dp{world} (independent sequences)"
     if rank == 0:
         line = {"metric": METRIC, "value": res["value"], "unit": "tokens/s", "n_gpus": world,
                 "steps": args.steps, "warmup": args.warmup, "ms_per_step": res["ms_per_step"],
-                "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
-                "data": "synthetic",
+                "higher_is_better": True, "scaling": "strong" if grouped else "weak",
+                "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
                 "config": {"workload": args.workload, "seq_len": sp.seq_kv,
-                           "global_batch": sp.batch * world, "heads": f"{sp.n_q_heads}q/{sp.n_kv_heads}kv",
+                           "global_batch": sp.batch * (1 if grouped else world),
+                           "heads": f"{sp.n_q_heads}q/{sp.n_kv_heads}kv",
                            "head_dim": sp.head_dim, "index_dim": sp.index_dim, "block": sp.block,
-                           "topk": sp.topk, "parallelism": f"dp{world} (independent sequences)",
+                           "topk": sp.topk, "parallelism": parallelism,
                            "l2": "inputs larger than L2 (Q 2 GiB, K/V 512 MiB per step)"},
                 "gpu_launches": res["gpu_launches"], "roofline": res["roofline"],
                 "stages": res["stages"], "kernels_ms_per_launch": res["kernels_ms_per_launch"],

@@ -11,3 +11,5 @@ from .msa import (  # noqa: F401
     profile_read, OP_INDEX_SCORES, OP_BLOCK_TOPK, OP_SPARSE_PREFILL, OP_SPARSE_DECODE, OP_FORWARD,
     OP_DENSE_PREFILL, OP_DENSE_DECODE, OP_FORWARD_ALIGNMENT,
 )
+from . import shard  # noqa: F401,E402
+from .shard import GroupShard, group_shard, shard_inputs, forward_group_shard  # noqa: F401,E402

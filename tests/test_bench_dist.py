@@ -2,8 +2,10 @@
 
 One process per GPU in the real runs (NCCL); here two host processes stand
 in for them: the rendezvous, the max-over-ranks timing, the barrier, the
-per-rank workloads (independent sequences: no exchange inside the layer) and
-the reference arm, which rank 0 alone runs.
+per-rank workloads (independent sequences: no exchange inside the layer),
+the group-sharded mode (each rank owns half of one sequence's KV groups; the
+oracle run on each shard, gathered over the ranks, must equal the unsharded
+layer) and the reference arm, which rank 0 alone runs.
 """
 import os
 import socket
@@ -39,6 +41,25 @@ def _rank_main(rank, world, port, out_dir):
     res["seed"] = sp.seed
     q = synth.make_tensor(sp, "q")
     res["q_head"] = q.flatten()[:8].float().tolist()
+    # group sharding: the oracle on this rank's groups, gathered along heads
+    import numpy as np
+    import oracle as O
+    gsp = synth.WorkloadSpec(1, 200, 1000, 800, 16, 4, 64, 32, 128, 4, seed=9)
+    pos = np.arange(gsp.q_offset, gsp.q_offset + gsp.seq_q)
+    gs, (q, k, v, qi, ki) = bench.group_shard_inputs(gsp, rank, w, "cpu")
+    o, _, sel, _ = O.msa_forward(q[0], k[0], v[0], qi[0], ki[0], pos, gsp.block, gsp.topk)
+    parts = [torch.empty((gsp.seq_q, gs.shape.n_q_heads, gsp.head_dim), dtype=torch.float64)
+             for _ in range(w)]
+    pg.all_gather(parts, torch.from_numpy(np.ascontiguousarray(o)))
+    sels = [torch.empty(tuple(sel.shape), dtype=torch.int32) for _ in range(w)]
+    pg.all_gather(sels, torch.from_numpy(np.ascontiguousarray(sel)))
+    res["heads"] = gs.heads
+    if rank == 0:
+        full = synth.make_inputs(gsp)
+        o_f, _, sel_f, _ = O.msa_forward(full.q[0], full.k[0], full.v[0], full.q_idx[0],
+                                         full.k_idx[0], pos, gsp.block, gsp.topk)
+        res["group_o_equal"] = bool(np.array_equal(torch.cat(parts, 1).numpy(), o_f))
+        res["group_sel_equal"] = bool(np.array_equal(torch.cat(sels, 1).numpy(), sel_f))
     line = bench.run_reference(args, w, r, pg)
     res["ref"] = None if line is None else sorted(line)
     bench.barrier(pg)
@@ -57,4 +78,6 @@ def test_two_ranks_over_gloo(tmp_path):
     assert res[0]["seed"] != res[1]["seed"]       # independent sequences per rank
     assert res[0]["q_head"] != res[1]["q_head"]
     assert res[1]["ref"] is None                  # the reference arm runs on rank 0 only
+    assert res[0]["heads"] == (0, 8) and res[1]["heads"] == (8, 16)
+    assert res[0]["group_o_equal"] and res[0]["group_sel_equal"]
     assert {"impl", "metric", "value", "unit", "cpu_baseline", "e2e"} <= set(res[0]["ref"])

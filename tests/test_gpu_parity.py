@@ -276,6 +276,32 @@ def test_forward_alignment_kl(sp):
             assert np.abs(kl_ref).max() <= 1e-12 and np.abs(got).max() <= 1e-5
 
 
+@pytest.mark.parametrize("world", [2, 4])
+def test_group_sharded_forward(world):
+    """Every rank's group shard as its own msa_forward (run one after another on
+    one GPU: the shards never wait on one another): selection bit-exact with the
+    oracle on the shard and with the unsharded run's groups, outputs against the
+    oracle on the shard."""
+    sp = spec(1, 300, 1000, 700, 16, 4, 64, 64, 5, seed=71)
+    inp = inputs_cpu(sp)
+    sh = M.Shape.of(sp)
+    _, _, sel_full = M.forward(sh, cuda(inp.q), cuda(inp.k), cuda(inp.v), cuda(inp.q_idx),
+                               cuda(inp.k_idx))
+    pos = positions(sp)
+    for rank in range(world):
+        gs = M.group_shard(sh, rank, world)
+        q, k, v, qi, ki = M.shard_inputs(gs, inp.q, inp.k, inp.v, inp.q_idx, inp.k_idx)
+        o, _, sel = M.forward_group_shard(gs, cuda(q), cuda(k), cuda(v), cuda(qi), cuda(ki))
+        torch.cuda.synchronize()
+        sref = O.block_topk(O.index_pooled(qi[0], ki[0], pos, sp.block), pos, sp.block, sp.topk)
+        g0, g1 = gs.groups
+        assert np.array_equal(sel[0].cpu().numpy(), sref)
+        assert torch.equal(sel[0].cpu(), sel_full[0, :, g0:g1].cpu())
+        O_ref, _ = O.sparse_attention(q[0], k[0], v[0], sref, pos, sp.block)
+        check_attn(o[0], O_ref, f"group shard {rank}/{world}")
+    assert M.device_status() == 0
+
+
 def test_device_status_clean():
     assert M.device_status() == 0
 
