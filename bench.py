@@ -219,6 +219,18 @@ def topk_bytes(sp):
     return float(sp.batch * sp.n_kv_heads * (4 * bt.sum() + 4 * sp.topk * sp.seq_q))
 
 
+def prefill_step_bound(sp, sel, peaks, ms):
+    """The whole prefill step against the sum of its steps' bounds (the
+    selection inversion and the combine are implementation steps with no
+    algorithmic bound of their own)."""
+    tpk = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]) * 1e12
+    bound_ms = 1e3 * (index_flops(sp) / tpk + topk_bytes(sp) / (peaks["hbm_gbs"] * 1e9)
+                      + selected_attention_flops(sp, sel) / tpk)
+    return {"ms_at_bounds": round(bound_ms, 3), "frac": round(bound_ms / ms, 4),
+            "terms": "index FLOP and selected-attention FLOP at sustained bf16, "
+                     "top-k bytes at HBM copy bandwidth"}
+
+
 def decode_kv_bytes(sp):
     return float(sp.batch * sp.n_kv_heads * sp.topk * 128 * sp.head_dim * 2 * 2)
 
@@ -306,6 +318,7 @@ def run_msa(args, world, rank, pg):
             stages[name] = {"ms": round(kernels[name], 4), "achieved": round(a, 2),
                             "frac": round(a / pk, 4)}
     out["stages"] = stages
+    out["step_roofline"] = prefill_step_bound(sp, sel, peaks, ms)
 
     # ---- the same workload through the dense causal GQA kernel (the baseline
     # the pages compare MSA against)
@@ -470,6 +483,10 @@ def run_decode(M, sp, args, pg, stream, world, peaks, dense):
     b = float(sp.batch * sp.seq_kv * sp.index_dim * 2)
     a = b / (kernels["index_scores"] / 1e3) / 1e9
     res["index_scan"] = {"achieved_gbs": round(a, 1), "frac": round(a / peaks["hbm_gbs"], 4)}
+    step_bytes = b + topk_bytes(sp) + decode_kv_bytes(sp)
+    bound_ms = 1e3 * step_bytes / (peaks["hbm_gbs"] * 1e9)
+    res["step_roofline"] = {"ms_at_bounds": round(bound_ms, 4), "frac": round(bound_ms / ms, 4),
+                            "terms": "k_idx scan + top-k + selected K/V bytes at HBM copy bandwidth"}
     del pooled, aws
     if dense:
         dws = M.alloc_workspace(sh, M.OP_DENSE_DECODE)
@@ -523,6 +540,7 @@ def run_long(M, args, pg, stream, world, rank, peaks):
                                     "speedup_msa_vs_dense": round(dms / ms, 2)}
     except M.MsaError as e:
         pre["dense_gqa_prefill"] = {"unavailable": str(e)}
+    pre["step_roofline"] = prefill_step_bound(sp, sel, peaks, ms)
     res["prefill"] = pre
     del inp, ws, o, sel
     torch.cuda.empty_cache()
@@ -678,7 +696,8 @@ def main():
                 "gpu_launches": res["gpu_launches"], "roofline": res["roofline"],
                 "stages": res["stages"], "kernels_ms_per_launch": res["kernels_ms_per_launch"],
                 "clocks": res["clocks"]}
-        for key in ("e2e", "dense_gqa_prefill", "topk_microbench", "decode", "ctx_1m"):
+        for key in ("step_roofline", "e2e", "dense_gqa_prefill", "topk_microbench", "decode",
+                    "ctx_1m"):
             if key in res:
                 line[key] = res[key]
         if world == 1 and not args.skip_cpu:
