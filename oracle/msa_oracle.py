@@ -48,8 +48,13 @@ Readings where the pages are silent (each listed in the design notes):
     P_index(b) = softmax over the selected blocks of the raw pooled index
     scores (no temperature), KL(P_main || P_index) in natural log.
 
-Precision: float64 throughout.  Parity of the attention outputs is unpinned
-beyond the special cases the tests check (dense equivalence, closed forms).
+Precision: float64 throughout.  Pins (tests/test_oracle_pins.py), each
+independent of this module's code: pooled scores by brute force and one-hot
+keys; the selection by a beaten-by-count definition with ties; the attention
+by torch SDPA (causal GQA when k covers every block, gathered keys, and a
+boolean block mask built from the definition over random selections) and by
+closed forms; the alignment KL by closed forms.  The pages print no worked
+example of an attention output, so none of the pins is a page value.
 """
 from __future__ import annotations
 

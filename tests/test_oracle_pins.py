@@ -199,6 +199,40 @@ def test_sparse_attention_is_dense_over_selected_keys():
     assert np.abs(L[0] - np.log(np.exp(logits).sum(axis=1))).max() < 1e-12
 
 
+def test_sparse_attention_equals_block_masked_sdpa():
+    # many rows, several groups, random selections: the oracle's gathered-key
+    # attention against SDPA over every key with a boolean mask built from the
+    # definition (key j of group g is attended by row t iff block(j) is in
+    # sel[t, g] and j <= p_t); ragged tail (N not a multiple of B)
+    rng = np.random.default_rng(15)
+    T, H, G, d, B, N, k = 40, 6, 2, 8, 8, 61, 3
+    q = rng.normal(size=(T, H, d)); kk = rng.normal(size=(G, N, d)); v = rng.normal(size=(G, N, d))
+    pos = rng.integers(0, N, size=T)
+    pos[:3] = [0, N - 1, 2 * B]
+    sel = np.full((T, G, k), -1, dtype=np.int32)
+    for t in range(T):
+        bt = pos[t] // B
+        for g in range(G):
+            others = rng.permutation(bt)[:k - 1]
+            sel[t, g, :len(others) + 1] = sorted(list(others) + [bt])
+    Os, L = O.sparse_attention(q, kk, v, sel, pos, B)
+    r = H // G
+    mask = np.zeros((H, T, N), dtype=bool)
+    for t in range(T):
+        for h in range(H):
+            blocks = set(int(b) for b in sel[t, h // r] if b >= 0)
+            mask[h, t] = [(j // B in blocks) and j <= pos[t] for j in range(N)]
+    qt = torch.from_numpy(q).permute(1, 0, 2)[None]
+    kt = torch.from_numpy(kk).repeat_interleave(r, dim=0)[None]
+    vt = torch.from_numpy(v).repeat_interleave(r, dim=0)[None]
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        qt, kt, vt, attn_mask=torch.from_numpy(mask)[None])[0].permute(1, 0, 2).numpy()
+    assert np.abs(Os - ref).max() < 1e-12
+    logits = np.einsum("thd,hnd->htn", q, np.repeat(kk, r, axis=0)) / math.sqrt(d)
+    lse = np.log(np.where(mask, np.exp(logits), 0.0).sum(axis=2)).T
+    assert np.abs(L - lse).max() < 1e-12
+
+
 def test_two_key_closed_form_and_scale():
     d = 4
     q = np.zeros((1, 1, d)); q[0, 0, 0] = 2.0            # logit = 2 * k0 / sqrt(4)
