@@ -418,8 +418,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         o_acc[nt][2] *= corr[1];
         o_acc[nt][3] *= corr[1];
       }
-      // ---- O[:, w*D/8 ..] += P V over the block's 128 keys
+      // ---- O[:, w*D/8 ..] += P V over the block's 128 keys.  Keys past the
+      // query have P = 0, but their V rows can hold anything (a ragged cache
+      // past its length), and 0 * NaN is NaN: in the block that holds the
+      // query, those rows are zeroed in the B fragments.  Register j of a
+      // fragment holds keys ks*16 + 8*(j&1) + 2*qd + {0 (low half), 1}.
       const int mi = lane >> 3, ri = lane & 7;
+      const bool past_query = blk * 128 + 127 > pos;
 #pragma unroll
       for (int ks = 0; ks < 8; ++ks) {
         uint32_t pa[4];
@@ -427,16 +432,20 @@ __global__ void __launch_bounds__(kThreads, 1)
                                               (ks * 16 + (mi >> 1) * 8) * 2),
                 pa);
         const int vkey = ks * 16 + (mi & 1) * 8 + ri;
-        if constexpr (NW == 2) {
-          uint32_t vb[4];
+        uint32_t vb[2 * NW];
+        if constexpr (NW == 2)
           ldsm_x4_trans(vbase + sw128_off(vkey, w * 16 + (mi >> 1) * 8), vb);
-          mma16816(o_acc[0], pa, vb);
-          mma16816(o_acc[1], pa, vb + 2);
-        } else {
-          uint32_t vb[2];
+        else
           ldsm_x2_trans(vbase + sw128_off(vkey, w * 8), vb);
-          mma16816(o_acc[0], pa, vb);
+        if (past_query) {
+#pragma unroll
+          for (int j = 0; j < 2 * NW; ++j) {
+            const int k0 = blk * 128 + ks * 16 + 8 * (j & 1) + 2 * qd;
+            vb[j] &= (k0 <= pos ? 0x0000FFFFu : 0u) | (k0 + 1 <= pos ? 0xFFFF0000u : 0u);
+          }
         }
+        mma16816(o_acc[0], pa, vb);
+        if constexpr (NW == 2) mma16816(o_acc[1], pa, vb + 2);
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&empty[s]);

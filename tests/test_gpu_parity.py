@@ -340,6 +340,38 @@ def test_forward_decode_ragged(sp, lens):
     assert np.abs(lse.double().cpu().numpy() - np.stack(l_ref)).max() < LSE_ABS
 
 
+@pytest.mark.parametrize("sp,lens", [
+    (spec(4, 1, 3000, 2999, 16, 2, 128, 64, 4, seed=54), [1, 130, 1000, 2050]),
+    (spec(3, 1, 2000, 1999, 8, 4, 64, 32, 5, seed=55), [7, 500, 1999]),
+])
+def test_forward_decode_ragged_ignores_rows_past_length(sp, lens):
+    """Cache rows past each sequence's length hold NaN and Inf (memory a
+    serving cache has not written yet): selections and outputs are those of
+    the oracle on the clean cache."""
+    inp = inputs_cpu(sp)
+    k, v, ki = inp.k.clone(), inp.v.clone(), inp.k_idx.clone()
+    for b, n in enumerate(lens):
+        k[b, :, n:] = float("nan")
+        v[b, :, n::2] = float("inf")
+        v[b, :, n + 1::2] = float("nan")
+        ki[b, n:] = float("nan")
+    sh = M.Shape.of(sp)
+    seq_lens = cuda(torch.tensor(lens, dtype=torch.int32))
+    o, lse, sel = M.forward_decode_ragged(sh, cuda(inp.q), cuda(k), cuda(v), cuda(inp.q_idx),
+                                          cuda(ki), seq_lens)
+    torch.cuda.synchronize()
+    assert M.device_status() == 0
+    o_ref = []
+    for b, n in enumerate(lens):
+        pos = np.array([n - 1])
+        sref = O.block_topk(O.index_pooled(inp.q_idx[b], inp.k_idx[b], pos, sp.block), pos,
+                            sp.block, sp.topk)
+        assert np.array_equal(sel[b].cpu().numpy(), sref), f"sel b={b} len={n}"
+        o_ref.append(O.sparse_attention(inp.q[b], inp.k[b], inp.v[b], sref, pos, sp.block)[0])
+    check_attn(o, np.stack(o_ref), "ragged decode over a poisoned tail")
+    assert torch.isfinite(lse).all()
+
+
 def test_forward_decode_ragged_length_out_of_range():
     # lengths 0 and capacity+5 are clamped to 1 and capacity; the kernels flag them
     sp = spec(2, 1, 1000, 999, 8, 2, 64, 32, 4, seed=53)
