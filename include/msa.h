@@ -185,10 +185,11 @@ msa_status msa_forward_alignment(const msa_shape* shape, const uint16_t* q,
  * its local block is (seq_lens[b] - 1) / 128 and only its causal blocks are
  * scored and selected.  seq_lens: device int32 [B], 4-byte aligned, each in
  * [1, seq_kv]; shape.seq_kv is the cache capacity (row stride of k, v,
- * k_idx) and shape.q_offset is ignored.  A length outside [1, seq_kv] is
- * clamped into it and sets bit 1 of the device error word.  Same layouts,
- * outputs and workspace (msa_workspace_size(MSA_OP_FORWARD) with T == 1) as
- * msa_forward. */
+ * k_idx) and shape.q_offset is ignored.  Cache rows at or past seq_lens[b]
+ * may hold any bits (NaN and Inf included): they never reach a result.  A
+ * length outside [1, seq_kv] is clamped into it and sets bit 1 of the device
+ * error word.  Same layouts, outputs and workspace (msa_workspace_size(
+ * MSA_OP_FORWARD) with T == 1) as msa_forward. */
 msa_status msa_forward_decode_ragged(const msa_shape* shape, const int32_t* seq_lens,
                                      const uint16_t* q, const uint16_t* k, const uint16_t* v,
                                      const uint16_t* q_idx, const uint16_t* k_idx, uint16_t* o,
