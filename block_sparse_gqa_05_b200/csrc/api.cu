@@ -312,6 +312,43 @@ msa_status msa_sparse_attn_decode(const msa_shape* s, const uint16_t* q, const u
 }  // extern "C"
 
 namespace msa {
+// One decode step over caches with per-sequence lengths, contiguous
+// (pages.table == nullptr) or paged: the ragged and paged entry points.
+msa_status forward_decode_lens(const msa_shape* s, const int32_t* seq_lens, PageTable pages,
+                               const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                               const uint16_t* q_idx, const uint16_t* k_idx, uint16_t* o,
+                               float* lse, int32_t* sel_out, void* ws, size_t ws_bytes,
+                               void* stream) {
+  if (!s) return MSA_ERR_NULL_PTR;
+  if (s->seq_q != 1) return MSA_ERR_INVALID_SHAPE;
+  // seq_kv is the cache capacity; each sequence's own length comes from seq_lens
+  msa_shape c = *s;
+  c.q_offset = c.seq_kv - 1;
+  msa_status st = check_shape(&c, true, true);
+  if (st != MSA_OK) return st;
+  if ((st = check_attn_ptrs(q, k, v, nullptr, false, o, lse)) != MSA_OK) return st;
+  if (!q_idx || !k_idx || !seq_lens) return MSA_ERR_NULL_PTR;
+  if (!aligned16(q_idx) || !aligned16(k_idx) || (sel_out && !aligned16(sel_out)) ||
+      !aligned4(seq_lens))
+    return MSA_ERR_MISALIGNED;
+  size_t need = 0;
+  if ((st = msa_workspace_size(&c, MSA_OP_FORWARD, &need)) != MSA_OK) return st;
+  if (!ws) return MSA_ERR_NULL_PTR;
+  if (ws_bytes < need) return MSA_ERR_WORKSPACE_TOO_SMALL;
+  if (!aligned16(ws)) return MSA_ERR_MISALIGNED;
+  if (!device_ctx()) return MSA_ERR_CUDA;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  char* w = static_cast<char*>(ws);
+  float* pooled = reinterpret_cast<float*>(w);
+  int32_t* sel = sel_out ? sel_out : reinterpret_cast<int32_t*>(w + pooled_bytes(c));
+  void* rest = w + pooled_bytes(c) + sel_bytes(c);
+  cudaError_t e = launch_index_scores(c, q_idx, k_idx, pooled, false, cs, seq_lens, pages);
+  if (e == cudaSuccess) e = launch_block_topk(c, pooled, sel, cs, seq_lens);
+  if (e == cudaSuccess)
+    e = launch_decode(c, q, k, v, sel, o, lse, rest, false, cs, seq_lens, pages);
+  return from_cuda(e);
+}
+
 // Argument checks of the decode entry point without a workspace argument.
 msa_status check_decode_static_args(const msa_shape* s, const uint16_t* q, const uint16_t* k,
                                     const uint16_t* v, const int32_t* sel, const uint16_t* o,
@@ -390,33 +427,28 @@ msa_status msa_forward_decode_ragged(const msa_shape* s, const int32_t* seq_lens
                                      const uint16_t* q_idx, const uint16_t* k_idx, uint16_t* o,
                                      float* lse, int32_t* sel_out, void* ws, size_t ws_bytes,
                                      void* stream) {
+  return forward_decode_lens(s, seq_lens, PageTable{}, q, k, v, q_idx, k_idx, o, lse, sel_out,
+                             ws, ws_bytes, stream);
+}
+
+msa_status msa_forward_decode_paged(const msa_shape* s, int num_pages, const int32_t* seq_lens,
+                                    const int32_t* page_table, const uint16_t* q,
+                                    const uint16_t* k, const uint16_t* v, const uint16_t* q_idx,
+                                    const uint16_t* k_idx, uint16_t* o, float* lse,
+                                    int32_t* sel_out, void* ws, size_t ws_bytes, void* stream) {
   if (!s) return MSA_ERR_NULL_PTR;
-  if (s->seq_q != 1) return MSA_ERR_INVALID_SHAPE;
-  // seq_kv is the cache capacity; each sequence's own length comes from seq_lens
-  msa_shape c = *s;
-  c.q_offset = c.seq_kv - 1;
-  msa_status st = check_shape(&c, true, true);
-  if (st != MSA_OK) return st;
-  if ((st = check_attn_ptrs(q, k, v, nullptr, false, o, lse)) != MSA_OK) return st;
-  if (!q_idx || !k_idx || !seq_lens) return MSA_ERR_NULL_PTR;
-  if (!aligned16(q_idx) || !aligned16(k_idx) || (sel_out && !aligned16(sel_out)) ||
-      (reinterpret_cast<uintptr_t>(seq_lens) & 3u) != 0)
-    return MSA_ERR_MISALIGNED;
-  size_t need = 0;
-  if ((st = msa_workspace_size(&c, MSA_OP_FORWARD, &need)) != MSA_OK) return st;
-  if (!ws) return MSA_ERR_NULL_PTR;
-  if (ws_bytes < need) return MSA_ERR_WORKSPACE_TOO_SMALL;
-  if (!aligned16(ws)) return MSA_ERR_MISALIGNED;
-  if (!device_ctx()) return MSA_ERR_CUDA;
-  cudaStream_t cs = static_cast<cudaStream_t>(stream);
-  char* w = static_cast<char*>(ws);
-  float* pooled = reinterpret_cast<float*>(w);
-  int32_t* sel = sel_out ? sel_out : reinterpret_cast<int32_t*>(w + pooled_bytes(c));
-  void* rest = w + pooled_bytes(c) + sel_bytes(c);
-  cudaError_t e = launch_index_scores(c, q_idx, k_idx, pooled, false, cs, seq_lens);
-  if (e == cudaSuccess) e = launch_block_topk(c, pooled, sel, cs, seq_lens);
-  if (e == cudaSuccess) e = launch_decode(c, q, k, v, sel, o, lse, rest, false, cs, seq_lens);
-  return from_cuda(e);
+  if (num_pages < 1) return MSA_ERR_INVALID_SHAPE;
+  // 32-bit TMA coordinates (page*G + g) and index-key row offsets
+  if (static_cast<int64_t>(num_pages) * s->n_kv_heads >= (1ll << 31) ||
+      static_cast<int64_t>(num_pages) * 128 >= (1ll << 31))
+    return MSA_ERR_UNSUPPORTED;
+  if (!page_table) return MSA_ERR_NULL_PTR;
+  if ((reinterpret_cast<uintptr_t>(page_table) & 3u) != 0) return MSA_ERR_MISALIGNED;
+  PageTable pt;
+  pt.table = page_table;
+  pt.num_pages = num_pages;
+  return forward_decode_lens(s, seq_lens, pt, q, k, v, q_idx, k_idx, o, lse, sel_out, ws,
+                             ws_bytes, stream);
 }
 
 msa_status msa_dense_attn_prefill(const msa_shape* s, const uint16_t* q, const uint16_t* k,

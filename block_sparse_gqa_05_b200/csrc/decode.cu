@@ -15,7 +15,8 @@
 // items all fall in one CTA is written directly; one that spans CTAs leaves
 // a normalised partial per CTA, merged by the last CTA to finish it (chosen
 // by an atomic counter: no CTA ever waits for another).  The kernel is bound
-// by HBM bandwidth on the K/V bytes.
+// by HBM bandwidth on the K/V bytes.  With a page table the K/V tile of
+// logical block j of a sequence is read from that block's page.
 #include <math.h>
 
 #include <mutex>
@@ -37,6 +38,8 @@ struct DecParams {
   const uint16_t* q;      // [B, 1, H, d]
   const int32_t* sel;     // [B, 1, G, k] (sparse) or nullptr (dense)
   const int32_t* lens;    // [B] cache lengths (ragged decode) or nullptr: all N
+  const int32_t* pages;   // [B, nb] page of each logical block, or nullptr (contiguous)
+  int num_pages, nb;
   uint16_t* o;            // [B, 1, H, d]
   float* lse;             // [B, 1, H] or nullptr
   uint32_t* counters;     // [B*G] CTAs done with a (sequence, group)
@@ -174,12 +177,23 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (long long base = i0; ok && base < i1; base += 32) {
       int bgv = 0;
       const int blk = base + lane < i1 ? item_block(p, base + lane, &bgv) : -1;
+      // TMA coordinates of the block's rows: (row, sequence*G + group) in a
+      // contiguous cache, (0, page*G + group) in a paged one
+      int yv = 0, zv = 0;
+      if (blk >= 0) {
+        if (p.pages) {
+          zv = page_of(p.pages, p.nb, p.num_pages, bgv / p.G, blk, p.err) * p.G + bgv % p.G;
+        } else {
+          yv = blk * 128;
+          zv = bgv;
+        }
+      }
       unsigned m = __ballot_sync(0xffffffffu, blk >= 0);
       while (m) {
         const int src = __ffs(m) - 1;
         m &= m - 1;
-        const int b_ = __shfl_sync(0xffffffffu, blk, src);
-        const int bg_ = __shfl_sync(0xffffffffu, bgv, src);
+        const int y_ = __shfl_sync(0xffffffffu, yv, src);
+        const int z_ = __shfl_sync(0xffffffffu, zv, src);
         const int s = cnt % S;
         if (lane == 0) {
           ok = mbar_wait(&empty[s], ((cnt / S) & 1) ^ 1, abort_flag, p.err);
@@ -187,13 +201,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_arrive_expect_tx(&kfull[s], L::kTile);
 #pragma unroll
             for (int c = 0; c < D / 64; ++c)
-              tma_load_3d(smem + s * 2 * L::kTile + c * 16384, &tm_k, &kfull[s], c * 64, b_ * 128,
-                          bg_);
+              tma_load_3d(smem + s * 2 * L::kTile + c * 16384, &tm_k, &kfull[s], c * 64, y_, z_);
             mbar_arrive_expect_tx(&vfull[s], L::kTile);
 #pragma unroll
             for (int c = 0; c < D / 64; ++c)
               tma_load_3d(smem + s * 2 * L::kTile + L::kTile + c * 16384, &tm_v, &vfull[s],
-                          c * 64, b_ * 128, bg_);
+                          c * 64, y_, z_);
           }
         }
         ok = __shfl_sync(0xffffffffu, ok, 0) != 0;
@@ -554,7 +567,8 @@ size_t decode_workspace_bytes(const msa_shape& s, bool dense) {
 
 cudaError_t launch_decode(const msa_shape& s, const uint16_t* q, const uint16_t* k,
                           const uint16_t* v, const int32_t* sel, uint16_t* o, float* lse,
-                          void* ws, bool dense, cudaStream_t st, const int32_t* lens) {
+                          void* ws, bool dense, cudaStream_t st, const int32_t* lens,
+                          PageTable pages) {
   const DevCtx* ctx = device_ctx();
   if (!ctx) return cudaErrorInitializationError;
   const int r = s.n_q_heads / s.n_kv_heads;
@@ -572,6 +586,9 @@ cudaError_t launch_decode(const msa_shape& s, const uint16_t* q, const uint16_t*
   p.q = q;
   p.sel = dense ? nullptr : sel;
   p.lens = lens;
+  p.pages = pages.table;
+  p.num_pages = pages.num_pages;
+  p.nb = static_cast<int>(ceil_div(s.seq_kv, 128));
   p.o = o;
   p.lse = lse;
   p.err = ctx->err;
@@ -586,10 +603,12 @@ cudaError_t launch_decode(const msa_shape& s, const uint16_t* q, const uint16_t*
   if (n_items == 0) return cudaSuccess;
 
   CUtensorMap tk, tv;
-  const uint64_t dims[3] = {static_cast<uint64_t>(s.head_dim), static_cast<uint64_t>(s.seq_kv),
-                            static_cast<uint64_t>(bg)};
+  // contiguous: [B*G][N][d]; paged: [num_pages*G][128][d]
+  const uint64_t rows = pages.table ? 128 : static_cast<uint64_t>(s.seq_kv);
+  const uint64_t mats = pages.table ? static_cast<uint64_t>(pages.num_pages) * s.n_kv_heads : bg;
+  const uint64_t dims[3] = {static_cast<uint64_t>(s.head_dim), rows, mats};
   const uint64_t strides[2] = {static_cast<uint64_t>(s.head_dim) * 2,
-                               static_cast<uint64_t>(s.seq_kv) * s.head_dim * 2};
+                               rows * s.head_dim * 2};
   const uint32_t box[3] = {64, 128, 1};
   if (!encode_tmap(&tk, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, k, dims, strides, box,
                    CU_TENSOR_MAP_SWIZZLE_128B) ||

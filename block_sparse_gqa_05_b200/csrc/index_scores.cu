@@ -266,7 +266,9 @@ __global__ void fill_upper_kernel(float* pooled, long long rows, int T, int G, i
 }
 
 // --------------------------------------------------------------- decode scan
-// One CTA per (sequence*T + t, chunk of 8 blocks); warp w owns block 8*chunk+w.
+// One CTA per (sequence*T + t, chunk of 8 blocks) (rows on grid.x, which has
+// no 65535 limit); warp w owns block 8*chunk+w.  With a page table the 128
+// index-key rows of a block are those of its page.
 // S[key, group] = k_idx[key, :] . q_idx[t, group, :] on mma.sync m16n8k16 with
 // the 16 keys of a tile as rows and 8 groups as columns.  The K dimension is
 // permuted identically for both operands so that each thread reads contiguous
@@ -286,20 +288,24 @@ __global__ void __launch_bounds__(256) index_scores_scan_kernel(const uint16_t* 
                                                                 float* __restrict__ pooled, int T,
                                                                 int N, int G, int q_off, int nb,
                                                                 const int32_t* __restrict__ lens,
-                                                                uint32_t* err) {
+                                                                const int32_t* __restrict__ pages,
+                                                                int num_pages, uint32_t* err) {
   constexpr int KS = DI / 16;          // k-steps
   constexpr int W = KS * 2;            // 32-bit words per thread per row
-  const int row_bt = blockIdx.y;       // seq * T + t
+  const int row_bt = blockIdx.x;       // seq * T + t
   const int seq = row_bt / T;
   const int t = row_bt - seq * T;
   // ragged decode: the query sits at the end of its own cache
   const int pos = lens ? ragged_len(lens, seq, N, err) - 1 : q_off + t;
   const int bt = pos >> 7;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int blk = blockIdx.x * 8 + warp;
+  const int blk = blockIdx.y * 8 + warp;
   if (blk > bt) return;
   const int gq = lane >> 2, qd = lane & 3;
-  const uint16_t* kbase = k_idx + static_cast<long long>(seq) * N * DI;
+  // the block's 128 index-key rows (rows past N exist only in a page)
+  const uint16_t* kblk =
+      pages ? k_idx + static_cast<long long>(page_of(pages, nb, num_pages, seq, blk, err)) * 128 * DI
+            : k_idx + (static_cast<long long>(seq) * N + blk * 128) * DI;
   for (int g0 = 0; g0 < G; g0 += 8) {
     // B operand: index query of group g0 + gq, this thread's dim range
     uint32_t bw[W];
@@ -320,7 +326,7 @@ __global__ void __launch_bounds__(256) index_scores_scan_kernel(const uint16_t* 
       const int key1 = key0 + 8;
       uint32_t r0[W], r1[W];
       if (key0 < N) {
-        const uint4* s0 = reinterpret_cast<const uint4*>(kbase + static_cast<long long>(key0) * DI +
+        const uint4* s0 = reinterpret_cast<const uint4*>(kblk + (tile * 16 + gq) * DI +
                                                          qd * 4 * KS);
 #pragma unroll
         for (int x = 0; x < W / 4; ++x) {
@@ -332,7 +338,7 @@ __global__ void __launch_bounds__(256) index_scores_scan_kernel(const uint16_t* 
         for (int x = 0; x < W; ++x) r0[x] = 0u;
       }
       if (key1 < N) {
-        const uint4* s1 = reinterpret_cast<const uint4*>(kbase + static_cast<long long>(key1) * DI +
+        const uint4* s1 = reinterpret_cast<const uint4*>(kblk + (tile * 16 + gq + 8) * DI +
                                                          qd * 4 * KS);
 #pragma unroll
         for (int x = 0; x < W / 4; ++x) {
@@ -423,33 +429,29 @@ cudaError_t launch_tc(const msa_shape& s, const uint16_t* q_idx, const uint16_t*
 
 cudaError_t launch_index_scores(const msa_shape& s, const uint16_t* q_idx, const uint16_t* k_idx,
                                 float* pooled, bool fill_upper, cudaStream_t st,
-                                const int32_t* lens) {
+                                const int32_t* lens, PageTable pages) {
   const DevCtx* ctx = device_ctx();
   if (!ctx) return cudaErrorInitializationError;
   const int nb = static_cast<int>(ceil_div(s.seq_kv, 128));
   const long long rows = static_cast<long long>(s.batch) * s.seq_q * s.n_kv_heads;
   cudaError_t e;
   // the tensor-core path needs a full 128-row query tile and a 256-key box;
-  // ragged decode always scans
-  if (lens || static_cast<long long>(s.seq_q) * s.n_kv_heads < 128 ||
+  // ragged and paged decode always scan
+  if (lens || pages.table || static_cast<long long>(s.seq_q) * s.n_kv_heads < 128 ||
       static_cast<long long>(s.batch) * s.seq_kv < 256) {
     const int last_bt = (s.q_offset + s.seq_q - 1) / 128;
-    dim3 grid(static_cast<unsigned>(ceil_div(last_bt + 1, 8)),
-              static_cast<unsigned>(s.batch * s.seq_q));
+    const dim3 grid(static_cast<unsigned>(s.batch * s.seq_q),
+                    static_cast<unsigned>(ceil_div(last_bt + 1, 8)));
+    if (grid.y > 65535u) return cudaErrorInvalidConfiguration;
+    ProfScope ps_("index_scores_scan", st);
     if (s.index_dim == 64)
-      {
-    ProfScope ps_("index_scores_scan", st);
-    index_scores_scan_kernel<64><<<grid, 256, 0, st>>>(q_idx, k_idx, pooled, s.seq_q, s.seq_kv,
+      index_scores_scan_kernel<64><<<grid, 256, 0, st>>>(q_idx, k_idx, pooled, s.seq_q, s.seq_kv,
                                                          s.n_kv_heads, s.q_offset, nb, lens,
-                                                         ctx->err);
-  }
+                                                         pages.table, pages.num_pages, ctx->err);
     else
-      {
-    ProfScope ps_("index_scores_scan", st);
-    index_scores_scan_kernel<32><<<grid, 256, 0, st>>>(q_idx, k_idx, pooled, s.seq_q, s.seq_kv,
+      index_scores_scan_kernel<32><<<grid, 256, 0, st>>>(q_idx, k_idx, pooled, s.seq_q, s.seq_kv,
                                                          s.n_kv_heads, s.q_offset, nb, lens,
-                                                         ctx->err);
-  }
+                                                         pages.table, pages.num_pages, ctx->err);
     e = cudaGetLastError();
   } else {
     e = s.index_dim == 64 ? launch_tc<64>(s, q_idx, k_idx, pooled, ctx, st)

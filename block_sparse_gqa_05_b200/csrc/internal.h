@@ -45,9 +45,17 @@ inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 // Each returns cudaSuccess or the launch error.  Shapes are already validated.
 // lens (device, [B], may be null): per-sequence cache lengths of ragged decode;
 // the query of sequence b then sits at position lens[b] - 1.
+// Paged caches (decode): one 128-row block per page, table [B, nb] of page
+// ids; k_idx then holds [num_pages, 128, d_i] rows and k, v [num_pages, G,
+// 128, d].  table == nullptr: contiguous caches.
+struct PageTable {
+  const int32_t* table = nullptr;
+  int num_pages = 0;
+};
 cudaError_t launch_index_scores(const msa_shape& s, const uint16_t* q_idx,
                                 const uint16_t* k_idx, float* pooled, bool fill_upper,
-                                cudaStream_t st, const int32_t* lens = nullptr);
+                                cudaStream_t st, const int32_t* lens = nullptr,
+                                PageTable pages = PageTable{});
 cudaError_t launch_block_topk(const msa_shape& s, const float* pooled, int32_t* sel,
                               cudaStream_t st, const int32_t* lens = nullptr);
 size_t prefill_workspace_bytes(const msa_shape& s);
@@ -59,7 +67,7 @@ size_t decode_workspace_bytes(const msa_shape& s, bool dense);
 cudaError_t launch_decode(const msa_shape& s, const uint16_t* q, const uint16_t* k,
                           const uint16_t* v, const int32_t* sel, uint16_t* o, float* lse,
                           void* ws, bool dense, cudaStream_t st,
-                          const int32_t* lens = nullptr);
+                          const int32_t* lens = nullptr, PageTable pages = PageTable{});
 msa_status check_decode_static_args(const msa_shape* s, const uint16_t* q, const uint16_t* k,
                                     const uint16_t* v, const int32_t* sel, const uint16_t* o,
                                     const float* lse);

@@ -15,6 +15,7 @@ namespace msa {
 // Device error word bits.
 constexpr uint32_t kErrTimeout = 1u;
 constexpr uint32_t kErrBadLength = 2u;   // a ragged-decode cache length outside [1, N]
+constexpr uint32_t kErrBadPage = 4u;     // a page-table entry outside [0, num_pages)
 // Bound of every mbarrier wait, in nanoseconds of %globaltimer.
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 
@@ -29,6 +30,16 @@ MSA_DEV int ragged_len(const int32_t* lens, int b, int N, uint32_t* err) {
   if (len >= 1 && len <= N) return len;
   atomicOr(err, kErrBadLength);
   return len < 1 ? 1 : N;
+}
+
+// Physical page of logical block blk of sequence b in a paged cache (one
+// 128-row block per page): table[b * nb + blk], clamped into [0, num_pages);
+// an entry outside that range also sets kErrBadPage in the error word.
+MSA_DEV int page_of(const int32_t* table, int nb, int num_pages, int b, int blk, uint32_t* err) {
+  const int pg = table[static_cast<long long>(b) * nb + blk];
+  if (pg >= 0 && pg < num_pages) return pg;
+  atomicOr(err, kErrBadPage);
+  return pg < 0 ? 0 : num_pages - 1;
 }
 
 MSA_DEV uint64_t globaltimer() {

@@ -64,6 +64,9 @@ _SIGS = {
                      ctypes.c_size_t, _vp], ctypes.c_int),
     "msa_forward_alignment": ([ctypes.POINTER(Shape), _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
                                _vp, _vp, ctypes.c_size_t, _vp], ctypes.c_int),
+    "msa_forward_decode_paged": ([ctypes.POINTER(Shape), ctypes.c_int, _vp, _vp, _vp, _vp, _vp,
+                                  _vp, _vp, _vp, _vp, _vp, _vp, ctypes.c_size_t, _vp],
+                                 ctypes.c_int),
     "msa_forward_decode_ragged": ([ctypes.POINTER(Shape), _vp, _vp, _vp, _vp, _vp, _vp, _vp,
                                    _vp, _vp, _vp, ctypes.c_size_t, _vp], ctypes.c_int),
     "msa_dense_attn_prefill": ([ctypes.POINTER(Shape), _vp, _vp, _vp, _vp, _vp, _vp,
@@ -243,6 +246,26 @@ def forward_decode_ragged(shape: Shape, q, k, v, q_idx, k_idx, seq_lens, o=None,
     return o, lse, sel
 
 
+def forward_decode_paged(shape: Shape, q, k_pages, v_pages, q_idx, kidx_pages, seq_lens,
+                         page_table, o=None, lse=None, sel=None, ws=None, want_lse=True,
+                         want_sel=True, stream=None):
+    """msa_forward_decode_paged: one decode step over paged caches.
+    k_pages / v_pages [P, G, 128, d] bf16, kidx_pages [P, 128, d_i] bf16,
+    seq_lens int32 [B], page_table int32 [B, ceil(shape.seq_kv / 128)]."""
+    o, lse = _attn_out(shape, q, o, lse, want_lse)
+    if sel is None and want_sel:
+        sel = torch.empty((shape.batch, 1, shape.n_kv_heads, shape.topk), dtype=torch.int32,
+                          device=q.device)
+    ws = alloc_workspace(shape, OP_FORWARD, q.device) if ws is None else ws
+    _check(lib().msa_forward_decode_paged(ctypes.byref(shape), int(k_pages.shape[0]),
+                                          _ptr(seq_lens), _ptr(page_table), _ptr(q),
+                                          _ptr(k_pages), _ptr(v_pages), _ptr(q_idx),
+                                          _ptr(kidx_pages), _ptr(o), _ptr(lse), _ptr(sel),
+                                          _ptr(ws), ws.numel(), _stream(stream)),
+           "msa_forward_decode_paged")
+    return o, lse, sel
+
+
 def dense_attn_prefill(shape: Shape, q, k, v, o=None, lse=None, want_lse=True, stream=None):
     o, lse = _attn_out(shape, q, o, lse, want_lse)
     _check(lib().msa_dense_attn_prefill(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(o),
@@ -284,7 +307,8 @@ def profile_read() -> dict:
 
 def device_status() -> int:
     """Raw device error word (bit 0: a bounded wait expired; bit 1: a ragged-decode
-    cache length was out of range); clears it."""
+    cache length was out of range; bit 2: a page-table entry was out of range);
+    clears it."""
     f = ctypes.c_uint32(0)
     st = lib().msa_device_status(ctypes.byref(f))
     if st not in (0, 7):

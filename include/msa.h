@@ -196,6 +196,31 @@ msa_status msa_forward_decode_ragged(const msa_shape* shape, const int32_t* seq_
                                      float* lse, int32_t* sel_out, void* ws, size_t ws_bytes,
                                      void* stream);
 
+/* One decode step over paged caches (serving; no counterpart on the pages):
+ * as msa_forward_decode_ragged, except that the caches are stored as
+ * num_pages pages of one 128-row block each and every sequence lists its
+ * pages in a table:
+ *   k, v        [num_pages, G, 128, d]  bf16
+ *   k_idx       [num_pages, 128, d_i]   bf16
+ *   page_table  [B, nb] int32 (device, 4-byte aligned), nb = ceil(seq_kv/128):
+ *               page_table[b, j] is the page holding rows 128j .. 128j+127 of
+ *               sequence b; only entries j <= (seq_lens[b] - 1) / 128 are read.
+ * q, q_idx, o, lse, sel_out, seq_lens, ws keep the layouts and meaning of the
+ * ragged call; shape.seq_kv is the largest length a table can describe
+ * (nb * 128 or less).  Several tables may share pages (a common prefix): the
+ * caches are only read.  Rows of a page past a sequence's length may hold any
+ * bits.  A page id outside [0, num_pages) is clamped into it (that block's
+ * result is then wrong) and sets bit 2 of the device error word.
+ * Errors: num_pages < 1 -> MSA_ERR_INVALID_SHAPE; num_pages * G or
+ * num_pages * 128 >= 2^31 -> MSA_ERR_UNSUPPORTED; NULL page_table ->
+ * MSA_ERR_NULL_PTR. */
+msa_status msa_forward_decode_paged(const msa_shape* shape, int num_pages,
+                                    const int32_t* seq_lens, const int32_t* page_table,
+                                    const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                                    const uint16_t* q_idx, const uint16_t* k_idx, uint16_t* o,
+                                    float* lse, int32_t* sel_out, void* ws, size_t ws_bytes,
+                                    void* stream);
+
 /* Dense causal GQA attention (every key x <= p_t), the baseline the pages
  * compare MSA against ([P1] GQA definition; [P2], [P4] speed-ups vs GQA).
  * Prefill: q-outer flash attention, no workspace needed (pass NULL/0). */
@@ -235,9 +260,9 @@ msa_status msa_sparse_attn_decode_static(const msa_shape* shape, const uint16_t*
 
 /* Reads and clears the device error word of the current device (bit 0: a
  * bounded wait timed out; bit 1: a ragged-decode cache length was out of
- * range).  Synchronises the current device.  Returns
- * MSA_ERR_DEVICE_TIMEOUT if any bit was set, MSA_OK otherwise; *flags (may be
- * NULL) receives the raw word. */
+ * range; bit 2: a page-table entry was out of range).  Synchronises the
+ * current device.  Returns MSA_ERR_DEVICE_TIMEOUT if any bit was set, MSA_OK
+ * otherwise; *flags (may be NULL) receives the raw word. */
 msa_status msa_device_status(uint32_t* flags);
 
 /* Per-kernel timing with CUDA events (diagnostics; no counterpart on the

@@ -94,6 +94,23 @@ def test_pointer_checks_precede_device_use(L):
                                    ctypes.c_void_p((1 << 20) + 2), ok, 1 << 40, None) == 3
     assert L.msa_forward_alignment(ctypes.byref(s), ok, ok, ok, ok, ok, ok, None, None, ok,
                                    ok, 16, None) == 4
+    # paged decode: pool size, table pointer, then the ragged call's checks
+    d1 = tiny(seq_q=1, seq_kv=4096, q_offset=0)
+    paged = L.msa_forward_decode_paged
+    assert paged(ctypes.byref(d1), 0, ok, ok, ok, ok, ok, ok, ok, ok, None, None, ok, 1 << 40,
+                 None) == 1
+    assert paged(ctypes.byref(d1), 1 << 30, ok, ok, ok, ok, ok, ok, ok, ok, None, None, ok,
+                 1 << 40, None) == 5
+    assert paged(ctypes.byref(d1), 8, ok, None, ok, ok, ok, ok, ok, ok, None, None, ok, 1 << 40,
+                 None) == 2
+    assert paged(ctypes.byref(d1), 8, ok, ctypes.c_void_p((1 << 20) + 2), ok, ok, ok, ok, ok, ok,
+                 None, None, ok, 1 << 40, None) == 3
+    assert paged(ctypes.byref(d1), 8, None, ok, ok, ok, ok, ok, ok, ok, None, None, ok, 1 << 40,
+                 None) == 2
+    assert paged(ctypes.byref(d1), 8, ok, ok, ok, ok, ok, ok, ok, ok, None, None, ok, 16,
+                 None) == 4
+    assert paged(ctypes.byref(tiny()), 8, ok, ok, ok, ok, ok, ok, ok, ok, None, None, ok, 1 << 40,
+                 None) == 1                                # T must be 1
     dec = tiny(seq_q=1, seq_kv=4096, q_offset=4095)
     assert L.msa_sparse_attn_decode(ctypes.byref(dec), ok, ok, ok, ok, ok, None, ok, 8, None) == 4
     assert L.msa_dense_attn_decode(ctypes.byref(s), ok, ok, ok, ok, None, ok, 1 << 30, None) == 1
