@@ -308,6 +308,13 @@ def run_msa(args, world, rank, pg):
                        "peak_source": f"{peak_src} ({'sustained' if bound == 'tensor' else 'copy'})",
                        "traffic": ncu_traffic(dom),
                        "algorithmic_per_launch": amount}
+    traffic = out["roofline"]["traffic"]
+    if traffic:
+        # the same launch against the time its measured DRAM bytes take at the
+        # copy bandwidth (the KV-outer schedule's gather and partial traffic)
+        floor_ms = traffic / (peaks["hbm_gbs"] * 1e9) * 1e3
+        out["roofline"]["traffic_floor"] = {"ms": round(floor_ms, 3),
+                                            "frac": round(floor_ms / kernels[dom], 4)}
     # every stage against its own roof
     stages = {}
     for name, (bnd, amt) in work.items():
