@@ -93,9 +93,13 @@ size_t carve_bytes(const msa_shape& s) {
 // ------------------------------------------------------- 1. invert selection
 // grid: (ceil(T / kHistTokens), B*G).  Pass 0 counts (sequence, group, block)
 // hits; pass 1 reserves a range per column and scatters (token, slot) entries.
+// Only entries 0 <= block <= b_t take part (negative ones are empty slots);
+// one past the query's block is ignored, and pass 0 flags it in the error
+// word, so a bad caller selection can never index past the histogram.
 __global__ void __launch_bounds__(256) sel_invert_kernel(const int32_t* __restrict__ sel,
                                                          PrefillWs w, int T, int G, int k,
-                                                         int nb, int pass) {
+                                                         int nb, int q_off, int pass,
+                                                         uint32_t* err) {
   extern __shared__ uint32_t hist[];   // [nb] counts, then [nb] cursors/bases
   uint32_t* base = hist + nb;
   const int bg = blockIdx.y;
@@ -107,7 +111,10 @@ __global__ void __launch_bounds__(256) sel_invert_kernel(const int32_t* __restri
   for (int x = threadIdx.x; x < (t1 - t0) * k; x += blockDim.x) {
     const int t = t0 + x / k, slot = x % k;
     const int c = sel[((static_cast<long long>(b) * T + t) * G + g) * k + slot];
-    if (c >= 0) atomicAdd(&hist[c], 1u);
+    if (c >= 0 && c <= (q_off + t) >> 7)
+      atomicAdd(&hist[c], 1u);
+    else if (c >= 0 && pass == 0)
+      atomicOr(err, kErrBadSel);
   }
   __syncthreads();
   const long long col0 = static_cast<long long>(bg) * nb;
@@ -124,7 +131,7 @@ __global__ void __launch_bounds__(256) sel_invert_kernel(const int32_t* __restri
   for (int x = threadIdx.x; x < (t1 - t0) * k; x += blockDim.x) {
     const int t = t0 + x / k, slot = x % k;
     const int c = sel[((static_cast<long long>(b) * T + t) * G + g) * k + slot];
-    if (c >= 0) {
+    if (c >= 0 && c <= (q_off + t) >> 7) {
       const uint32_t pos = base[c] + atomicAdd(&hist[c], 1u);
       w.entries[pos] = (static_cast<uint32_t>(t) << 6) | static_cast<uint32_t>(slot);
       w.inv[((static_cast<long long>(b) * T + t) * G + g) * k + slot] = pos;
@@ -789,7 +796,7 @@ template <int D, bool KL>
 __global__ void __launch_bounds__(256, 8) combine_kernel(const int32_t* __restrict__ sel,
                                                       const PrefillWs w, uint16_t* __restrict__ o,
                                                       float* __restrict__ lse, int H, int G,
-                                                      int r, int k,
+                                                      int r, int k, int T, int q_off,
                                                       const float* __restrict__ pooled,
                                                       float* __restrict__ kl, int nb) {
   constexpr int CH = D / 8;                  // 16-byte chunks per head row
@@ -801,10 +808,12 @@ __global__ void __launch_bounds__(256, 8) combine_kernel(const int32_t* __restri
   const float2* ml_all = reinterpret_cast<const float2*>(w.part_ml);
   const int32_t* srow = sel + bt * G * k;
   const uint32_t* irow = w.inv + bt * G * k;
+  const int lb = (q_off + static_cast<int>(bt % T)) >> 7;   // the query's block
   for (int x = threadIdx.x; x < G * k; x += blockDim.x) {
     const int j = srow[x];
-    sm_pos[x] = j >= 0 ? irow[x] : 0xFFFFFFFFu;
-    if constexpr (KL) sm_z[x] = j >= 0 ? pooled[(bt * G + x / k) * nb + j] : -INFINITY;
+    const bool used = j >= 0 && j <= lb;     // the slots the inversion kept
+    sm_pos[x] = used ? irow[x] : 0xFFFFFFFFu;
+    if constexpr (KL) sm_z[x] = used ? pooled[(bt * G + x / k) * nb + j] : -INFINITY;
   }
   __syncthreads();
   for (int x = threadIdx.x; x < k * H; x += blockDim.x) {
@@ -839,7 +848,7 @@ __global__ void __launch_bounds__(256, 8) combine_kernel(const int32_t* __restri
         acc[2 * e + 1] += ws * f.y;
       }
     }
-    const float inv = 1.f / den;
+    const float inv = den > 0.f ? 1.f / den : 0.f;   // no block at all: o = 0, lse = -inf
     uint32_t out[4];
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
@@ -958,7 +967,8 @@ cudaError_t launch_sparse_prefill(const msa_shape& s, const uint16_t* q, const u
   if (e != cudaSuccess) return e;
   {
     ProfScope ps_("sel_count", st);
-    sel_invert_kernel<<<hgrid, 256, hsmem, st>>>(sel, w, s.seq_q, s.n_kv_heads, s.topk, nb, 0);
+    sel_invert_kernel<<<hgrid, 256, hsmem, st>>>(sel, w, s.seq_q, s.n_kv_heads, s.topk, nb,
+                                                 s.q_offset, 0, ctx->err);
   }
   {
     ProfScope ps_("scan_columns", st);
@@ -966,7 +976,8 @@ cudaError_t launch_sparse_prefill(const msa_shape& s, const uint16_t* q, const u
   }
   {
     ProfScope ps_("sel_scatter", st);
-    sel_invert_kernel<<<hgrid, 256, hsmem, st>>>(sel, w, s.seq_q, s.n_kv_heads, s.topk, nb, 1);
+    sel_invert_kernel<<<hgrid, 256, hsmem, st>>>(sel, w, s.seq_q, s.n_kv_heads, s.topk, nb,
+                                                 s.q_offset, 1, ctx->err);
   }
   {
     ProfScope ps_("make_tiles", st);
@@ -998,19 +1009,19 @@ cudaError_t launch_sparse_prefill(const msa_shape& s, const uint16_t* q, const u
                        4u * s.n_kv_heads * s.topk;
   {
     ProfScope ps_(with_kl ? "combine_kl" : "combine", st);
-    const int H = s.n_q_heads, G = s.n_kv_heads, kk = s.topk;
+    const int H = s.n_q_heads, G = s.n_kv_heads, kk = s.topk, T = s.seq_q, qo = s.q_offset;
     if (s.head_dim == 128 && with_kl)
-      combine_kernel<128, true><<<ntok, 256, csmem, st>>>(sel, w, o, lse, H, G, r, kk, pooled, kl,
-                                                          nb);
+      combine_kernel<128, true><<<ntok, 256, csmem, st>>>(sel, w, o, lse, H, G, r, kk, T, qo,
+                                                          pooled, kl, nb);
     else if (s.head_dim == 128)
-      combine_kernel<128, false><<<ntok, 256, csmem, st>>>(sel, w, o, lse, H, G, r, kk, nullptr,
-                                                           nullptr, nb);
+      combine_kernel<128, false><<<ntok, 256, csmem, st>>>(sel, w, o, lse, H, G, r, kk, T, qo,
+                                                           nullptr, nullptr, nb);
     else if (with_kl)
-      combine_kernel<64, true><<<ntok, 256, csmem, st>>>(sel, w, o, lse, H, G, r, kk, pooled, kl,
-                                                         nb);
+      combine_kernel<64, true><<<ntok, 256, csmem, st>>>(sel, w, o, lse, H, G, r, kk, T, qo,
+                                                         pooled, kl, nb);
     else
-      combine_kernel<64, false><<<ntok, 256, csmem, st>>>(sel, w, o, lse, H, G, r, kk, nullptr,
-                                                          nullptr, nb);
+      combine_kernel<64, false><<<ntok, 256, csmem, st>>>(sel, w, o, lse, H, G, r, kk, T, qo,
+                                                          nullptr, nullptr, nb);
   }
   return cudaGetLastError();
 }

@@ -16,6 +16,7 @@ namespace msa {
 constexpr uint32_t kErrTimeout = 1u;
 constexpr uint32_t kErrBadLength = 2u;   // a ragged-decode cache length outside [1, N]
 constexpr uint32_t kErrBadPage = 4u;     // a page-table entry outside [0, num_pages)
+constexpr uint32_t kErrBadSel = 8u;      // a prefill selection entry past its query's block
 // Bound of every mbarrier wait, in nanoseconds of %globaltimer.
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 

@@ -307,8 +307,8 @@ def profile_read() -> dict:
 
 def device_status() -> int:
     """Raw device error word (bit 0: a bounded wait expired; bit 1: a ragged-decode
-    cache length was out of range; bit 2: a page-table entry was out of range);
-    clears it."""
+    cache length was out of range; bit 2: a page-table entry was out of range;
+    bit 3: a prefill selection entry lay past its query's block); clears it."""
     f = ctypes.c_uint32(0)
     st = lib().msa_device_status(ctypes.byref(f))
     if st not in (0, 7):

@@ -127,7 +127,11 @@ msa_status msa_block_topk(const msa_shape* shape, const float* pooled, int32_t* 
  * attention), [P5]:  for head h of group g = floor(h/r),
  *   o[b,t,h,:] = sum_x softmax_x(q[b,t,h,:] . k[b,g,x,:] / sqrt(d)) v[b,g,x,:]
  * over keys x in the blocks listed in sel[b,t,g,:] (entries -1 ignored) with
- * x <= p_t.  Blocks listed must satisfy 0 <= block <= b_t.  lse may be NULL.
+ * x <= p_t.  Entries must lie in 0 .. b_t: negative ones are empty slots,
+ * larger ones are ignored and set bit 3 of the device error word.  Each block
+ * should be listed once (a repeated block is weighted twice, as in the
+ * formula taken literally).  A row with no block gets o = 0, lse = -inf.
+ * lse may be NULL.
  * ws/ws_bytes: workspace of at least msa_workspace_size(MSA_OP_SPARSE_PREFILL).
  * KV-outer schedule ([P4]): each selected 128-row K/V block of a group is
  * loaded once and reused by every (token, head) row that selected it. */
@@ -140,6 +144,8 @@ msa_status msa_sparse_attn_prefill(const msa_shape* shape, const uint16_t* q,
  * token is already the last cache row).  A persistent grid streams the
  * selected blocks of every (sequence, group) through a TMA pipeline; a group
  * whose blocks fall to several CTAs is merged in-kernel by the last of them.
+ * Entries outside 0 .. b_t are ignored; a (sequence, group) with no block
+ * left gets o = 0, lse = -inf.
  * ws >= msa_workspace_size(MSA_OP_SPARSE_DECODE). */
 msa_status msa_sparse_attn_decode(const msa_shape* shape, const uint16_t* q,
                                   const uint16_t* k, const uint16_t* v,
@@ -260,8 +266,9 @@ msa_status msa_sparse_attn_decode_static(const msa_shape* shape, const uint16_t*
 
 /* Reads and clears the device error word of the current device (bit 0: a
  * bounded wait timed out; bit 1: a ragged-decode cache length was out of
- * range; bit 2: a page-table entry was out of range).  Synchronises the
- * current device.  Returns MSA_ERR_DEVICE_TIMEOUT if any bit was set, MSA_OK
+ * range; bit 2: a page-table entry was out of range; bit 3: a prefill
+ * selection entry lay past its query's block).  Synchronises the current
+ * device.  Returns MSA_ERR_DEVICE_TIMEOUT if any bit was set, MSA_OK
  * otherwise; *flags (may be NULL) receives the raw word. */
 msa_status msa_device_status(uint32_t* flags);
 

@@ -158,6 +158,34 @@ def test_sparse_prefill_spans_token_chunks():
     assert np.abs(lse[0].double().cpu().numpy() - L_ref).max() < LSE_ABS
 
 
+def test_sparse_prefill_ignores_and_flags_bad_selection():
+    """Caller selections with a block past the pool, a block past the query's
+    own, and a row with no block at all: the bad entries are dropped (bit 3 of
+    the device error word), the rest is the oracle on what remains, and the
+    empty row gives o = 0, lse = -inf."""
+    sp = spec(1, 300, 1000, 700, 16, 4, 64, 64, 5, seed=59)
+    inp = inputs_cpu(sp)
+    sel_ok = oracle_sel(sp, oracle_pooled(sp, inp, 0))
+    bad = sel_ok.copy()
+    bt = positions(sp) // sp.block
+    bad[0, 0, -1] = sp.nb + 7                 # past every block of the cache
+    bad[1, 1, -1] = bt[1] + 1                 # the block after the query's
+    bad[2] = -1                               # nothing selected
+    o, lse = M.sparse_attn_prefill(M.Shape.of(sp), cuda(inp.q), cuda(inp.k), cuda(inp.v),
+                                   cuda(torch.from_numpy(bad)[None]))
+    flags = M.device_status()
+    assert flags & 8, flags
+    keep = bad.copy()
+    keep[0, 0, -1] = keep[1, 1, -1] = -1
+    keep[2] = sel_ok[2]                       # any selection: row 2 is checked separately
+    O_ref, L_ref = oracle_attention(sp, inp, keep, 0)
+    rows = np.array([t for t in range(sp.seq_q) if t != 2])
+    check_attn(o[0, torch.as_tensor(rows, device=o.device)], O_ref[rows], "bad selection")
+    got_l = lse[0].double().cpu().numpy()
+    assert np.abs(got_l[rows] - L_ref[rows]).max() < LSE_ABS
+    assert torch.count_nonzero(o[0, 2]).item() == 0 and np.all(np.isneginf(got_l[2]))
+
+
 @pytest.mark.parametrize("sp", [spec(3, 1, 3000, 2999, 16, 2, 128, 64, 4, seed=21),
                                 spec(2, 1, 5000, 4999, 8, 2, 64, 32, 16, seed=22),
                                 spec(2, 1, 129, 128, 16, 1, 128, 64, 16, seed=23),
