@@ -116,6 +116,41 @@ def _ptr(t):
     return ctypes.c_void_p(t.data_ptr())
 
 
+def _sizes(shape: Shape, pages: int = 0) -> dict:
+    """dtype and element count of every array argument, from the C-ABI layouts."""
+    B, T, N, H, G = shape.batch, shape.seq_q, shape.seq_kv, shape.n_q_heads, shape.n_kv_heads
+    d, di, k, nb = shape.head_dim, shape.index_dim, shape.topk, shape.nb
+    bf16, f32, i32 = torch.bfloat16, torch.float32, torch.int32
+    return {"q": (bf16, B * T * H * d), "o": (bf16, B * T * H * d),
+            "k": (bf16, B * G * N * d), "v": (bf16, B * G * N * d),
+            "q_idx": (bf16, B * T * G * di), "k_idx": (bf16, B * N * di),
+            "pooled": (f32, B * T * G * nb), "sel": (i32, B * T * G * k),
+            "lse": (f32, B * T * H), "kl": (f32, B * T * G), "seq_lens": (i32, B),
+            "page_table": (i32, B * nb), "k_pages": (bf16, pages * G * 128 * d),
+            "v_pages": (bf16, pages * G * 128 * d), "kidx_pages": (bf16, pages * 128 * di)}
+
+
+def _args(shape: Shape, pages: int = 0, **tensors) -> dict:
+    """Device pointers of the named tensors after checking each one's dtype and
+    that it holds at least the elements its layout needs (None stays None)."""
+    need = _sizes(shape, pages)
+    out = {}
+    for name, t in tensors.items():
+        if t is not None:
+            dtype, n = need[name]
+            if t.dtype != dtype:
+                raise ValueError(f"{name}: expected {dtype}, got {t.dtype}")
+            if t.numel() < n:
+                raise ValueError(f"{name}: {t.numel()} elements, the shape needs {n}")
+        out[name] = _ptr(t)
+    return out
+
+
+def _ws(ws):
+    """(pointer, size in bytes) of a workspace tensor."""
+    return _ptr(ws), ws.numel() * ws.element_size()
+
+
 def _stream(stream):
     s = torch.cuda.current_stream() if stream is None else stream
     return ctypes.c_void_p(s.cuda_stream)
@@ -141,7 +176,8 @@ def index_scores(shape: Shape, q_idx, k_idx, pooled=None, stream=None):
     if pooled is None:
         pooled = torch.empty((shape.batch, shape.seq_q, shape.n_kv_heads, shape.nb),
                              dtype=torch.float32, device=q_idx.device)
-    _check(lib().msa_index_scores(ctypes.byref(shape), _ptr(q_idx), _ptr(k_idx), _ptr(pooled),
+    a = _args(shape, q_idx=q_idx, k_idx=k_idx, pooled=pooled)
+    _check(lib().msa_index_scores(ctypes.byref(shape), a["q_idx"], a["k_idx"], a["pooled"],
                                   _stream(stream)), "msa_index_scores")
     return pooled
 
@@ -150,7 +186,8 @@ def block_topk(shape: Shape, pooled, sel=None, stream=None):
     if sel is None:
         sel = torch.empty((shape.batch, shape.seq_q, shape.n_kv_heads, shape.topk),
                           dtype=torch.int32, device=pooled.device)
-    _check(lib().msa_block_topk(ctypes.byref(shape), _ptr(pooled), _ptr(sel), _stream(stream)),
+    a = _args(shape, pooled=pooled, sel=sel)
+    _check(lib().msa_block_topk(ctypes.byref(shape), a["pooled"], a["sel"], _stream(stream)),
            "msa_block_topk")
     return sel
 
@@ -168,8 +205,9 @@ def sparse_attn_prefill(shape: Shape, q, k, v, sel, o=None, lse=None, ws=None, w
                         stream=None):
     o, lse = _attn_out(shape, q, o, lse, want_lse)
     ws = alloc_workspace(shape, OP_SPARSE_PREFILL, q.device) if ws is None else ws
-    _check(lib().msa_sparse_attn_prefill(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(sel),
-                                         _ptr(o), _ptr(lse), _ptr(ws), ws.numel(), _stream(stream)),
+    a = _args(shape, q=q, k=k, v=v, sel=sel, o=o, lse=lse)
+    _check(lib().msa_sparse_attn_prefill(ctypes.byref(shape), a["q"], a["k"], a["v"], a["sel"],
+                                         a["o"], a["lse"], *_ws(ws), _stream(stream)),
            "msa_sparse_attn_prefill")
     return o, lse
 
@@ -178,8 +216,9 @@ def sparse_attn_decode(shape: Shape, q, k, v, sel, o=None, lse=None, ws=None, wa
                        stream=None):
     o, lse = _attn_out(shape, q, o, lse, want_lse)
     ws = alloc_workspace(shape, OP_SPARSE_DECODE, q.device) if ws is None else ws
-    _check(lib().msa_sparse_attn_decode(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(sel),
-                                        _ptr(o), _ptr(lse), _ptr(ws), ws.numel(), _stream(stream)),
+    a = _args(shape, q=q, k=k, v=v, sel=sel, o=o, lse=lse)
+    _check(lib().msa_sparse_attn_decode(ctypes.byref(shape), a["q"], a["k"], a["v"], a["sel"],
+                                        a["o"], a["lse"], *_ws(ws), _stream(stream)),
            "msa_sparse_attn_decode")
     return o, lse
 
@@ -190,8 +229,9 @@ def sparse_attn_decode_static(shape: Shape, q, k, v, sel, o=None, lse=None, want
     library's static device array, so nothing is allocated for it.  Calls
     that may overlap on the GPU share that array and must be serialised."""
     o, lse = _attn_out(shape, q, o, lse, want_lse)
-    _check(lib().msa_sparse_attn_decode_static(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v),
-                                               _ptr(sel), _ptr(o), _ptr(lse), _stream(stream)),
+    a = _args(shape, q=q, k=k, v=v, sel=sel, o=o, lse=lse)
+    _check(lib().msa_sparse_attn_decode_static(ctypes.byref(shape), a["q"], a["k"], a["v"],
+                                               a["sel"], a["o"], a["lse"], _stream(stream)),
            "msa_sparse_attn_decode_static")
     return o, lse
 
@@ -203,9 +243,10 @@ def forward(shape: Shape, q, k, v, q_idx, k_idx, o=None, lse=None, sel=None, ws=
         sel = torch.empty((shape.batch, shape.seq_q, shape.n_kv_heads, shape.topk),
                           dtype=torch.int32, device=q.device)
     ws = alloc_workspace(shape, OP_FORWARD, q.device) if ws is None else ws
-    _check(lib().msa_forward(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(q_idx),
-                             _ptr(k_idx), _ptr(o), _ptr(lse), _ptr(sel), _ptr(ws), ws.numel(),
-                             _stream(stream)), "msa_forward")
+    a = _args(shape, q=q, k=k, v=v, q_idx=q_idx, k_idx=k_idx, o=o, lse=lse, sel=sel)
+    _check(lib().msa_forward(ctypes.byref(shape), a["q"], a["k"], a["v"], a["q_idx"], a["k_idx"],
+                             a["o"], a["lse"], a["sel"], *_ws(ws), _stream(stream)),
+           "msa_forward")
     return o, lse, sel
 
 
@@ -222,9 +263,10 @@ def forward_alignment(shape: Shape, q, k, v, q_idx, k_idx, o=None, lse=None, sel
         kl = torch.empty((shape.batch, shape.seq_q, shape.n_kv_heads), dtype=torch.float32,
                          device=q.device)
     ws = alloc_workspace(shape, OP_FORWARD_ALIGNMENT, q.device) if ws is None else ws
-    _check(lib().msa_forward_alignment(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v),
-                                       _ptr(q_idx), _ptr(k_idx), _ptr(o), _ptr(lse), _ptr(sel),
-                                       _ptr(kl), _ptr(ws), ws.numel(), _stream(stream)),
+    a = _args(shape, q=q, k=k, v=v, q_idx=q_idx, k_idx=k_idx, o=o, lse=lse, sel=sel, kl=kl)
+    _check(lib().msa_forward_alignment(ctypes.byref(shape), a["q"], a["k"], a["v"], a["q_idx"],
+                                       a["k_idx"], a["o"], a["lse"], a["sel"], a["kl"],
+                                       *_ws(ws), _stream(stream)),
            "msa_forward_alignment")
     return o, lse, sel, kl
 
@@ -239,9 +281,11 @@ def forward_decode_ragged(shape: Shape, q, k, v, q_idx, k_idx, seq_lens, o=None,
         sel = torch.empty((shape.batch, 1, shape.n_kv_heads, shape.topk), dtype=torch.int32,
                           device=q.device)
     ws = alloc_workspace(shape, OP_FORWARD, q.device) if ws is None else ws
-    _check(lib().msa_forward_decode_ragged(ctypes.byref(shape), _ptr(seq_lens), _ptr(q), _ptr(k),
-                                           _ptr(v), _ptr(q_idx), _ptr(k_idx), _ptr(o), _ptr(lse),
-                                           _ptr(sel), _ptr(ws), ws.numel(), _stream(stream)),
+    a = _args(shape, seq_lens=seq_lens, q=q, k=k, v=v, q_idx=q_idx, k_idx=k_idx, o=o, lse=lse,
+              sel=sel)
+    _check(lib().msa_forward_decode_ragged(ctypes.byref(shape), a["seq_lens"], a["q"], a["k"],
+                                           a["v"], a["q_idx"], a["k_idx"], a["o"], a["lse"],
+                                           a["sel"], *_ws(ws), _stream(stream)),
            "msa_forward_decode_ragged")
     return o, lse, sel
 
@@ -257,19 +301,22 @@ def forward_decode_paged(shape: Shape, q, k_pages, v_pages, q_idx, kidx_pages, s
         sel = torch.empty((shape.batch, 1, shape.n_kv_heads, shape.topk), dtype=torch.int32,
                           device=q.device)
     ws = alloc_workspace(shape, OP_FORWARD, q.device) if ws is None else ws
-    _check(lib().msa_forward_decode_paged(ctypes.byref(shape), int(k_pages.shape[0]),
-                                          _ptr(seq_lens), _ptr(page_table), _ptr(q),
-                                          _ptr(k_pages), _ptr(v_pages), _ptr(q_idx),
-                                          _ptr(kidx_pages), _ptr(o), _ptr(lse), _ptr(sel),
-                                          _ptr(ws), ws.numel(), _stream(stream)),
+    P = int(k_pages.shape[0])
+    a = _args(shape, P, seq_lens=seq_lens, page_table=page_table, q=q, k_pages=k_pages,
+              v_pages=v_pages, q_idx=q_idx, kidx_pages=kidx_pages, o=o, lse=lse, sel=sel)
+    _check(lib().msa_forward_decode_paged(ctypes.byref(shape), P, a["seq_lens"], a["page_table"],
+                                          a["q"], a["k_pages"], a["v_pages"], a["q_idx"],
+                                          a["kidx_pages"], a["o"], a["lse"], a["sel"],
+                                          *_ws(ws), _stream(stream)),
            "msa_forward_decode_paged")
     return o, lse, sel
 
 
 def dense_attn_prefill(shape: Shape, q, k, v, o=None, lse=None, want_lse=True, stream=None):
     o, lse = _attn_out(shape, q, o, lse, want_lse)
-    _check(lib().msa_dense_attn_prefill(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(o),
-                                        _ptr(lse), None, 0, _stream(stream)),
+    a = _args(shape, q=q, k=k, v=v, o=o, lse=lse)
+    _check(lib().msa_dense_attn_prefill(ctypes.byref(shape), a["q"], a["k"], a["v"], a["o"],
+                                        a["lse"], None, 0, _stream(stream)),
            "msa_dense_attn_prefill")
     return o, lse
 
@@ -278,8 +325,9 @@ def dense_attn_decode(shape: Shape, q, k, v, o=None, lse=None, ws=None, want_lse
                       stream=None):
     o, lse = _attn_out(shape, q, o, lse, want_lse)
     ws = alloc_workspace(shape, OP_DENSE_DECODE, q.device) if ws is None else ws
-    _check(lib().msa_dense_attn_decode(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(o),
-                                       _ptr(lse), _ptr(ws), ws.numel(), _stream(stream)),
+    a = _args(shape, q=q, k=k, v=v, o=o, lse=lse)
+    _check(lib().msa_dense_attn_decode(ctypes.byref(shape), a["q"], a["k"], a["v"], a["o"],
+                                       a["lse"], *_ws(ws), _stream(stream)),
            "msa_dense_attn_decode")
     return o, lse
 
