@@ -224,6 +224,7 @@ msa_status msa_workspace_size(const msa_shape* s, msa_op op, size_t* bytes) {
       return check_shape(s, false, false);
     case MSA_OP_SPARSE_PREFILL:
       if ((st = check_shape(s, true, false)) != MSA_OK) return st;
+      if (!prefill_shape_supported(*s)) return MSA_ERR_UNSUPPORTED;
       *bytes = prefill_workspace_bytes(*s);
       return MSA_OK;
     case MSA_OP_SPARSE_DECODE:
@@ -234,6 +235,7 @@ msa_status msa_workspace_size(const msa_shape* s, msa_op op, size_t* bytes) {
       return MSA_OK;
     case MSA_OP_FORWARD:
       if ((st = check_shape(s, true, true)) != MSA_OK) return st;
+      if (!forward_is_decode(*s) && !prefill_shape_supported(*s)) return MSA_ERR_UNSUPPORTED;
       *bytes = pooled_bytes(*s) + sel_bytes(*s) +
                (forward_is_decode(*s) ? decode_workspace_bytes(*s, false)
                                       : prefill_workspace_bytes(*s));
@@ -242,6 +244,7 @@ msa_status msa_workspace_size(const msa_shape* s, msa_op op, size_t* bytes) {
       return check_shape(s, true, false);
     case MSA_OP_FORWARD_ALIGNMENT:
       if ((st = check_shape(s, true, true)) != MSA_OK) return st;
+      if (!prefill_shape_supported(*s)) return MSA_ERR_UNSUPPORTED;
       *bytes = pooled_bytes(*s) + sel_bytes(*s) + prefill_workspace_bytes(*s);
       return MSA_OK;
   }
@@ -283,6 +286,7 @@ msa_status msa_sparse_attn_prefill(const msa_shape* s, const uint16_t* q, const 
                                    float* lse, void* ws, size_t ws_bytes, void* stream) {
   msa_status st = check_shape(s, true, false);
   if (st != MSA_OK) return st;
+  if (!prefill_shape_supported(*s)) return MSA_ERR_UNSUPPORTED;
   if ((st = check_attn_ptrs(q, k, v, sel, true, o, lse)) != MSA_OK) return st;
   const size_t need = prefill_workspace_bytes(*s);
   if (need && !ws) return MSA_ERR_NULL_PTR;

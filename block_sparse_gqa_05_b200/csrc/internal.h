@@ -59,6 +59,11 @@ cudaError_t launch_index_scores(const msa_shape& s, const uint16_t* q_idx,
 cudaError_t launch_block_topk(const msa_shape& s, const float* pooled, int32_t* sel,
                               cudaStream_t st, const int32_t* lens = nullptr);
 size_t prefill_workspace_bytes(const msa_shape& s);
+// Shared-memory limits of the prefill path's per-CTA tables: the inversion's
+// [2 nb] histogram and the combine's [k][H] (max, sum) pairs plus its [G][k]
+// entry map (and, with the alignment output, [H] head sums and [G][k] pooled
+// scores).  False when a shape needs more than one CTA can hold.
+bool prefill_shape_supported(const msa_shape& s);
 cudaError_t launch_sparse_prefill(const msa_shape& s, const uint16_t* q, const uint16_t* k,
                                   const uint16_t* v, const int32_t* sel, uint16_t* o,
                                   float* lse, void* ws, cudaStream_t st,

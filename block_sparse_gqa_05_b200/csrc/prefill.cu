@@ -945,6 +945,20 @@ cudaError_t launch_attn(const msa_shape& s, const uint16_t* q, const uint16_t* k
 
 size_t prefill_workspace_bytes(const msa_shape& s) { return carve_bytes(s); }
 
+constexpr size_t kHistSmemMax = 200u * 1024u;
+constexpr size_t kCombineSmemMax = 227u * 1024u;    // the opt-in maximum per CTA
+constexpr size_t kDefaultSmem = 48u * 1024u;
+
+static size_t combine_smem_bytes(const msa_shape& s, bool with_kl) {
+  const size_t H = s.n_q_heads, G = s.n_kv_heads, k = s.topk;
+  return 8 * k * H + (with_kl ? 8 * H + 4 * G * k : 0) + 4 * G * k;
+}
+
+bool prefill_shape_supported(const msa_shape& s) {
+  const size_t nb = static_cast<size_t>(ceil_div(s.seq_kv, 128));
+  return 8 * nb <= kHistSmemMax && combine_smem_bytes(s, true) <= kCombineSmemMax;
+}
+
 cudaError_t launch_sparse_prefill(const msa_shape& s, const uint16_t* q, const uint16_t* k,
                                   const uint16_t* v, const int32_t* sel, uint16_t* o,
                                   float* lse, void* ws, cudaStream_t st, const float* pooled,
@@ -961,7 +975,7 @@ cudaError_t launch_sparse_prefill(const msa_shape& s, const uint16_t* q, const u
   const dim3 hgrid(static_cast<unsigned>(ceil_div(s.seq_q, kHistTokens)),
                    static_cast<unsigned>(s.batch * s.n_kv_heads));
   const size_t hsmem = 8ull * nb;
-  if (hsmem > 200 * 1024) return cudaErrorInvalidValue;
+  if (!prefill_shape_supported(s)) return cudaErrorInvalidValue;
   e = cudaFuncSetAttribute(sel_invert_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(hsmem));
   if (e != cudaSuccess) return e;
@@ -1004,9 +1018,18 @@ cudaError_t launch_sparse_prefill(const msa_shape& s, const uint16_t* q, const u
   if (e != cudaSuccess) return e;
   const unsigned ntok = static_cast<unsigned>(static_cast<long long>(s.batch) * s.seq_q);
   const bool with_kl = kl != nullptr;
-  const size_t csmem = sizeof(float2) * s.topk * s.n_q_heads +
-                       (with_kl ? sizeof(float2) * s.n_q_heads + 4u * s.n_kv_heads * s.topk : 0) +
-                       4u * s.n_kv_heads * s.topk;
+  const size_t csmem = combine_smem_bytes(s, with_kl);
+  if (csmem > kDefaultSmem) {
+    // many heads x many slots: opt in to more than the default 48 KB
+    const void* fn = s.head_dim == 128
+                         ? (with_kl ? reinterpret_cast<const void*>(combine_kernel<128, true>)
+                                    : reinterpret_cast<const void*>(combine_kernel<128, false>))
+                         : (with_kl ? reinterpret_cast<const void*>(combine_kernel<64, true>)
+                                    : reinterpret_cast<const void*>(combine_kernel<64, false>));
+    e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(csmem));
+    if (e != cudaSuccess) return e;
+  }
   {
     ProfScope ps_(with_kl ? "combine_kl" : "combine", st);
     const int H = s.n_q_heads, G = s.n_kv_heads, kk = s.topk, T = s.seq_q, qo = s.q_offset;

@@ -65,6 +65,19 @@ def test_workspace_sizes_and_validation():
     assert ws(tiny(), M.OP_SPARSE_DECODE)[0] == 1
 
 
+def test_prefill_shared_memory_limits():
+    # the combine keeps k x H (max, sum) pairs of a token on chip, the
+    # inversion a 2 x nb histogram: shapes past one CTA's shared memory are
+    # refused up front (decode, which uses neither, is not limited)
+    many = dict(seq_q=256, seq_kv=4096, q_offset=3840, n_q_heads=1024, n_kv_heads=64, topk=64)
+    for op in (M.OP_SPARSE_PREFILL, M.OP_FORWARD, M.OP_FORWARD_ALIGNMENT):
+        assert ws(tiny(**many), op)[0] == 5
+    assert ws(tiny(**dict(many, n_q_heads=256, n_kv_heads=16)), M.OP_FORWARD)[0] == 0
+    n = 26000 * 128
+    assert ws(tiny(seq_q=256, seq_kv=n, q_offset=n - 256), M.OP_FORWARD)[0] == 5
+    assert ws(tiny(seq_q=1, seq_kv=n, q_offset=n - 1), M.OP_FORWARD)[0] == 0
+
+
 @pytest.mark.parametrize("bad,code", [
     (dict(block=64), 5), (dict(topk=0), 1), (dict(topk=65), 5), (dict(head_dim=96), 5),
     (dict(index_dim=48), 5), (dict(n_q_heads=7), 1), (dict(n_q_heads=6), 5), (dict(n_kv_heads=3, n_q_heads=6), 5),
