@@ -1,6 +1,7 @@
 """C-ABI checks that need no GPU: the library loads, exports every symbol the
 header declares, and rejects bad arguments before touching the device."""
 import ctypes
+import os
 
 import pytest
 
@@ -136,3 +137,22 @@ def test_binding_rejects_cpu_tensors():
         M.index_scores(s, torch.zeros(1, 2048, 2, 32, dtype=torch.bfloat16),
                        torch.zeros(1, 2048, 32, dtype=torch.bfloat16),
                        pooled=torch.zeros(1, 2048, 2, 16))
+
+
+def test_plain_c_caller(tmp_path):
+    """tests/c_abi_host.c, compiled as C99 against include/msa.h and linked
+    with libmsa, sizes workspaces and gets argument errors back as statuses."""
+    import shutil
+    import subprocess
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("no C compiler")
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    pkg = os.path.join(root, "block_sparse_gqa_05_b200")
+    exe = str(tmp_path / "c_abi_host")
+    subprocess.run([gcc, "-std=c99", "-Wall", "-Wextra", "-Werror", "-I",
+                    os.path.join(root, "include"), os.path.join(root, "tests", "c_abi_host.c"),
+                    "-o", exe, os.path.join(pkg, "libmsa.so"), "-Wl,-rpath," + pkg],
+                   check=True)
+    out = subprocess.run([exe], capture_output=True, text=True)
+    assert out.returncode == 0 and out.stdout.strip() == "ok", out.stdout + out.stderr
