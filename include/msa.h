@@ -35,6 +35,9 @@
  *   q_idx    [B, T, G, d_i] bf16        k_idx  [B, N, d_i]   bf16
  *   pooled   [B, T, G, nb]  float32     sel    [B, T, G, k]  int32
  *   lse      [B, T, H]      float32 (natural-log softmax normaliser; optional)
+ *   kl       [B, T, G]      float32 (alignment divergence, msa_forward_alignment)
+ *   paged decode caches: k, v [P, G, 128, d], k_idx [P, 128, d_i] bf16 with
+ *   a page table [B, nb] int32 (msa_forward_decode_paged)
  *
  * Ownership: the caller allocates every buffer (device memory unless stated)
  * and the optional workspace.  The library never allocates or frees device
@@ -48,7 +51,9 @@
  * read by msa_device_status() and the kernel returns early.
  *
  * Limits: Bk == 128; d in {64, 128}; d_i in {32, 64}; 1 <= k <= 64;
- * r = H/G in {1, 2, 4, 8, 16}; G divides 128; q_offset + T <= N.
+ * r = H/G in {1, 2, 4, 8, 16}; G divides 128; q_offset + T <= N.  Prefill
+ * also needs 8 * nb <= 200 KiB and 8*k*H + 8*H + 8*G*k <= 227 KiB (per-CTA
+ * tables); shapes past them return MSA_ERR_UNSUPPORTED.
  */
 #ifndef MSA_H_
 #define MSA_H_
