@@ -231,6 +231,20 @@ def prefill_step_bound(sp, sel, peaks, ms):
                      "top-k bytes at HBM copy bandwidth"}
 
 
+def dense_flops(sp):
+    """Causal GQA attention: 4*H*d FLOP per (query, causal key) pair."""
+    pos = positions(sp)
+    return float(sp.batch * 4 * sp.n_q_heads * sp.head_dim * (pos + 1).sum())
+
+
+def dense_roofline(sp, ms, peaks):
+    """The dense causal GQA prefill kernel against the sustained bf16 peak."""
+    pk = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
+    a = dense_flops(sp) / (ms / 1e3) / 1e12
+    return {"bound": "tensor", "achieved": round(a, 1), "peak": pk, "unit": "TFLOP/s",
+            "frac": round(a / pk, 4), "algorithmic_per_launch": dense_flops(sp)}
+
+
 def decode_kv_bytes(sp):
     return float(sp.batch * sp.n_kv_heads * sp.topk * 128 * sp.head_dim * 2 * 2)
 
@@ -334,7 +348,8 @@ def run_msa(args, world, rank, pg):
             M.dense_attn_prefill(sh, inp.q, inp.k, inp.v, o=o, lse=None, want_lse=False)
         dms = timed_loop(dstep, 2, 1, pg, stream)
         out["dense_gqa_prefill"] = {"ms_per_step": dms, "value": tokens * token_ranks / (dms / 1e3),
-                                    "speedup_msa_vs_dense": round(dms / ms, 2)}
+                                    "speedup_msa_vs_dense": round(dms / ms, 2),
+                                    "roofline": dense_roofline(sp, dms, peaks)}
 
     # ---- end to end through the public API with host buffers.  Each step
     # copies its inputs from pinned host memory, runs msa_forward and copies
@@ -544,7 +559,8 @@ def run_long(M, args, pg, stream, world, rank, peaks):
             M.dense_attn_prefill(sh, inp.q, inp.k, inp.v, o=o, lse=None, want_lse=False)
         dms = timed_loop(dstep, 2, 1, pg, stream)
         pre["dense_gqa_prefill"] = {"ms_per_step": dms, "value": sp.seq_q * world / (dms / 1e3),
-                                    "speedup_msa_vs_dense": round(dms / ms, 2)}
+                                    "speedup_msa_vs_dense": round(dms / ms, 2),
+                                    "roofline": dense_roofline(sp, dms, peaks)}
     except M.MsaError as e:
         pre["dense_gqa_prefill"] = {"unavailable": str(e)}
     pre["step_roofline"] = prefill_step_bound(sp, sel, peaks, ms)
@@ -621,6 +637,7 @@ def run_oracle_sample(sp, budget_s, rng_seed=0):
 def cpu_baseline(sp, budget_s):
     n, s, desc = run_oracle_sample(sp, budget_s)
     return {"value": n / s, "unit": "tokens/s", "cores": oracle_threads(), "kind": "oracle",
+            "precision": "fp64 NumPy (the oracle as it stands, stricter than fp32)",
             "sample": desc, "seconds": round(s, 2)}
 
 
@@ -644,7 +661,9 @@ def run_reference(args, world, rank, pg):
             "config": {"workload": args.workload, "seq_len": sp.seq_kv, "global_batch": sp.batch,
                        "parallelism": "single process on host cores (oracle)"},
             "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": oracle_threads(),
-                             "kind": "oracle", "sample": desc},
+                             "kind": "oracle",
+                             "precision": "fp64 NumPy (the oracle as it stands, stricter than fp32)",
+                             "sample": desc},
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
     return line

@@ -12,7 +12,6 @@ __device__ uint32_t g_device_error;
 
 namespace {
 
-constexpr int kMaxDevices = 64;
 DevCtx g_ctx[kMaxDevices];
 std::mutex g_ctx_mu;
 

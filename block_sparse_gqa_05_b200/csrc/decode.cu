@@ -642,19 +642,20 @@ cudaError_t launch_decode(const msa_shape& s, const uint16_t* q, const uint16_t*
 // ------------------------------------------------ decode without allocation
 // Split-K scratch of msa_sparse_attn_decode_static: one static array in
 // device memory, shared by every call on a device.  Host code only ever
-// passes its device address, looked up once per device.
+// passes its device address, looked up once per device and cached for the
+// life of the process (like the error word: a device reset makes it stale).
 namespace msa {
 namespace {
 
 static __device__ __align__(256) unsigned char g_decode_static_scratch[MSA_DECODE_STATIC_SCRATCH_BYTES];
 
 std::mutex g_static_mu;
-void* g_static_addr[64] = {};
+void* g_static_addr[kMaxDevices] = {};
 
 // Device address of the scratch array on the current device (nullptr on error).
 void* static_scratch_address() {
   int dev = -1;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
   std::lock_guard<std::mutex> lk(g_static_mu);
   if (!g_static_addr[dev]) {
     void* ptr = nullptr;

@@ -10,7 +10,13 @@
 
 namespace msa {
 
+// Most devices a process may use the library on (per-device tables are this long).
+constexpr int kMaxDevices = 64;
+
 // Per-device context: the device error word (a __device__ symbol) and SM count.
+// Looked up once per device and kept for the life of the process: after a
+// cudaDeviceReset the cached device addresses are stale, so a process that
+// resets a device must not call the library on it again.
 struct DevCtx {
   uint32_t* err = nullptr;
   int num_sms = 0;

@@ -139,7 +139,15 @@ msa_status msa_block_topk(const msa_shape* shape, const float* pooled, int32_t* 
  * lse may be NULL.
  * ws/ws_bytes: workspace of at least msa_workspace_size(MSA_OP_SPARSE_PREFILL).
  * KV-outer schedule ([P4]): each selected 128-row K/V block of a group is
- * loaded once and reused by every (token, head) row that selected it. */
+ * loaded once and reused by every (token, head) row that selected it.
+ * Workspace growth: the schedule keeps one bf16 partial output per selected
+ * (token, group, block), so the workspace grows with B*T*H*k*d: about
+ * 2*H*k*d + 8*H*k bytes per query token (264 KiB at H = 64, k = 16, d = 128;
+ * some 34 GiB at T = 131072).  A prefill that does not fit is run as several
+ * calls over consecutive chunks of query rows against the same caches: each
+ * chunk passes its own rows of q/q_idx/o, T = chunk length and q_offset =
+ * position of its first row (causality and the local block follow from
+ * q_offset alone). */
 msa_status msa_sparse_attn_prefill(const msa_shape* shape, const uint16_t* q,
                                    const uint16_t* k, const uint16_t* v,
                                    const int32_t* sel, uint16_t* o, float* lse,
@@ -160,8 +168,9 @@ msa_status msa_sparse_attn_decode(const msa_shape* shape, const uint16_t* q,
 /* Whole layer: index scores -> top-k -> sparse attention (prefill path when
  * T > 1, decode path when T == 1), one stream, no host synchronisation.
  * sel_out (may be NULL) receives the selection.  ws >= msa_workspace_size(
- * MSA_OP_FORWARD); the pooled scores live in the workspace and entries with
- * j > b_t are left unwritten there. */
+ * MSA_OP_FORWARD); it grows with B*T*H*k*d like the prefill attention's (see
+ * msa_sparse_attn_prefill: long prefills are run in chunks of query rows with
+ * q_offset set to each chunk's first position). */
 msa_status msa_forward(const msa_shape* shape, const uint16_t* q, const uint16_t* k,
                        const uint16_t* v, const uint16_t* q_idx, const uint16_t* k_idx,
                        uint16_t* o, float* lse, int32_t* sel_out, void* ws,

@@ -29,7 +29,7 @@ Attention (MSA) : attention block-sparse à deux branches…"):
    main branch's attention distribution over the selected blocks against the
    index branch's distribution over the same blocks.
 
-Readings where the pages are silent (each listed in the design notes):
+Readings where the pages are silent:
   * index score: raw dot product, no scale / activation (P3 names only Q_idx.K_idx;
     only the ordering is used);
   * blocks are aligned at absolute position 0: block b = [bB, (b+1)B);
