@@ -7,7 +7,10 @@
 // Schedule (KV-outer):
 //  1. invert sel: for every (sequence, group, block) column, the list of
 //     (token, slot) pairs that selected it (counting sort in three passes);
-//  2. cut every column into tiles of 128/r tokens = 128 (token, head) rows;
+//  2. cut every column into tiles of 128/r tokens = 128 (token, head) rows and
+//     deal the tiles of every (sequence, group) segment evenly over the CTAs,
+//     segment after segment, so that every CTA gets the same share of every
+//     group's work;
 //  3. persistent tcgen05 kernel: each selected K/V block is TMA-loaded once per
 //     CTA that works on it and reused by every tile of its column; for a tile,
 //     S = Q K^T (TMEM), softmax over the block (causal mask on the local
@@ -19,6 +22,8 @@
 //     position of each (token, group, slot) in the entry list.
 #include <math.h>
 
+#include <algorithm>
+
 #include "internal.h"
 #include "ptx.cuh"
 
@@ -29,18 +34,24 @@ constexpr float kLog2e = 1.4426950408889634f;
 constexpr int kAttnThreads = 512;   // 4 warpgroups: TMA+MMA, 2 softmax, epilogue
 constexpr int kHistTokens = 1024;   // tokens per CTA of the inversion passes
 
+constexpr int kMaxAttnGrid = 1024;  // most CTAs of the attention kernel (one per SM)
 struct PrefillWs {
   uint32_t* col_count;   // [ncol]
   uint32_t* col_fill;    // [ncol]
   uint32_t* col_off;     // [ncol + 1]
-  uint32_t* tile_off;    // [ncol + 1]
+  uint32_t* tile_off;    // [ncol + 1]  tiles of the columns in column order
   uint32_t* entries;     // [B*T*G*k]   (t << 6) | slot, sorted by column
   uint32_t* inv;         // [B*T*G*k]   position in entries of each selected (t, g, slot)
-  int4* tiles;           // [max_tiles] (column, entry start, count, 0)
+  uint32_t* cta_off;     // [kMaxAttnGrid + 1] first tile of each CTA in the dealt order
+  uint32_t* seg_prefix;  // [nseg * kMaxAttnGrid] tiles of a CTA in the segments before one
+  int4* tiles;           // [max_tiles] (column, entry start, count, 0), dealt order
   uint32_t* tile_ent;    // [max_tiles * tpt] entries of each tile, 0xFFFFFFFF past its count
   uint16_t* part_o;      // [entry, r, d] bf16 partial outputs, normalised by their own l
   float* part_ml;        // [entry, r, 2] (running max m, sum l) of each partial, log2 units
-  long long ncol, max_tiles;
+  // columns are (b * G + g) * nb + block; a segment is the nb columns of one
+  // (b, g)
+  long long ncol, nseg, max_tiles;
+  size_t bytes;
 };
 
 PrefillWs carve(const msa_shape& s, void* base) {
@@ -48,9 +59,10 @@ PrefillWs carve(const msa_shape& s, void* base) {
   const long long nb = ceil_div(s.seq_kv, 128);
   const int r = s.n_q_heads / s.n_kv_heads;
   const int tpt = 128 / r;
-  w.ncol = static_cast<long long>(s.batch) * s.n_kv_heads * nb;
+  w.nseg = static_cast<long long>(s.batch) * s.n_kv_heads;
+  w.ncol = w.nseg * nb;
   const long long nent = static_cast<long long>(s.batch) * s.seq_q * s.n_kv_heads * s.topk;
-  w.max_tiles = ceil_div(nent, tpt) + w.ncol;
+  w.max_tiles = ceil_div(nent, tpt) + std::min(w.ncol, nent);
   char* p = static_cast<char*>(base);
   size_t off = 0;
   auto take = [&](size_t bytes) {
@@ -64,31 +76,18 @@ PrefillWs carve(const msa_shape& s, void* base) {
   w.tile_off = reinterpret_cast<uint32_t*>(take(4 * (w.ncol + 1)));
   w.entries = reinterpret_cast<uint32_t*>(take(4 * nent));
   w.inv = reinterpret_cast<uint32_t*>(take(4 * nent));
+  w.cta_off = reinterpret_cast<uint32_t*>(take(4 * (kMaxAttnGrid + 1)));
+  w.seg_prefix = reinterpret_cast<uint32_t*>(take(4ull * w.nseg * kMaxAttnGrid));
   w.tiles = reinterpret_cast<int4*>(take(16 * w.max_tiles));
   w.tile_ent = reinterpret_cast<uint32_t*>(take(4ull * w.max_tiles * tpt));
   w.part_o = reinterpret_cast<uint16_t*>(take(2ull * s.batch * s.seq_q * s.n_q_heads *
                                               s.topk * s.head_dim));
   w.part_ml = reinterpret_cast<float*>(take(8ull * s.batch * s.seq_q * s.n_q_heads * s.topk));
+  w.bytes = off;
   return w;
 }
 
-size_t carve_bytes(const msa_shape& s) {
-  const long long nb = ceil_div(s.seq_kv, 128);
-  const int r = s.n_q_heads / s.n_kv_heads;
-  const int tpt = 128 / r;
-  const long long ncol = static_cast<long long>(s.batch) * s.n_kv_heads * nb;
-  const long long nent = static_cast<long long>(s.batch) * s.seq_q * s.n_kv_heads * s.topk;
-  const long long max_tiles = ceil_div(nent, tpt) + ncol;
-  size_t b = 0;
-  b += align_up(4 * ncol, 256) * 2;
-  b += align_up(4 * (ncol + 1), 256) * 2;
-  b += align_up(4 * nent, 256) * 2;
-  b += align_up(16 * max_tiles, 256);
-  b += align_up(4ull * max_tiles * tpt, 256);
-  b += align_up(2ull * s.batch * s.seq_q * s.n_q_heads * s.topk * s.head_dim, 256);
-  b += align_up(8ull * s.batch * s.seq_q * s.n_q_heads * s.topk, 256);
-  return b;
-}
+size_t carve_bytes(const msa_shape& s) { return carve(s, nullptr).bytes; }
 
 // ------------------------------------------------------- 1. invert selection
 // grid: (ceil(T / kHistTokens), B*G).  Pass 0 counts (sequence, group, block)
@@ -199,9 +198,57 @@ __global__ void __launch_bounds__(1024) scan_columns_kernel(PrefillWs w, int tpt
   }
 }
 
+// Tiles of segment s dealt to CTA c: [first(c), first(c + 1)) of its n_s
+// tiles in column order, first(c) = c * n_s / grid, and the CTA holding
+// segment tile x.
+__device__ __forceinline__ long long deal_first(long long c, long long n, int grid) {
+  return c * n / grid;
+}
+__device__ __forceinline__ int deal_cta(long long x, long long n, int grid) {
+  return static_cast<int>(((x + 1) * grid + n - 1) / n - 1);
+}
+
+// One CTA: per attention CTA c, the tiles it holds in the segments before
+// each segment (seg_prefix) and its first tile in the dealt order (cta_off).
+__global__ void __launch_bounds__(1024) plan_ctas_kernel(PrefillWs w, int nb, int grid) {
+  __shared__ uint32_t warp_sum[32];
+  const int c = threadIdx.x, lane = c & 31, warp = c >> 5;
+  uint32_t acc = 0;
+  if (c < grid) {
+    for (long long sg = 0; sg < w.nseg; ++sg) {
+      const long long lo = w.tile_off[sg * nb];
+      const long long n = static_cast<long long>(w.tile_off[(sg + 1) * nb]) - lo;
+      w.seg_prefix[sg * grid + c] = acc;
+      acc += static_cast<uint32_t>(deal_first(c + 1, n, grid) - deal_first(c, n, grid));
+    }
+  }
+  uint32_t incl = acc;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const uint32_t y = __shfl_up_sync(0xffffffffu, incl, off);
+    if (lane >= off) incl += y;
+  }
+  if (lane == 31) warp_sum[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    uint32_t v = warp_sum[lane];
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const uint32_t y = __shfl_up_sync(0xffffffffu, v, off);
+      if (lane >= off) v += y;
+    }
+    warp_sum[lane] = v;
+  }
+  __syncthreads();
+  const uint32_t excl = (warp ? warp_sum[warp - 1] : 0u) + incl - acc;
+  if (c < grid) w.cta_off[c] = excl;
+  if (c == grid - 1) w.cta_off[grid] = excl + acc;
+}
+
 // One thread per tile: find its column (upper bound in the tile offsets),
-// write the descriptor and the tile's entries padded to tpt.
-__global__ void make_tiles_kernel(PrefillWs w, int tpt) {
+// write the descriptor and the tile's entries padded to tpt at the tile's
+// place in the dealt order.
+__global__ void make_tiles_kernel(PrefillWs w, int tpt, int nb, int grid) {
   const long long ntiles = static_cast<long long>(w.tile_off[w.ncol]);
   for (long long ti = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; ti < ntiles;
        ti += static_cast<long long>(gridDim.x) * blockDim.x) {
@@ -214,9 +261,16 @@ __global__ void make_tiles_kernel(PrefillWs w, int tpt) {
     const uint32_t i = static_cast<uint32_t>(ti - w.tile_off[c]);
     const uint32_t start = w.col_off[c] + i * tpt;
     const uint32_t cnt = min(static_cast<uint32_t>(tpt), w.col_count[c] - i * tpt);
-    w.tiles[ti] = make_int4(static_cast<int>(c), static_cast<int>(start), static_cast<int>(cnt), 0);
+    const long long sg = c / nb;
+    const long long slo = w.tile_off[sg * nb];
+    const long long n = static_cast<long long>(w.tile_off[(sg + 1) * nb]) - slo;
+    const long long x = ti - slo;
+    const int cta = deal_cta(x, n, grid);
+    const long long dst = static_cast<long long>(w.cta_off[cta]) + w.seg_prefix[sg * grid + cta] +
+                          (x - deal_first(cta, n, grid));
+    w.tiles[dst] = make_int4(static_cast<int>(c), static_cast<int>(start), static_cast<int>(cnt), 0);
     for (int j = 0; j < tpt; ++j)
-      w.tile_ent[ti * tpt + j] = j < static_cast<int>(cnt) ? w.entries[start + j] : 0xFFFFFFFFu;
+      w.tile_ent[dst * tpt + j] = j < static_cast<int>(cnt) ? w.entries[start + j] : 0xFFFFFFFFu;
   }
 }
 
@@ -229,38 +283,48 @@ struct AttnParams {
   float scale_log2;
 };
 
-constexpr int kNQ = 3;        // query tile buffers
-constexpr int kNS = 3;        // S/P buffers in TMEM (128 columns each)
+constexpr int kNS = 2;        // S/P buffers in TMEM (128 columns each), one per softmax warpgroup
+constexpr int kNO = 2;        // O buffers in TMEM (D columns each), one per softmax warpgroup
 constexpr int kMBMax = 16;    // most tiles per metadata batch (two batches in flight)
 constexpr int kTentWords = 256; // entry words in the metadata ring (both batches)
 
 template <int D>
 struct AttnSmem {
+  static constexpr int kNQ = D == 128 ? 2 : 3;   // query tile buffers
+  // V tiles: with two, the next column's V loads while this one's PVs run
+  static constexpr int kNV = 2;
   static constexpr uint32_t kKV = 128u * D * 2u;     // one K (or V) block tile
   static constexpr uint32_t kQ = 128u * D * 2u;      // 128 query rows
   static constexpr uint32_t kOffK = 0;                      // two K stages
-  static constexpr uint32_t kOffV = 2 * kKV;                // one V tile
-  static constexpr uint32_t kOffQ = 3 * kKV;
+  static constexpr uint32_t kOffV = 2 * kKV;                // kNV V stages
+  static constexpr uint32_t kOffQ = kOffV + kNV * kKV;
   static constexpr uint32_t kOffStage = kOffQ + kNQ * kQ;   // epilogue staging (128 rows x D)
   static constexpr uint32_t kOffLinv = kOffStage + kQ;      // float [2][128]
-  static constexpr uint32_t kOffMeta = kOffLinv + 1024;     // int [kNQ][4]
+  static constexpr uint32_t kOffMeta = kOffLinv + 1024;     // int [kNQ][4] (kNQ <= 4)
   // int4 [2*kMBMax] per tile: group (b*G+g), block, entries, flags (1: first
   // tile of its column here, 2: last)
   static constexpr uint32_t kOffThdr = kOffMeta + 64;
   static constexpr uint32_t kOffTrow = kOffThdr + 2 * kMBMax * 16;   // int [kTentWords] query row
   static constexpr uint32_t kOffBar = kOffTrow + kTentWords * 4;
-  static constexpr uint32_t kBytes = kOffBar + 256;
+  // barriers: K 2+2, V kNV+kNV, Q kNQ+kNQ, S/P kNS+kNS, O 2+2, 1/l 2+2,
+  // metadata 2+2; then the TMEM address and the abort flag
+  static constexpr uint32_t kNBars = 4 + 2 * kNV + 2 * kNQ + 2 * kNS + 12;
+  static constexpr uint32_t kBytes = kOffBar + kNBars * 8 + 8;
+  static_assert(kBytes <= 227u * 1024u, "shared memory of one CTA");
 };
 
-// Roles by warpgroup: WG0 = warp 0 TMA producer + warp 1 MMA issuer (warps 2-3
-// idle), WG1 and WG2 = softmax of alternate tiles, WG3 = epilogue.  Register
-// budget per thread is moved from WG0/WG3 to the softmax warpgroups so that a
-// softmax thread holds its whole 128-score row.
-// TMEM: three S/P buffers at columns [0,384) (P is written over the first 64
-// columns of its tile's S as packed bf16 and consumed from there by the PV
-// MMA), so S(j+1) and S(j+2) can be computed while tile j's softmax runs;
-// then the O buffers: one of 128 columns for d = 128 (the epilogue drains it
-// long before the next PV completes), two of 64 for d = 64.
+// Roles by warpgroup: WG0 = warps 0 and 3 gather the query tiles (TMA) and
+// load K (warp 0) and V (warp 3) at column changes, warp 1 issues the MMAs,
+// warp 2 prepares tile metadata; WG1 and WG2 = softmax of alternate tiles;
+// WG3 = epilogue.  Register budget per thread is moved from WG0/WG3 to the
+// softmax warpgroups so that a softmax thread holds its whole 128-score row.
+// TMEM: each softmax warpgroup owns one S/P buffer of 128 columns (P is
+// written over the first 64 columns of its tile's S as packed bf16 and
+// consumed from there by the PV MMA) and one O buffer of D columns, so a
+// tile's PV never waits for the previous tile's output to be drained: the
+// epilogue has a whole tile of time to read O out.  S(j + 2) reuses tile j's
+// buffer and is issued once PV(j) is (tcgen05 MMAs of one thread run in
+// issue order).
 template <int D>
 __global__ void __launch_bounds__(kAttnThreads, 1)
     kvouter_attn_kernel(const __grid_constant__ CUtensorMap tm_q,
@@ -269,10 +333,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                         const __grid_constant__ CUtensorMap tm_o,
                         const __grid_constant__ CUtensorMap tm_ot, const AttnParams p) {
   using L = AttnSmem<D>;
+  constexpr int kNQ = L::kNQ;
+  constexpr int kNV = L::kNV;
+  static_assert(kNQ <= 4, "meta holds four query buffers");
   constexpr uint32_t kIdescS = idesc_bf16(128, 128, 0, 0);   // Q (K-major) x K (K-major)
   constexpr uint32_t kIdescO = idesc_bf16(128, D, 0, 1);     // P (TMEM) x V (MN-major)
   constexpr uint32_t kTmemCols = 512;
-  constexpr int kNO = D == 128 ? 1 : 2;    // O buffers: kNS*128 + kNO*D = 512 columns
   static_assert(kNS * 128 + kNO * D <= static_cast<int>(kTmemCols), "TMEM columns");
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   // the swizzled operand tiles need 1024-byte alignment; the launch reserves no slack
@@ -287,11 +353,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kOffBar);
   uint64_t* kfull = bars;               // [2]  K stage loaded
   uint64_t* kempty = bars + 2;          // [2]  K stage free (last S of its column done)
-  uint64_t* vfull = bars + 4;           // V tile loaded
-  uint64_t* vempty = bars + 5;          // V tile free (last PV of its column done)
-  uint64_t* qfull = bars + 6;           // [kNQ]
-  uint64_t* qempty = bars + 6 + kNQ;    // [kNQ]
-  uint64_t* sfull = bars + 6 + 2 * kNQ; // [kNS]
+  uint64_t* vfull = bars + 4;           // [kNV] V stage loaded
+  uint64_t* vempty = vfull + kNV;       // [kNV] V stage free (last PV of its column done)
+  uint64_t* qfull = vempty + kNV;       // [kNQ]
+  uint64_t* qempty = qfull + kNQ;       // [kNQ]
+  uint64_t* sfull = qempty + kNQ;       // [kNS]
   uint64_t* pfull = sfull + kNS;        // [kNS]
   uint64_t* ofull = pfull + kNS;        // [kNO]
   uint64_t* ofree = ofull + 2;          // [kNO]
@@ -307,8 +373,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int wgid = warp >> 2;
   const long long ntiles = static_cast<long long>(p.w.tile_off[p.w.ncol]);
-  const long long t_begin = ntiles * blockIdx.x / gridDim.x;
-  const long long t_end = ntiles * (blockIdx.x + 1) / gridDim.x;
+  const long long t_begin = p.w.cta_off[blockIdx.x];
+  const long long t_end = p.w.cta_off[blockIdx.x + 1];
   const long long n = t_end - t_begin;
   const int tpt = p.tpt;
 
@@ -325,12 +391,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       mbar_init(&lfull[i], 128);
       mbar_init(&lempty[i], 128);
       mbar_init(&mfull[i], 32);
-      mbar_init(&mempty[i], 1);
+      mbar_init(&mempty[i], 2);          // both gather warps
     }
-    mbar_init(vfull, 1);
-    mbar_init(vempty, 1);
+    for (int i = 0; i < kNV; ++i) {
+      mbar_init(&vfull[i], 1);
+      mbar_init(&vempty[i], 1);
+    }
     for (int i = 0; i < kNQ; ++i) {
-      mbar_init(&qfull[i], 1);
+      mbar_init(&qfull[i], 2);           // both gather warps (expect_tx arrivals)
       mbar_init(&qempty[i], 1);
     }
     *abort_flag = 0;
@@ -349,26 +417,26 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   const uint32_t tO = tmem + kNS * 128;    // kNO O buffers of D columns
 
   if (wgid == 0) {
-    regs_dec<56>();
-    if (warp == 0) {
-      // --------------------------------------------------------------- TMA
-      // The whole warp walks the tiles: lane j gathers tokens j, j+32, ... of
-      // a tile (up to 128 tokens when r = 1).  Tile metadata comes from the
-      // shared ring filled by warp 2.
+    regs_dec<64>();
+    if (warp == 0 || warp == 3) {
+      // ------------------------------------------------------- query gather
+      // Warps 0 and 3 walk the tiles together and split every tile's tokens
+      // (token j goes to warp j & 1): one TMA request from one thread moves
+      // slowly, so two warps issue in parallel.  At a column change warp 0
+      // also loads the column's K and warp 3 its V.  Tile metadata comes from
+      // the shared ring filled by warp 2.
+      const int gw = warp == 0 ? 0 : 1;
       if (n > 0) {
         if (lane == 0) {
           tma_prefetch_desc(&tm_q);
-          tma_prefetch_desc(&tm_k);
-          tma_prefetch_desc(&tm_v);
+          tma_prefetch_desc(gw == 0 ? &tm_k : &tm_v);
         }
-        // running counters only, and every per-tile value prepared by the
-        // metadata warp: this loop is the pacing stage of the kernel
         int u = -1;                    // column ordinal
         int ib = 0, ms = 0;            // tile within its metadata batch, batch slot
         uint32_t mph = 0;              // parity of that slot's barriers
         int qb = 0;                    // query buffer
         uint32_t qph = 0;              // its parity
-        const int nx = (tpt + 31) >> 5;
+        const int nx = (tpt + 63) >> 6;   // this warp's tokens per lane (<= 2)
         for (long long i = 0; i < n; ++i) {
           int ok = 1;
           if (ib == 0) {
@@ -378,9 +446,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           }
           const int4 hd = thdr[ms * kMBMax + ib];
           const int* tr = trow + (ms * kmb + ib) * tpt;
-          int rows[4];
+          // this warp's tokens j = 2 * (lane + 32 x) + gw
+          int rows[2];
 #pragma unroll
-          for (int x = 0; x < 4; ++x) rows[x] = x < nx && lane + 32 * x < tpt ? tr[lane + 32 * x] : -1;
+          for (int x = 0; x < 2; ++x) {
+            const int j = 2 * (lane + 32 * x) + gw;
+            rows[x] = x < nx && j < tpt ? tr[j] : -1;
+          }
           __syncwarp();
           if (++ib == kmb || i + 1 == n) {
             if (lane == 0) mbar_arrive(&mempty[ms]);
@@ -389,37 +461,28 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             if (ms == 0) mph ^= 1u;
           }
           const bool newcol = (hd.w & 1) != 0;
-          if (newcol) {
-            ++u;
-            const int st = u & 1;
-            if (lane == 0) {
-              ok = mbar_wait(&kempty[st], ((u >> 1) & 1) ^ 1, abort_flag, p.err) ? 1 : 0;
-              if (ok) {
-                mbar_arrive_expect_tx(&kfull[st], L::kKV);
-#pragma unroll
-                for (int c = 0; c < D / 64; ++c)
-                  tma_load_3d(smem + L::kOffK + st * L::kKV + c * 16384, &tm_k, &kfull[st],
-                              c * 64, hd.y * 128, hd.x);
-              }
-            }
-            ok = __shfl_sync(0xffffffffu, ok, 0);
-            if (!ok) break;
-          }
+          if (newcol) ++u;
+          // the tile's queries first: they never wait on a K or V stage, and
+          // S(i) may be needed before the PV that frees the next column's V
           if (lane == 0) {
             ok = mbar_wait(&qempty[qb], qph ^ 1u, abort_flag, p.err) ? 1 : 0;
             if (ok) {
-              meta[qb * 4 + 0] = u & 1;
-              meta[qb * 4 + 1] = newcol ? 1 : 0;
-              meta[qb * 4 + 2] = (hd.w & 2) != 0 ? 1 : 0;
-              mbar_arrive_expect_tx(&qfull[qb], static_cast<uint32_t>(hd.z * p.r * D * 2));
+              if (gw == 0) {
+                meta[qb * 4 + 0] = u & 1;
+                meta[qb * 4 + 1] = newcol ? 1 : 0;
+                meta[qb * 4 + 2] = (hd.w & 2) != 0 ? 1 : 0;
+              }
+              // this warp's tokens of the tile's hd.z
+              const int mine = (hd.z + 1 - gw) >> 1;
+              mbar_arrive_expect_tx(&qfull[qb], static_cast<uint32_t>(mine * p.r * D * 2));
             }
           }
           ok = __shfl_sync(0xffffffffu, ok, 0);
           if (!ok) break;
           uint8_t* qdst = smem + L::kOffQ + qb * L::kQ;
 #pragma unroll
-          for (int x = 0; x < 4; ++x) {
-            const int j = lane + 32 * x;
+          for (int x = 0; x < 2; ++x) {
+            const int j = 2 * (lane + 32 * x) + gw;
             if (rows[x] >= 0) {
               if (p.q3d) {
                 // token j's 8 heads x 128 columns as [half][head][64]: two 1 KB
@@ -432,6 +495,36 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                               rows[x]);
               }
             }
+          }
+          // then the column's K (warp 0: stage u % 2 is free once the last S
+          // of column u - 2 is done) or V (warp 3: stage u % kNV is free once
+          // the last PV of column u - kNV is done)
+          if (newcol) {
+            if (lane == 0) {
+              if (gw == 0) {
+                const int st = u & 1;
+                ok = mbar_wait(&kempty[st], ((u >> 1) & 1) ^ 1, abort_flag, p.err) ? 1 : 0;
+                if (ok) {
+                  mbar_arrive_expect_tx(&kfull[st], L::kKV);
+#pragma unroll
+                  for (int c = 0; c < D / 64; ++c)
+                    tma_load_3d(smem + L::kOffK + st * L::kKV + c * 16384, &tm_k, &kfull[st],
+                                c * 64, hd.y * 128, hd.x);
+                }
+              } else {
+                const int vs = u % kNV;
+                ok = mbar_wait(&vempty[vs], ((u / kNV) & 1) ^ 1, abort_flag, p.err) ? 1 : 0;
+                if (ok) {
+                  mbar_arrive_expect_tx(&vfull[vs], L::kKV);
+#pragma unroll
+                  for (int c = 0; c < D / 64; ++c)
+                    tma_load_3d(smem + L::kOffV + vs * L::kKV + c * 16384, &tm_v, &vfull[vs],
+                                c * 64, hd.y * 128, hd.x);
+                }
+              }
+            }
+            ok = __shfl_sync(0xffffffffu, ok, 0);
+            if (!ok) break;
           }
           if (++qb == kNQ) {
             qb = 0;
@@ -490,42 +583,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         mbar_arrive(&mfull[ms]);
       }
       __syncwarp();
-    } else if (warp == 3) {
-      // ------------------------------------------------------------ V loader
-      // One V tile, reloaded when the column changes, as soon as the last PV
-      // of the previous column has completed.  Columns are read 32 tiles at a
-      // time.
-      long long u = -1;
-      int prev_col = -1;
-      bool ok = true;
-      for (long long base = 0; ok && base < n; base += 32) {
-        const int mycol = base + lane < n ? p.w.tiles[t_begin + base + lane].x : -1;
-        const int prevlane = __shfl_up_sync(0xffffffffu, mycol, 1);
-        const bool starts = base + lane < n && (lane == 0 ? mycol != prev_col : mycol != prevlane);
-        unsigned m = __ballot_sync(0xffffffffu, starts);
-        prev_col = __shfl_sync(0xffffffffu, mycol, 31);
-        if (base + 32 > n) prev_col = __shfl_sync(0xffffffffu, mycol, static_cast<int>(n - 1 - base));
-        while (m) {
-          const int src = __ffs(m) - 1;
-          m &= m - 1;
-          const int col = __shfl_sync(0xffffffffu, mycol, src);
-          ++u;
-          if (lane == 0) {
-            ok = mbar_wait(vempty, (u & 1) ^ 1, abort_flag, p.err);
-            if (ok) {
-              const int bg = static_cast<int>(col / p.nb);
-              const int blk = static_cast<int>(col - static_cast<long long>(bg) * p.nb);
-              mbar_arrive_expect_tx(vfull, L::kKV);
-#pragma unroll
-              for (int c = 0; c < D / 64; ++c)
-                tma_load_3d(smem + L::kOffV + c * 16384, &tm_v, vfull, c * 64, blk * 128, bg);
-            }
-          }
-          ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
-          if (!ok) break;
-        }
-      }
-      __syncwarp();
     } else if (warp == 1) {
       // --------------------------------------------------------------- MMA
       // Two in-order streams, S(j) = Q K^T and PV(i) = P V, issued by one
@@ -535,10 +592,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       // of one thread execute in issue order, which makes that reuse safe.
       if (lane == 0 && n > 0) {
         const bool q3d = p.q3d != 0;
+        // descriptors of the operand buffers; a K step adds its byte offset / 16
+        const uint64_t dq0 = smem_desc(smem_u32(smem + L::kOffQ), 16, q3d ? 2048 : 1024, 2);
+        const uint64_t dk0 = smem_desc(smem_u32(smem + L::kOffK), 16, 1024, 2);
+        const uint64_t dv0 = smem_desc(smem_u32(smem + L::kOffV), 16384, 1024, 2);
         long long ns = 0, np = 0;   // next S, next PV
         long long u = -1;           // K column ordinal (S side)
         long long uv = -1;          // V column ordinal (PV side)
-        int stage_of[4] = {0, 0, 0, 0};
         bool last_of_col[4] = {false, false, false, false};
         bool first_of_col[4] = {false, false, false, false};
         bool s_meta = false;        // meta of S(ns) read, waiting for its K stage
@@ -556,7 +616,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
               s_last = meta[qb * 4 + 2] != 0;
               last_of_col[ns & 3] = s_last;
               first_of_col[ns & 3] = newcol;
-              stage_of[ns & 3] = s_st;
               if (newcol) ++u;
               s_meta = true;
               s_st |= newcol ? 0x100 : 0;
@@ -564,15 +623,15 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             if (s_meta && (!(s_st & 0x100) || mbar_test(&kfull[s_st & 1], (u >> 1) & 1))) {
               const int st = s_st & 1;
               tc_fence_after();
-              const uint32_t qa = smem_u32(smem + L::kOffQ + qb * L::kQ);
-              const uint32_t ka = smem_u32(smem + L::kOffK + st * L::kKV);
               const int sb = static_cast<int>(ns % kNS);
+              const uint64_t dq = dq0 + (qb * L::kQ >> 4);
+              const uint64_t dk = dk0 + (st * L::kKV >> 4);
 #pragma unroll
               for (int ks = 0; ks < D / 16; ++ks) {
                 const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
                 const uint32_t qoff = q3d ? (ks >> 2) * 1024 + (ks & 3) * 32 : off;
-                tc_mma_ss(tS + sb * 128, smem_desc(qa + qoff, 16, q3d ? 2048 : 1024, 2),
-                          smem_desc(ka + off, 16, 1024, 2), kIdescS, ks > 0 ? 1u : 0u);
+                tc_mma_ss(tS + sb * 128, dq + (qoff >> 4), dk + (off >> 4), kIdescS,
+                          ks > 0 ? 1u : 0u);
               }
               tc_commit(&sfull[sb]);
               tc_commit(&qempty[qb]);
@@ -587,19 +646,19 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             const int sb = static_cast<int>(np % kNS);
             const int ob = static_cast<int>(np % kNO);
             const bool need_v = first_of_col[np & 3];
-            if ((!need_v || mbar_test(vfull, (uv + 1) & 1)) &&
+            const long long un = need_v ? uv + 1 : uv;   // V column of PV(np)
+            if ((!need_v || mbar_test(&vfull[un % kNV], (un / kNV) & 1)) &&
                 mbar_test(&pfull[sb], (np / kNS) & 1) &&
                 mbar_test(&ofree[ob], ((np / kNO) & 1) ^ 1)) {
-              if (need_v) ++uv;
+              uv = un;
               tc_fence_after();
-              const uint32_t va = smem_u32(smem + L::kOffV);
+              const uint64_t dv = dv0 + ((uv % kNV) * L::kKV >> 4);
 #pragma unroll
-              for (int ks = 0; ks < 8; ++ks) {   // 128 keys in steps of 16 (8 packed columns)
-                const uint64_t bd = smem_desc(va + ks * 16 * 128, 16384, 1024, 2);
-                tc_mma_ts(tO + ob * D, tS + sb * 128 + ks * 8, bd, kIdescO, ks > 0 ? 1u : 0u);
-              }
+              for (int ks = 0; ks < 8; ++ks)   // 128 keys in steps of 16 (8 packed columns)
+                tc_mma_ts(tO + ob * D, tS + sb * 128 + ks * 8, dv + (ks * 16 * 128 >> 4), kIdescO,
+                          ks > 0 ? 1u : 0u);
               tc_commit(&ofull[ob]);
-              if (last_of_col[np & 3]) tc_commit(vempty);
+              if (last_of_col[np & 3]) tc_commit(&vempty[uv % kNV]);
               ++np;
               progress = true;
             }
@@ -616,7 +675,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             break;
           }
         }
-        (void)stage_of;
       }
       __syncwarp();
     }
@@ -893,6 +951,9 @@ __global__ void __launch_bounds__(256, 8) combine_kernel(const int32_t* __restri
   }
 }
 
+// One CTA per SM, at most kMaxAttnGrid (the size of the dealing tables).
+int attn_grid(const DevCtx* ctx) { return std::min(std::max(ctx->num_sms, 1), kMaxAttnGrid); }
+
 template <int D>
 cudaError_t launch_attn(const msa_shape& s, const uint16_t* q, const uint16_t* k,
                         const uint16_t* v, const AttnParams& p, const DevCtx* ctx,
@@ -936,7 +997,7 @@ cudaError_t launch_attn(const msa_shape& s, const uint16_t* q, const uint16_t* k
   if (e != cudaSuccess) return e;
   {
     ProfScope ps_("kvouter_attn", st);
-    kvouter_attn_kernel<D><<<ctx->num_sms, kAttnThreads, smem, st>>>(tq, tk, tv, to, tot, p);
+    kvouter_attn_kernel<D><<<attn_grid(ctx), kAttnThreads, smem, st>>>(tq, tk, tv, to, tot, p);
   }
   return cudaGetLastError();
 }
@@ -956,7 +1017,11 @@ static size_t combine_smem_bytes(const msa_shape& s, bool with_kl) {
 
 bool prefill_shape_supported(const msa_shape& s) {
   const size_t nb = static_cast<size_t>(ceil_div(s.seq_kv, 128));
-  return 8 * nb <= kHistSmemMax && combine_smem_bytes(s, true) <= kCombineSmemMax;
+  const PrefillWs w = carve(s, nullptr);
+  const long long nent = static_cast<long long>(s.batch) * s.seq_q * s.n_kv_heads * s.topk;
+  // 32-bit columns, tile ids and entry positions
+  return 8 * nb <= kHistSmemMax && combine_smem_bytes(s, true) <= kCombineSmemMax &&
+         w.ncol < (1ll << 31) && w.max_tiles < (1ll << 31) && nent < (1ll << 32);
 }
 
 cudaError_t launch_sparse_prefill(const msa_shape& s, const uint16_t* q, const uint16_t* k,
@@ -994,8 +1059,13 @@ cudaError_t launch_sparse_prefill(const msa_shape& s, const uint16_t* q, const u
                                                  s.q_offset, 1, ctx->err);
   }
   {
+    ProfScope ps_("plan_ctas", st);
+    plan_ctas_kernel<<<1, 1024, 0, st>>>(w, nb, attn_grid(ctx));
+  }
+  {
     ProfScope ps_("make_tiles", st);
-    make_tiles_kernel<<<static_cast<unsigned>(ceil_div(w.max_tiles, 256)), 256, 0, st>>>(w, tpt);
+    make_tiles_kernel<<<static_cast<unsigned>(ceil_div(w.max_tiles, 256)), 256, 0, st>>>(
+        w, tpt, nb, attn_grid(ctx));
   }
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
 

@@ -149,6 +149,22 @@ MSA_DEV void bulk_wait_read0() { asm volatile("cp.async.bulk.wait_group.read 0;"
 // Wait until every committed bulk store of this thread has completed.
 MSA_DEV void bulk_wait0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
+// ------------------------------------------------------------- cp.async
+// 16-byte copy global -> shared through L2 only (no L1 allocation).
+MSA_DEV void cp_async16(void* smem_dst, const void* gmem_src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;"
+               ::"r"(smem_u32(smem_dst)), "l"(gmem_src)
+               : "memory");
+}
+// The barrier's current phase cannot complete before every cp.async this
+// thread issued so far has landed (its pending count is raised now and
+// lowered when they land); the thread still makes its own counted arrival.
+MSA_DEV void cp_async_mbar_track(uint64_t* bar) {
+  asm volatile("cp.async.mbarrier.arrive.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+// Wait until every cp.async of this thread has landed.
+MSA_DEV void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+
 // Named barrier over ``count`` threads (id 0 is __syncthreads).
 MSA_DEV void named_bar_sync(uint32_t id, uint32_t count) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
