@@ -78,6 +78,12 @@ bool forward_is_decode(const msa_shape& s) {
   return s.seq_q == 1 && s.q_offset == s.seq_kv - 1;
 }
 
+// Pooled scores in the forward workspace: none when the prefill path fuses
+// the top-k into the index scores (the selection is written directly).
+size_t forward_pooled_bytes(const msa_shape& s) {
+  return !forward_is_decode(s) && index_topk_fusable(s) ? 0 : pooled_bytes(s);
+}
+
 msa_status from_cuda(cudaError_t e) { return e == cudaSuccess ? MSA_OK : MSA_ERR_CUDA; }
 
 // ------------------------------------------------------------- profiling
@@ -235,7 +241,7 @@ msa_status msa_workspace_size(const msa_shape* s, msa_op op, size_t* bytes) {
     case MSA_OP_FORWARD:
       if ((st = check_shape(s, true, true)) != MSA_OK) return st;
       if (!forward_is_decode(*s) && !prefill_shape_supported(*s)) return MSA_ERR_UNSUPPORTED;
-      *bytes = pooled_bytes(*s) + sel_bytes(*s) +
+      *bytes = forward_pooled_bytes(*s) + sel_bytes(*s) +
                (forward_is_decode(*s) ? decode_workspace_bytes(*s, false)
                                       : prefill_workspace_bytes(*s));
       return MSA_OK;
@@ -383,10 +389,18 @@ msa_status msa_forward(const msa_shape* s, const uint16_t* q, const uint16_t* k,
   if (!device_ctx()) return MSA_ERR_CUDA;
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
   char* w = static_cast<char*>(ws);
+  const size_t pb = forward_pooled_bytes(*s);
   float* pooled = reinterpret_cast<float*>(w);
-  int32_t* sel = sel_out ? sel_out : reinterpret_cast<int32_t*>(w + pooled_bytes(*s));
-  void* rest = w + pooled_bytes(*s) + sel_bytes(*s);
-  cudaError_t e = launch_index_scores(*s, q_idx, k_idx, pooled, false, cs);
+  int32_t* sel = sel_out ? sel_out : reinterpret_cast<int32_t*>(w + pb);
+  void* rest = w + pb + sel_bytes(*s);
+  cudaError_t e;
+  if (pb == 0) {
+    // prefill: index scores with the top-k fused in, then the attention
+    e = launch_index_topk(*s, q_idx, k_idx, sel, cs);
+    if (e == cudaSuccess) e = launch_sparse_prefill(*s, q, k, v, sel, o, lse, rest, cs);
+    return from_cuda(e);
+  }
+  e = launch_index_scores(*s, q_idx, k_idx, pooled, false, cs);
   if (e == cudaSuccess) e = launch_block_topk(*s, pooled, sel, cs);
   if (e == cudaSuccess) {
     if (forward_is_decode(*s))

@@ -6,6 +6,13 @@
 // B = two 128-key blocks of k_idx, D = 128 x 256 fp32 scores in TMEM.  The
 // epilogue masks keys past each row's position and reduces the 128 columns to
 // one pooled value, so token scores never leave the SM.
+// With the top-k fused in (the whole layer's prefill path), each CTA walks
+// whole row tiles over all of their causal key blocks, the epilogue hands each
+// block maximum to a top-k warpgroup through a shared-memory ring, and that
+// warpgroup keeps every row's running top-(k-1) and writes the selection
+// (lumi-systems AI news: the exponential-free top-k; yhxrc.cn 第一步: the index
+// branch only has to produce the ordering), so the pooled scores never reach
+// memory either.
 // Decode (T*G < 128): a bandwidth-bound scan of k_idx with mma.sync.
 #include <math.h>
 
@@ -17,13 +24,22 @@ namespace {
 
 constexpr int kStages = 4;       // 256-key k_idx tiles in flight
 constexpr int kAcc = 2;          // TMEM accumulator buffers of 256 columns
-constexpr int kThreads = 320;    // warp 0: TMA, warp 1: MMA, warps 2..9: epilogue
+// warp 0: TMA, warp 1: MMA (warps 2-3 idle), warps 4..11: epilogue, in whole
+// warpgroups so that the fused variant can move registers between them
+constexpr int kThreads = 384;
+constexpr int kTopkThreads = 128;   // fused top-k: warps 12..15, one thread per row
 constexpr int kChunkBlocks = 32; // key blocks per work item
+constexpr int kRing = 8;         // fused top-k: ring slots of one 256-key tile's two block maxima
+// barriers (K stages, Q, accumulators, ring), the TMEM address and the abort
+// flag, rounded up; the fused top-k ring follows them
+constexpr uint32_t kBarBytes = ((2 * kStages + 4 + 2 * kAcc + 2 * kRing) * 8 + 8 + 127) / 128 * 128;
 
 struct IdxParams {
   float* pooled;
+  int32_t* sel;  // fused top-k: [B, T, G, k]
   uint32_t* err;
-  int T, N, G, q_off, nb;
+  int T, N, G, q_off, nb, k;
+  int rowmajor;  // items are whole row tiles, largest first (fused top-k)
   int M;         // row tiles per sequence = ceil(T*G / 128)
   int tpt;       // tokens per row tile = 128 / G
   int kc;        // key blocks per chunk
@@ -57,6 +73,13 @@ struct ItemCursor {
 // in increasing order, so the chunk cursor only moves forward.
 __device__ inline void item_decode(const IdxParams& p, long long w, ItemCursor& cur, int& seq,
                                    int& m, int& b0, int& b1) {
+  if (p.rowmajor) {
+    seq = static_cast<int>(w / p.M);
+    m = p.M - 1 - static_cast<int>(w - static_cast<long long>(seq) * p.M);
+    b0 = 0;
+    b1 = tile_causal_blocks(p, m);
+    return;
+  }
   const int s = static_cast<int>(w / p.items_per_seq);
   const long long r = w - static_cast<long long>(s) * p.items_per_seq;
   if (s != cur.seq) {
@@ -77,8 +100,25 @@ __device__ inline void item_decode(const IdxParams& p, long long w, ItemCursor& 
   b1 = min(b0 + p.kc, ncb);
 }
 
-template <int DI>
-__global__ void __launch_bounds__(kThreads, 1)
+// Maximum of 128 scores with three-input max (four chains of 32 values).
+MSA_DEV float block_max128(const float* v) {
+  float m4[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) m4[i] = fmax3(v[i], v[i + 4], v[i + 8]);
+#pragma unroll
+  for (int c = 12; c < 124; c += 8)
+#pragma unroll
+    for (int i = 0; i < 4; ++i) m4[i] = fmax3(m4[i], v[c + i], v[c + 4 + i]);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) m4[i] = fmaxf(m4[i], v[124 + i]);
+  return fmaxf(fmax3(m4[0], m4[1], m4[2]), m4[3]);
+}
+
+// KMAX = 0: pooled scores out.  KMAX in {16, 32}: the top-k is fused (k <=
+// KMAX) and the selection is written instead; each row keeps the KMAX - 1
+// best of its candidate blocks.
+template <int DI, int KMAX>
+__global__ void __launch_bounds__(kThreads + (KMAX > 0 ? kTopkThreads : 0), 1)
     index_scores_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
                            const __grid_constant__ CUtensorMap tm_k, const IdxParams p) {
   constexpr uint32_t kQTile = 128u * DI * 2u;       // 128 (token, group) rows
@@ -99,8 +139,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* qempty = qfull + 2;
   uint64_t* accfull = qempty + 2;
   uint64_t* accempty = accfull + kAcc;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accempty + kAcc);
+  uint64_t* ring_full = accempty + kAcc;     // fused top-k: [kRing] block maxima written
+  uint64_t* ring_empty = ring_full + kRing;  // fused top-k: [kRing] block maxima consumed
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(ring_empty + kRing);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  // fused top-k: [kRing][2 blocks][128 rows] block maxima, after the barriers
+  float* ring = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(bars) + kBarBytes);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -118,6 +162,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&accfull[i], 1);
       mbar_init(&accempty[i], 128);
     }
+    if constexpr (KMAX > 0) {
+      for (int i = 0; i < kRing; ++i) {
+        mbar_init(&ring_full[i], 128);
+        mbar_init(&ring_empty[i], kTopkThreads);
+      }
+    }
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -127,6 +177,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
+  // fused variant: registers from the producer warpgroup and the top-k
+  // warpgroup to the epilogue (which holds a 128-score row)
+  constexpr uint32_t kRegEpi = KMAX == 0 ? 0 : (KMAX <= 16 ? 176 : 152);
+  constexpr uint32_t kRegTopk = KMAX == 0 ? 0 : (KMAX <= 16 ? 104 : 152);
+  static_assert(KMAX == 0 || (56 + 2 * kRegEpi + kRegTopk <= 4 * 128 && kRegEpi > 128),
+                "register split of the launch (128 per thread)");
+  if (warp < 4) {
+    if constexpr (KMAX > 0) regs_dec<56>();
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
@@ -183,11 +241,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
     __syncwarp();
-  } else {
+  }
+  } else if (warp < 12) {
     // --------------------------------------------- epilogue: mask + block max
     // Warpgroup wg owns accumulator wg and takes every other 256-key tile;
     // each tile holds two key blocks.
-    const int wg = (warp - 2) >> 2;
+    if constexpr (KMAX > 0) regs_inc<kRegEpi>();
+    const int wg = (warp - 4) >> 2;
     const int quarter = warp & 3;            // TMEM lanes 32*quarter .. +31
     const int row = quarter * 32 + lane;
     const uint32_t taddr_row = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + wg * 256;
@@ -203,12 +263,19 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int t = trow / p.G;
       const int pos = p.q_off + t;
       const int bt = pos >> 7;
-      float* out = p.pooled + (static_cast<long long>(seq) * rows_per_seq + trow) *
-                                  static_cast<long long>(p.nb);
+      float* out = KMAX > 0 ? nullptr
+                            : p.pooled + (static_cast<long long>(seq) * rows_per_seq + trow) *
+                                             static_cast<long long>(p.nb);
       for (int b = b0; b < b1; b += 2, ++j) {
         if ((j & 1) != wg) continue;
         if (!(ok = mbar_wait(&accfull[wg], (j >> 1) & 1, abort_flag, p.err))) break;
         tc_fence_after();
+        const int slot = static_cast<int>(j % kRing);
+        if constexpr (KMAX > 0) {
+          // the ring slot must have been consumed by the top-k warpgroup
+          if (!(ok = mbar_wait(&ring_empty[slot], ((j / kRing) & 1) ^ 1, abort_flag, p.err)))
+            break;
+        }
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
           float v[128];
@@ -220,19 +287,15 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_arrive(&accempty[wg]);
           }
           const int bb = b + h;
-          if (valid && bb < b1 && bb <= bt) {
+          if constexpr (KMAX > 0) {
+            // every candidate block lies below the row's local block, so all
+            // of its keys are causal: no mask
+            ring[(slot * 2 + h) * 128 + row] = block_max128(v);
+          } else if (valid && bb < b1 && bb <= bt) {
             const int lim = (bb == bt) ? (pos & 127) : 127;
             float mx;
             if (lim == 127) {
-              float m4[4] = {v[0], v[1], v[2], v[3]};
-#pragma unroll
-              for (int c = 4; c < 128; c += 4) {
-                m4[0] = fmaxf(m4[0], v[c]);
-                m4[1] = fmaxf(m4[1], v[c + 1]);
-                m4[2] = fmaxf(m4[2], v[c + 2]);
-                m4[3] = fmaxf(m4[3], v[c + 3]);
-              }
-              mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
+              mx = block_max128(v);
             } else {
               mx = -INFINITY;
 #pragma unroll
@@ -241,7 +304,88 @@ __global__ void __launch_bounds__(kThreads, 1)
             out[bb] = mx;
           }
         }
+        if constexpr (KMAX > 0) mbar_arrive(&ring_full[slot]);
       }
+    }
+  } else if constexpr (KMAX > 0) {
+    // ------------------------------------------------------- fused top-k
+    // Thread t owns row t of every row tile.  Candidate blocks 0 .. b_t - 1
+    // arrive in increasing order; the row keeps its KMAX - 1 best as
+    // order-preserving score keys, sorted descending.  A block enters only if
+    // its key beats the last kept one (strictly: an equal score from a later,
+    // higher block loses the tie to the lower block already kept), and it is
+    // inserted below every kept key it does not beat.  No exponentials.
+    // the launch gives every thread 128 registers: a larger share is an
+    // increase, a smaller one a release
+    if constexpr (kRegTopk > 128) regs_inc<kRegTopk>();
+    else regs_dec<kRegTopk>();
+    constexpr int L = KMAX > 1 ? KMAX - 1 : 1;
+    const int row = threadIdx.x - kThreads;
+    ItemCursor cur;
+    long long j = 0;
+    bool ok = true;
+    const int rows_per_seq = p.T * p.G;
+    for (long long w = blockIdx.x; ok && w < p.items_total; w += gridDim.x) {
+      int seq, m, b0, b1;
+      item_decode(p, w, cur, seq, m, b0, b1);
+      const int trow = m * 128 + row;
+      const bool valid = trow < rows_per_seq;
+      const int bt = (p.q_off + trow / p.G) >> 7;   // the row's local block
+      uint32_t tk[L];
+      int ti[L];
+#pragma unroll
+      for (int x = 0; x < L; ++x) {
+        tk[x] = 0u;   // below every score key
+        ti[x] = 0x7FFFFFFF;
+      }
+      for (int b = b0; b < b1; b += 2, ++j) {
+        const int slot = static_cast<int>(j % kRing);
+        if (!(ok = mbar_wait(&ring_full[slot], (j / kRing) & 1, abort_flag, p.err))) break;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const int bb = b + h;
+          const uint32_t u = float_order_key(ring[(slot * 2 + h) * 128 + row]);
+          if (bb < bt && u > tk[L - 1]) {
+            bool c[L];
+#pragma unroll
+            for (int x = 0; x < L; ++x) c[x] = u > tk[x];
+#pragma unroll
+            for (int x = L - 1; x > 0; --x) {
+              tk[x] = c[x - 1] ? tk[x - 1] : (c[x] ? u : tk[x]);
+              ti[x] = c[x - 1] ? ti[x - 1] : (c[x] ? bb : ti[x]);
+            }
+            tk[0] = c[0] ? u : tk[0];
+            ti[0] = c[0] ? bb : ti[0];
+          }
+        }
+        mbar_arrive(&ring_empty[slot]);
+      }
+      if (!ok) break;
+      if (!valid) continue;
+      // the kk best in ascending block order, then the local block, then -1
+      const int kk = min(p.k - 1, bt);
+      constexpr int S = L + 1;   // a power of two
+      int srt[S];
+#pragma unroll
+      for (int x = 0; x < S; ++x) srt[x] = x < L && x < kk ? ti[x] : 0x7FFFFFFF;
+#pragma unroll
+      for (int a = 2; a <= S; a <<= 1)
+#pragma unroll
+        for (int d = a >> 1; d > 0; d >>= 1)
+#pragma unroll
+          for (int x = 0; x < S; ++x) {
+            const int y = x ^ d;
+            if (y > x) {
+              const bool up = (x & a) == 0;
+              const int lo = min(srt[x], srt[y]), hi = max(srt[x], srt[y]);
+              srt[x] = up ? lo : hi;
+              srt[y] = up ? hi : lo;
+            }
+          }
+      int32_t* out = p.sel + (static_cast<long long>(seq) * rows_per_seq + trow) * p.k;
+#pragma unroll
+      for (int x = 0; x < KMAX; ++x)
+        if (x < p.k) out[x] = x < kk ? srt[x] : (x == kk ? bt : -1);
     }
   }
 
@@ -379,11 +523,16 @@ __global__ void __launch_bounds__(256) index_scores_scan_kernel(const uint16_t* 
   }
 }
 
-template <int DI>
+// KMAX = 0: pooled scores into ``pooled``; KMAX > 0: the fused top-k writes
+// the selection into ``sel`` (k <= KMAX).
+template <int DI, int KMAX>
 cudaError_t launch_tc(const msa_shape& s, const uint16_t* q_idx, const uint16_t* k_idx,
-                      float* pooled, const DevCtx* ctx, cudaStream_t st) {
+                      float* pooled, int32_t* sel, const DevCtx* ctx, cudaStream_t st) {
   IdxParams p{};
   p.pooled = pooled;
+  p.sel = sel;
+  p.k = s.topk;
+  p.rowmajor = KMAX > 0 ? 1 : 0;
   p.err = ctx->err;
   p.T = s.seq_q;
   p.N = s.seq_kv;
@@ -395,7 +544,11 @@ cudaError_t launch_tc(const msa_shape& s, const uint16_t* q_idx, const uint16_t*
   p.kc = kChunkBlocks;
   p.C = static_cast<int>(ceil_div(static_cast<int64_t>(p.q_off) + p.T, p.kc * 128));
   long long per = 0;
-  for (int c = 0; c < p.C; ++c) per += p.M - chunk_mmin(p, c);
+  if (KMAX > 0) {
+    per = p.M;   // whole row tiles
+  } else {
+    for (int c = 0; c < p.C; ++c) per += p.M - chunk_mmin(p, c);
+  }
   p.items_per_seq = per;
   p.items_total = per * s.batch;
 
@@ -412,17 +565,27 @@ cudaError_t launch_tc(const msa_shape& s, const uint16_t* q_idx, const uint16_t*
       !encode_tmap(&tk, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, k_idx, dk, stride, kbox, sw))
     return cudaErrorInvalidValue;
 
-  const size_t smem = 1024 + (2 * 128 + kStages * 256) * DI * 2 + 256;
-  cudaError_t e = cudaFuncSetAttribute(index_scores_tc_kernel<DI>,
+  // alignment slack, operand tiles, barriers, fused top-k ring
+  const size_t smem = 1024 + (2 * 128 + kStages * 256) * DI * 2 + kBarBytes +
+                      (KMAX > 0 ? kRing * 2 * 128 * 4 : 0);
+  cudaError_t e = cudaFuncSetAttribute(index_scores_tc_kernel<DI, KMAX>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   const long long grid = p.items_total < ctx->num_sms ? p.items_total : ctx->num_sms;
+  const int threads = kThreads + (KMAX > 0 ? kTopkThreads : 0);
   {
-    ProfScope ps_("index_scores_tc", st);
-    index_scores_tc_kernel<DI><<<static_cast<unsigned>(grid), kThreads, smem, st>>>(tq, tk, p);
+    ProfScope ps_(KMAX > 0 ? "index_topk_tc" : "index_scores_tc", st);
+    index_scores_tc_kernel<DI, KMAX><<<static_cast<unsigned>(grid), threads, smem, st>>>(tq, tk, p);
   }
   return cudaGetLastError();
+}
+
+// The tensor-core path needs a full 128-row query tile and a 256-key box;
+// ragged and paged decode always scan.
+bool tc_path(const msa_shape& s) {
+  return static_cast<long long>(s.seq_q) * s.n_kv_heads >= 128 &&
+         static_cast<long long>(s.batch) * s.seq_kv >= 256;
 }
 
 }  // namespace
@@ -435,10 +598,7 @@ cudaError_t launch_index_scores(const msa_shape& s, const uint16_t* q_idx, const
   const int nb = static_cast<int>(ceil_div(s.seq_kv, 128));
   const long long rows = static_cast<long long>(s.batch) * s.seq_q * s.n_kv_heads;
   cudaError_t e;
-  // the tensor-core path needs a full 128-row query tile and a 256-key box;
-  // ragged and paged decode always scan
-  if (lens || pages.table || static_cast<long long>(s.seq_q) * s.n_kv_heads < 128 ||
-      static_cast<long long>(s.batch) * s.seq_kv < 256) {
+  if (lens || pages.table || !tc_path(s)) {
     const int last_bt = (s.q_offset + s.seq_q - 1) / 128;
     const dim3 grid(static_cast<unsigned>(s.batch * s.seq_q),
                     static_cast<unsigned>(ceil_div(last_bt + 1, 8)));
@@ -454,8 +614,8 @@ cudaError_t launch_index_scores(const msa_shape& s, const uint16_t* q_idx, const
                                                          pages.table, pages.num_pages, ctx->err);
     e = cudaGetLastError();
   } else {
-    e = s.index_dim == 64 ? launch_tc<64>(s, q_idx, k_idx, pooled, ctx, st)
-                          : launch_tc<32>(s, q_idx, k_idx, pooled, ctx, st);
+    e = s.index_dim == 64 ? launch_tc<64, 0>(s, q_idx, k_idx, pooled, nullptr, ctx, st)
+                          : launch_tc<32, 0>(s, q_idx, k_idx, pooled, nullptr, ctx, st);
   }
   if (e != cudaSuccess || !fill_upper) return e;
   const long long warps_needed = rows;
@@ -467,6 +627,31 @@ cudaError_t launch_index_scores(const msa_shape& s, const uint16_t* q_idx, const
                                                                    s.n_kv_heads, s.q_offset, nb);
   }
   return cudaGetLastError();
+}
+
+// Whole row tiles are the fused kernel's work items.  Few, long ones (the
+// 1M-context chunk: 512 row tiles of 8192 blocks each) leave the persistent
+// grid's CTAs with uneven shares, and there the chunked kernel plus the
+// standalone top-k is faster; many row tiles, or short rows, balance.  The
+// rule depends on the shape alone, so workspace sizes do not depend on the
+// device.
+bool index_topk_fusable(const msa_shape& s) {
+  if (!tc_path(s) || s.topk > 32) return false;
+  const long long row_tiles = static_cast<long long>(s.batch) *
+                              ceil_div(static_cast<int64_t>(s.seq_q) * s.n_kv_heads, 128);
+  return row_tiles >= 1024 || ceil_div(s.seq_kv, 128) <= 1024;
+}
+
+cudaError_t launch_index_topk(const msa_shape& s, const uint16_t* q_idx, const uint16_t* k_idx,
+                              int32_t* sel, cudaStream_t st) {
+  const DevCtx* ctx = device_ctx();
+  if (!ctx) return cudaErrorInitializationError;
+  if (!index_topk_fusable(s)) return cudaErrorNotSupported;
+  if (s.topk <= 16)
+    return s.index_dim == 64 ? launch_tc<64, 16>(s, q_idx, k_idx, nullptr, sel, ctx, st)
+                             : launch_tc<32, 16>(s, q_idx, k_idx, nullptr, sel, ctx, st);
+  return s.index_dim == 64 ? launch_tc<64, 32>(s, q_idx, k_idx, nullptr, sel, ctx, st)
+                           : launch_tc<32, 32>(s, q_idx, k_idx, nullptr, sel, ctx, st);
 }
 
 }  // namespace msa

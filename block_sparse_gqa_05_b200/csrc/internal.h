@@ -62,6 +62,11 @@ cudaError_t launch_index_scores(const msa_shape& s, const uint16_t* q_idx,
                                 const uint16_t* k_idx, float* pooled, bool fill_upper,
                                 cudaStream_t st, const int32_t* lens = nullptr,
                                 PageTable pages = PageTable{});
+// Index scores with the block top-k fused in (prefill shapes on the tensor-core
+// path, k <= 32): writes the selection directly, no pooled scores.
+bool index_topk_fusable(const msa_shape& s);
+cudaError_t launch_index_topk(const msa_shape& s, const uint16_t* q_idx, const uint16_t* k_idx,
+                              int32_t* sel, cudaStream_t st);
 cudaError_t launch_block_topk(const msa_shape& s, const float* pooled, int32_t* sel,
                               cudaStream_t st, const int32_t* lens = nullptr);
 size_t prefill_workspace_bytes(const msa_shape& s);

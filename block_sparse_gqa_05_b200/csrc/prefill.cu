@@ -298,15 +298,19 @@ struct AttnSmem {
   static constexpr uint32_t kOffK = 0;                      // two K stages
   static constexpr uint32_t kOffV = 2 * kKV;                // kNV V stages
   static constexpr uint32_t kOffQ = kOffV + kNV * kKV;
-  static constexpr uint32_t kOffStage = kOffQ + kNQ * kQ;   // epilogue staging (128 rows x D)
-  static constexpr uint32_t kOffLinv = kOffStage + kQ;      // float [2][128]
-  static constexpr uint32_t kOffMeta = kOffLinv + 1024;     // int [kNQ][4] (kNQ <= 4)
+  // epilogue staging: 128 rows x 64 columns (the rows' halves go out in turn)
+  static constexpr uint32_t kOffStage = kOffQ + kNQ * kQ;
+  // softmax exchange: float [2 tile parities][2 warpgroups][128 rows] partial
+  // row maxima, then the same for the partial row sums
+  static constexpr uint32_t kOffXmax = kOffStage + 16384;
+  static constexpr uint32_t kOffXsum = kOffXmax + 2048;
+  static constexpr uint32_t kOffMeta = kOffXsum + 2048;     // int [kNQ][4] (kNQ <= 4)
   // int4 [2*kMBMax] per tile: group (b*G+g), block, entries, flags (1: first
   // tile of its column here, 2: last)
   static constexpr uint32_t kOffThdr = kOffMeta + 64;
   static constexpr uint32_t kOffTrow = kOffThdr + 2 * kMBMax * 16;   // int [kTentWords] query row
   static constexpr uint32_t kOffBar = kOffTrow + kTentWords * 4;
-  // barriers: K 2+2, V kNV+kNV, Q kNQ+kNQ, S/P kNS+kNS, O 2+2, 1/l 2+2,
+  // barriers: K 2+2, V kNV+kNV, Q kNQ+kNQ, S/P kNS+kNS, O 2+2, row sums 2+2,
   // metadata 2+2; then the TMEM address and the abort flag
   static constexpr uint32_t kNBars = 4 + 2 * kNV + 2 * kNQ + 2 * kNS + 12;
   static constexpr uint32_t kBytes = kOffBar + kNBars * 8 + 8;
@@ -348,7 +352,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   }
   uint8_t* smem = smem_raw;
   const int kmb = min(kMBMax, (kTentWords / 2) / p.tpt);   // tiles per metadata batch
-  float* linv = reinterpret_cast<float*>(smem + L::kOffLinv);
+  float* xmax = reinterpret_cast<float*>(smem + L::kOffXmax);
+  float* xsum = reinterpret_cast<float*>(smem + L::kOffXsum);
   int* meta = reinterpret_cast<int*>(smem + L::kOffMeta);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kOffBar);
   uint64_t* kfull = bars;               // [2]  K stage loaded
@@ -361,8 +366,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   uint64_t* pfull = sfull + kNS;        // [kNS]
   uint64_t* ofull = pfull + kNS;        // [kNO]
   uint64_t* ofree = ofull + 2;          // [kNO]
-  uint64_t* lfull = ofree + 2;          // [2]
-  uint64_t* lempty = lfull + 2;         // [2]
+  uint64_t* lfull = ofree + 2;          // [2] by tile parity: partial row sums written
+  uint64_t* lempty = lfull + 2;         // [2] by tile parity: partial row sums read
   uint64_t* mfull = lempty + 2;         // [2] metadata batch ready
   uint64_t* mempty = mfull + 2;         // [2] metadata batch consumed
   int4* thdr = reinterpret_cast<int4*>(smem + L::kOffThdr);
@@ -381,14 +386,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   if (threadIdx.x == 0) {
     for (int i = 0; i < kNS; ++i) {
       mbar_init(&sfull[i], 1);
-      mbar_init(&pfull[i], 128);
+      mbar_init(&pfull[i], 256);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&kfull[i], 1);
       mbar_init(&kempty[i], 1);
       mbar_init(&ofull[i], 1);
       mbar_init(&ofree[i], 128);
-      mbar_init(&lfull[i], 128);
+      mbar_init(&lfull[i], 256);
       mbar_init(&lempty[i], 128);
       mbar_init(&mfull[i], 32);
       mbar_init(&mempty[i], 2);          // both gather warps
@@ -680,25 +685,47 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     }
   } else if (wgid <= 2) {
     // ------------------------------------------- softmax (two warpgroups)
+    // Both warpgroups work on every tile: warpgroup wg takes the 64 columns
+    // [64 wg, 64 wg + 64) of each row (a warp reaches its quarter's 32 TMEM
+    // lanes), which halves a tile's softmax latency, the link of the
+    // S -> softmax -> PV chain that paces the kernel.  The two halves'
+    // row maxima meet in shared memory (a named barrier over both
+    // warpgroups, which also orders every S load before any P store over
+    // those columns), and the partial row sums go to the epilogue, which adds
+    // them and normalises.
     regs_inc<176>();
-    const int wg = wgid - 1;                 // takes tiles i with i % 2 == wg
+    const int wg = wgid - 1;
     const int quarter = warp & 3;
     const int row = quarter * 32 + lane;
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
     const uint32_t sbase = tS + lane_off;
     const int tok = row / p.r, head = row % p.r;
-    for (long long i = wg; i < n; i += 2) {
-      const long long ti = t_begin + i;
-      const int2 cs = *reinterpret_cast<const int2*>(&p.w.tiles[ti]);   // column, entry start
+    const uint64_t sc2 = f2_pack(p.scale_log2, p.scale_log2);
+    // the next tile's descriptor and entry are loaded one tile ahead: their
+    // latency would otherwise sit between S and the mask of every tile
+    int2 cs_next = make_int2(0, 0);
+    uint32_t e_next = 0xFFFFFFFFu;
+    if (n > 0) {
+      cs_next = *reinterpret_cast<const int2*>(&p.w.tiles[t_begin]);
+      e_next = tok < tpt ? p.w.tile_ent[t_begin * tpt + tok] : 0xFFFFFFFFu;
+    }
+    for (long long i = 0; i < n; ++i) {
+      const int2 cs = cs_next;   // column, entry start
+      const uint32_t e = e_next;
+      if (i + 1 < n) {
+        const long long tn = t_begin + i + 1;
+        cs_next = *reinterpret_cast<const int2*>(&p.w.tiles[tn]);
+        e_next = tok < tpt ? p.w.tile_ent[tn * tpt + tok] : 0xFFFFFFFFu;
+      }
       const int col = cs.x;
-      const uint32_t e = tok < tpt ? p.w.tile_ent[ti * tpt + tok] : 0xFFFFFFFFu;
       const int sb = static_cast<int>(i % kNS);
+      const int par = static_cast<int>(i & 1);
       const uint32_t sbuf = sbase + sb * 128;
       if (!mbar_wait(&sfull[sb], (i / kNS) & 1, abort_flag, p.err)) break;
       tc_fence_after();
-      float sv[128];
-#pragma unroll
-      for (int c = 0; c < 4; ++c) tmem_ld32(sbuf + c * 32, sv + c * 32);
+      float sv[64];
+      tmem_ld32(sbuf + wg * 64, sv);
+      tmem_ld32(sbuf + wg * 64 + 32, sv + 32);
       const int blk = col - (col / p.nb) * p.nb;
       const bool valid = e != 0xFFFFFFFFu;
       int lim = 127;
@@ -714,51 +741,69 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       const bool full = __all_sync(0xffffffffu, lim == 127);
       if (!full) {
 #pragma unroll
-        for (int x = 0; x < 128; ++x) sv[x] = x <= lim ? sv[x] : -INFINITY;
+        for (int x = 0; x < 64; ++x) sv[x] = wg * 64 + x <= lim ? sv[x] : -INFINITY;
       }
+      // half-row max with three-input max: eight chains of eight values
       float m8[8];
 #pragma unroll
-      for (int x = 0; x < 8; ++x) m8[x] = sv[x];
+      for (int x = 0; x < 8; ++x) m8[x] = fmax3(sv[x], sv[x + 8], sv[x + 16]);
 #pragma unroll
-      for (int x = 8; x < 128; ++x) m8[x & 7] = fmaxf(m8[x & 7], sv[x]);
-      const float mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
-                             fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
+      for (int b = 24; b < 56; b += 16)
+#pragma unroll
+        for (int x = 0; x < 8; ++x) m8[x] = fmax3(m8[x], sv[b + x], sv[b + 8 + x]);
+#pragma unroll
+      for (int x = 0; x < 8; ++x) m8[x] = fmaxf(m8[x], sv[56 + x]);
+      const float mloc = fmaxf(fmax3(m8[0], m8[1], m8[2]),
+                               fmax3(fmax3(m8[3], m8[4], m8[5]), m8[6], m8[7]));
+      xmax[(par * 2 + wg) * 128 + row] = mloc;
+      named_bar_sync(2, 256);
+      const float mx = fmaxf(mloc, xmax[(par * 2 + (wg ^ 1)) * 128 + row]);
       const float mxs = mx * p.scale_log2;
-      // P = 2^(s*scale - max) as bf16, written over the S columns; l sums the
-      // rounded values the PV product uses
-      float l8[8];
+      // P = 2^(s*scale - max) as bf16, written over the S columns (keys
+      // 64 wg .. 64 wg + 63 are packed columns 32 wg .. 32 wg + 31); the sum
+      // is of the rounded values the PV product uses, so that the partial
+      // output is an exact convex combination of V rows before its own
+      // rounding.  Scale-and-shift and the sums run on packed fp32 pairs.
+      const uint64_t nm2 = f2_pack(-mxs, -mxs);
+      uint64_t l4[4];
 #pragma unroll
-      for (int x = 0; x < 8; ++x) l8[x] = 0.f;
+      for (int x = 0; x < 4; ++x) l4[x] = 0ull;
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
+      for (int c = 0; c < 2; ++c) {
         uint32_t pk[16];
 #pragma unroll
         for (int x = 0; x < 32; x += 2) {
-          const float e0 = fast_exp2(fmaf(sv[c * 32 + x], p.scale_log2, -mxs));
-          const float e1 = fast_exp2(fmaf(sv[c * 32 + x + 1], p.scale_log2, -mxs));
+          const float2 a = f2_unpack(ffma2(f2_pack(sv[c * 32 + x], sv[c * 32 + x + 1]), sc2, nm2));
+          const float e0 = fast_exp2(a.x);
+          const float e1 = fast_exp2(a.y);
           __nv_bfloat162 h2 = __floats2bfloat162_rn(e0, e1);
           const uint32_t w = *reinterpret_cast<uint32_t*>(&h2);
           pk[x >> 1] = w;
-          l8[(x >> 1) & 7] += __uint_as_float(w << 16) + __uint_as_float(w & 0xFFFF0000u);
+          // the pair widened exactly (bf16 is the top half of an fp32)
+          l4[(x >> 1) & 3] = fadd2(l4[(x >> 1) & 3],
+                                   f2_pack(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u)));
         }
-        tmem_st16(sbuf + c * 16, pk);
+        tmem_st16(sbuf + wg * 32 + c * 16, pk);
       }
-      const float l = ((l8[0] + l8[1]) + (l8[2] + l8[3])) + ((l8[4] + l8[5]) + (l8[6] + l8[7]));
+      const float2 la = f2_unpack(fadd2(fadd2(l4[0], l4[1]), fadd2(l4[2], l4[3])));
+      const float lpart = la.x + la.y;
       tc_wait_st();
       tc_fence_before();
       mbar_arrive(&pfull[sb]);
-      if (valid) reinterpret_cast<float2*>(p.w.part_ml)[prow] = make_float2(mxs, l);
-      // 1/l for the epilogue of this tile
-      if (!mbar_wait(&lempty[wg], ((i >> 1) & 1) ^ 1, abort_flag, p.err)) break;
-      linv[wg * 128 + row] = 1.f / l;
-      mbar_arrive(&lfull[wg]);
+      if (valid && wg == 0) p.w.part_ml[2 * prow] = mxs;
+      // the partial sum for the epilogue of this tile
+      if (!mbar_wait(&lempty[par], ((i >> 1) & 1) ^ 1, abort_flag, p.err)) break;
+      xsum[(par * 2 + wg) * 128 + row] = lpart;
+      mbar_arrive(&lfull[par]);
     }
   } else {
     // ------------------------------------------------------------- epilogue
-    // O row (scaled by 1/l, bf16) -> swizzled staging tile -> TMA stores.
-    // Partials are stored in entry order, so the 128 rows of a full tile are
-    // one contiguous block: one store per 64-column half.  The last, partial
-    // tile of a column stores its tokens' r rows one token at a time.
+    // O row (scaled by 1/l, bf16) -> swizzled staging tile -> TMA stores, one
+    // 64-column half of the rows at a time.  Partials are stored in entry
+    // order, so the 128 rows of a full tile are one contiguous block: one
+    // store per half.  The last, partial tile of a column stores its tokens'
+    // r rows one token at a time.  l is the sum of the two softmax
+    // warpgroups' partial sums.
     regs_dec<96>();
     const int quarter = warp & 3;
     const int row = quarter * 32 + lane;
@@ -767,60 +812,64 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     uint8_t* stage = smem + L::kOffStage;
     uint8_t* srow = stage + row * 128;
     bool stored = false;   // this thread has bulk stores in flight
+    int4 td_next = n > 0 ? p.w.tiles[t_begin] : make_int4(0, 0, 0, 0);   // one tile ahead
     for (long long i = 0; i < n; ++i) {
-      const long long ti = t_begin + i;
-      const int4 td = p.w.tiles[ti];   // column, entry start, entries
+      const int4 td = td_next;   // column, entry start, entries
+      if (i + 1 < n) td_next = p.w.tiles[t_begin + i + 1];
       const int ob = static_cast<int>(i % kNO);
-      const int lb = static_cast<int>(i & 1);   // softmax warpgroup of this tile
+      const int par = static_cast<int>(i & 1);
       if (!mbar_wait(&ofull[ob], (i / kNO) & 1, abort_flag, p.err)) break;
-      if (!mbar_wait(&lfull[lb], (i >> 1) & 1, abort_flag, p.err)) break;
+      if (!mbar_wait(&lfull[par], (i >> 1) & 1, abort_flag, p.err)) break;
       tc_fence_after();
-      const float il = linv[lb * 128 + row];
-      mbar_arrive(&lempty[lb]);
-      // the staging tile must be free: own stores read out, then everyone's
-      if (stored) {
-        bulk_wait_read0();
-        stored = false;
-      }
-      named_bar_sync(1, 128);
+      const float l = xsum[(par * 2) * 128 + row] + xsum[(par * 2 + 1) * 128 + row];
+      mbar_arrive(&lempty[par]);
+      if (tok < td.z) p.w.part_ml[2 * ((static_cast<long long>(td.y) + tok) * p.r + head) + 1] = l;
+      const float il = 1.f / l;
+      const uint64_t il2 = f2_pack(il, il);
 #pragma unroll
-      for (int c = 0; c < D / 32; c += 2) {
+      for (int h = 0; h < D / 64; ++h) {
+        // the staging tile must be free: own stores read out, then everyone's
+        if (stored) {
+          bulk_wait_read0();
+          stored = false;
+        }
+        named_bar_sync(1, 128);
         float ov[64];
-        tmem_ld32(tO + ob * D + lane_off + c * 32, ov);
-        tmem_ld32(tO + ob * D + lane_off + c * 32 + 32, ov + 32);
+        tmem_ld32(tO + ob * D + lane_off + h * 64, ov);
+        tmem_ld32(tO + ob * D + lane_off + h * 64 + 32, ov + 32);
         tc_wait_ld();
-        if (c + 2 >= D / 32) {
+        if (h + 1 == D / 64) {
           tc_fence_before();
           mbar_arrive(&ofree[ob]);
         }
 #pragma unroll
         for (int x = 0; x < 8; ++x) {
-          __nv_bfloat162 h0 = __floats2bfloat162_rn(ov[8 * x] * il, ov[8 * x + 1] * il);
-          __nv_bfloat162 h1 = __floats2bfloat162_rn(ov[8 * x + 2] * il, ov[8 * x + 3] * il);
-          __nv_bfloat162 h2 = __floats2bfloat162_rn(ov[8 * x + 4] * il, ov[8 * x + 5] * il);
-          __nv_bfloat162 h3 = __floats2bfloat162_rn(ov[8 * x + 6] * il, ov[8 * x + 7] * il);
-          const int u = (c * 32 + 8 * x) >> 3;            // 16-byte unit of the row
-          uint4* dst = reinterpret_cast<uint4*>(srow + (u >> 3) * 16384 +
-                                                (((u & 7) ^ (row & 7)) << 4));
+          // scale by 1/l on packed pairs, then round to bf16
+          float2 q[4];
+#pragma unroll
+          for (int y = 0; y < 4; ++y)
+            q[y] = f2_unpack(fmul2(f2_pack(ov[8 * x + 2 * y], ov[8 * x + 2 * y + 1]), il2));
+          __nv_bfloat162 h0 = __floats2bfloat162_rn(q[0].x, q[0].y);
+          __nv_bfloat162 h1 = __floats2bfloat162_rn(q[1].x, q[1].y);
+          __nv_bfloat162 h2 = __floats2bfloat162_rn(q[2].x, q[2].y);
+          __nv_bfloat162 h3 = __floats2bfloat162_rn(q[3].x, q[3].y);
+          uint4* dst = reinterpret_cast<uint4*>(srow + ((x ^ (row & 7)) << 4));
           *dst = make_uint4(*reinterpret_cast<uint32_t*>(&h0), *reinterpret_cast<uint32_t*>(&h1),
                             *reinterpret_cast<uint32_t*>(&h2), *reinterpret_cast<uint32_t*>(&h3));
         }
-      }
-      fence_proxy_async_smem();
-      named_bar_sync(1, 128);
-      if (td.z == tpt) {
-        if (row == 0) {
-#pragma unroll
-          for (int c = 0; c < D / 64; ++c) tma_store_2d(&tm_ot, stage + c * 16384, c * 64, td.y * p.r);
+        fence_proxy_async_smem();
+        named_bar_sync(1, 128);
+        if (td.z == tpt) {
+          if (row == 0) {
+            tma_store_2d(&tm_ot, stage, h * 64, td.y * p.r);
+            bulk_commit_group();
+            stored = true;
+          }
+        } else if (head == 0 && tok < td.z) {
+          tma_store_2d(&tm_o, stage + tok * p.r * 128, h * 64, (td.y + tok) * p.r);
           bulk_commit_group();
           stored = true;
         }
-      } else if (head == 0 && tok < td.z) {
-#pragma unroll
-        for (int c = 0; c < D / 64; ++c)
-          tma_store_2d(&tm_o, stage + c * 16384 + tok * p.r * 128, c * 64, (td.y + tok) * p.r);
-        bulk_commit_group();
-        stored = true;
       }
     }
     if (stored) bulk_wait0();

@@ -229,6 +229,39 @@ def test_forward_tiny(tiny_inputs, tiny_oracle):
     check_attn(o[0], O_ref, "forward tiny")
 
 
+@pytest.mark.parametrize("sp,mode", [
+    (spec(1, 700, 4000, 3300, 16, 8, 64, 64, 16, seed=71), "ties"),     # G = 8, index values in {-1, 0, 1}
+    (spec(1, 300, 3001, 2701, 8, 1, 64, 32, 17, seed=72), "ties"),     # G = 1: a row tile spans a block edge; k = 17
+    (spec(2, 260, 5000, 4740, 16, 4, 64, 64, 32, seed=73), "random"),  # k = 32, the longest fused list
+    (spec(1, 400, 3000, 2600, 16, 8, 64, 64, 16, seed=74), "equal"),   # every score equal
+    (spec(1, 600, 600, 0, 16, 8, 128, 64, 16, seed=75), "random"),     # rows with fewer than k causal blocks
+])
+def test_forward_fused_topk(sp, mode):
+    """The prefill forward selects blocks inside the index-score kernel (no
+    pooled scores in memory).  Its selection must equal, bit for bit, the
+    oracle's and the standalone msa_index_scores + msa_block_topk pipeline's,
+    tie order included."""
+    inp = inputs_cpu(sp)
+    if mode == "ties":
+        inp.q_idx = inp.q_idx.float().clamp(-1, 1).to(torch.bfloat16)
+        inp.k_idx = inp.k_idx.float().clamp(-1, 1).to(torch.bfloat16)
+    elif mode == "equal":
+        inp.q_idx = torch.zeros_like(inp.q_idx)
+    sh = M.Shape.of(sp)
+    assert M.workspace_size(sh, M.OP_FORWARD) < M.workspace_size(sh, M.OP_FORWARD_ALIGNMENT)
+    qi, ki = cuda(inp.q_idx), cuda(inp.k_idx)
+    o, lse, sel = M.forward(sh, cuda(inp.q), cuda(inp.k), cuda(inp.v), qi, ki)
+    sel_two = M.block_topk(sh, M.index_scores(sh, qi, ki))
+    torch.cuda.synchronize()
+    assert M.device_status() == 0
+    assert torch.equal(sel, sel_two), "fused and two-kernel selections differ"
+    for b in range(sp.batch):
+        sref = oracle_sel(sp, oracle_pooled(sp, inp, b))
+        assert np.array_equal(sel[b].cpu().numpy(), sref), f"selection b={b}"
+    O_ref, _ = oracle_attention(sp, inp, oracle_sel(sp, oracle_pooled(sp, inp, 0)), 0)
+    check_attn(o[0], O_ref, "fused top-k forward")
+
+
 def test_forward_decode():
     sp = spec(4, 1, 20000, 19999, 16, 2, 128, 64, 16, seed=41, planted=4)
     inp = inputs_cpu(sp)
