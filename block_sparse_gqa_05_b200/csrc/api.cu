@@ -517,6 +517,17 @@ msa_status msa_profile_read(int index, const char** name, double* total_ms, long
   return MSA_OK;
 }
 
+msa_status msa_set_wait_limit_ns(uint64_t ns) {
+  if (!device_ctx()) return MSA_ERR_CUDA;
+  // no kernel of the library is running when the limit changes
+  cudaError_t e = cudaDeviceSynchronize();
+  if (e == cudaSuccess) e = set_wait_limit_decode(ns);
+  if (e == cudaSuccess) e = set_wait_limit_dense(ns);
+  if (e == cudaSuccess) e = set_wait_limit_index(ns);
+  if (e == cudaSuccess) e = set_wait_limit_prefill(ns);
+  return from_cuda(e);
+}
+
 msa_status msa_device_status(uint32_t* flags) {
   const DevCtx* c = device_ctx();
   if (!c) return MSA_ERR_CUDA;

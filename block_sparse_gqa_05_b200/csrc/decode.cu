@@ -221,7 +221,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t ph = (x / S) & 1;
         const uint64_t t0 = globaltimer();
         while (!(mbar_test(&kfull[s], ph) && mbar_test(&vfull[s], ph)))
-          if (globaltimer() - t0 > kWaitLimitNs) {
+          if (globaltimer() - t0 > kDrainLimitNs) {
             atomicOr(p.err, kErrTimeout);
             break;
           }
@@ -682,3 +682,7 @@ extern "C" msa_status msa_sparse_attn_decode_static(const msa_shape* s, const ui
                                            static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? MSA_OK : MSA_ERR_CUDA;
 }
+
+namespace msa {
+cudaError_t set_wait_limit_decode(uint64_t ns) { return set_wait_limit_here(ns); }
+}  // namespace msa

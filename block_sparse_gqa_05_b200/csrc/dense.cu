@@ -62,7 +62,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* sfull = bars + 5;      // [2]
   uint64_t* pfull = bars + 7;      // [2]
   uint64_t* pvdone = bars + 9;     // [1] one arrival per PV
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 10);
+  uint64_t* mma_drain = bars + 10; // [1] the MMA thread's last commit before exit
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 11);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -83,6 +84,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&pfull[i], 128);
     }
     mbar_init(pvdone, 1);
+    mbar_init(mma_drain, 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -111,10 +113,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int c = 0; c < D / 64; ++c)
           tma_load_2d(smem + L::kOffQ + c * 16384 + j * p.r * 128, &tm_q, qfull, c * 64, row);
       }
+      int armed = 0;   // K/V blocks whose loads were issued
       for (int j = 0; j < nblk; ++j) {
         const int st = j & 1;
         if (!mbar_wait(&kvempty[st], ((j >> 1) & 1) ^ 1, abort_flag, p.err)) break;
         mbar_arrive_expect_tx(&kvfull[st], 2 * L::kTile);
+        ++armed;
 #pragma unroll
         for (int c = 0; c < D / 64; ++c) {
           tma_load_3d(smem + L::kOffK + st * L::kTile + c * 16384, &tm_k, &kvfull[st], c * 64,
@@ -123,6 +127,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                       j * 128, bg);
         }
       }
+      // every load issued lands before the CTA may exit
+      mbar_drain(qfull, 0);
+      for (int j = armed > 2 ? armed - 2 : 0; j < armed; ++j) mbar_drain(&kvfull[j & 1], (j >> 1) & 1);
     }
     __syncwarp();
   } else if (warp == 1) {
@@ -162,6 +169,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_commit(&kvempty[st]);
         if (j + 2 < nblk && !(ok = issue_s(j + 2))) break;
       }
+      // every MMA issued completes before TMEM is released
+      tc_drain(mma_drain, 0);
     }
     __syncwarp();
   } else {
@@ -332,4 +341,8 @@ cudaError_t launch_dense_prefill(const msa_shape& s, const uint16_t* q, const ui
                            : launch<64>(s, q, k, v, o, lse, ctx, st);
 }
 
+}  // namespace msa
+
+namespace msa {
+cudaError_t set_wait_limit_dense(uint64_t ns) { return set_wait_limit_here(ns); }
 }  // namespace msa

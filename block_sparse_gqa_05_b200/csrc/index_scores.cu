@@ -32,7 +32,7 @@ constexpr int kChunkBlocks = 32; // key blocks per work item
 constexpr int kRing = 8;         // fused top-k: ring slots of one 256-key tile's two block maxima
 // barriers (K stages, Q, accumulators, ring), the TMEM address and the abort
 // flag, rounded up; the fused top-k ring follows them
-constexpr uint32_t kBarBytes = ((2 * kStages + 4 + 2 * kAcc + 2 * kRing) * 8 + 8 + 127) / 128 * 128;
+constexpr uint32_t kBarBytes = ((2 * kStages + 4 + 2 * kAcc + 2 * kRing + 1) * 8 + 8 + 127) / 128 * 128;
 
 struct IdxParams {
   float* pooled;
@@ -141,7 +141,8 @@ __global__ void __launch_bounds__(kThreads + (KMAX > 0 ? kTopkThreads : 0), 1)
   uint64_t* accempty = accfull + kAcc;
   uint64_t* ring_full = accempty + kAcc;     // fused top-k: [kRing] block maxima written
   uint64_t* ring_empty = ring_full + kRing;  // fused top-k: [kRing] block maxima consumed
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(ring_empty + kRing);
+  uint64_t* mma_drain = ring_empty + kRing;  // the MMA thread's last commit before exit
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   // fused top-k: [kRing][2 blocks][128 rows] block maxima, after the barriers
   float* ring = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(bars) + kBarBytes);
@@ -168,6 +169,7 @@ __global__ void __launch_bounds__(kThreads + (KMAX > 0 ? kTopkThreads : 0), 1)
         mbar_init(&ring_empty[i], kTopkThreads);
       }
     }
+    mbar_init(mma_drain, 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -191,22 +193,28 @@ __global__ void __launch_bounds__(kThreads + (KMAX > 0 ? kTopkThreads : 0), 1)
       tma_prefetch_desc(&tm_q);
       tma_prefetch_desc(&tm_k);
       ItemCursor cur;
-      long long j = 0, q = 0;
+      long long j = 0, q = 0;   // K tiles and query tiles whose loads were issued
       bool ok = true;
-      for (long long w = blockIdx.x; ok && w < p.items_total; w += gridDim.x, ++q) {
+      for (long long w = blockIdx.x; ok && w < p.items_total; w += gridDim.x) {
         int seq, m, b0, b1;
         item_decode(p, w, cur, seq, m, b0, b1);
         const int qb = static_cast<int>(q & 1);
         if (!(ok = mbar_wait(&qempty[qb], ((q >> 1) & 1) ^ 1, abort_flag, p.err))) break;
         mbar_arrive_expect_tx(&qfull[qb], kQTile);
         tma_load_2d(qbuf + qb * kQTile, &tm_q, &qfull[qb], 0, seq * p.T * p.G + m * 128);
-        for (int b = b0; b < b1; b += 2, ++j) {
+        ++q;
+        for (int b = b0; b < b1; b += 2) {
           const int s = static_cast<int>(j % kStages);
           if (!(ok = mbar_wait(&kempty[s], ((j / kStages) & 1) ^ 1, abort_flag, p.err))) break;
           mbar_arrive_expect_tx(&kfull[s], kKTile);
           tma_load_2d(kbuf + s * kKTile, &tm_k, &kfull[s], 0, seq * p.N + b * 128);
+          ++j;
         }
       }
+      // every load issued lands before the CTA may exit
+      for (long long t = q > 2 ? q - 2 : 0; t < q; ++t) mbar_drain(&qfull[t & 1], (t >> 1) & 1);
+      for (long long t = j > kStages ? j - kStages : 0; t < j; ++t)
+        mbar_drain(&kfull[t % kStages], (t / kStages) & 1);
     }
     __syncwarp();
   } else if (warp == 1) {
@@ -239,6 +247,8 @@ __global__ void __launch_bounds__(kThreads + (KMAX > 0 ? kTopkThreads : 0), 1)
         }
         if (ok) tc_commit(&qempty[qb]);
       }
+      // every MMA issued completes before TMEM is released
+      tc_drain(mma_drain, 0);
     }
     __syncwarp();
   }
@@ -654,4 +664,8 @@ cudaError_t launch_index_topk(const msa_shape& s, const uint16_t* q_idx, const u
                            : launch_tc<32, 32>(s, q_idx, k_idx, nullptr, sel, ctx, st);
 }
 
+}  // namespace msa
+
+namespace msa {
+cudaError_t set_wait_limit_index(uint64_t ns) { return set_wait_limit_here(ns); }
 }  // namespace msa

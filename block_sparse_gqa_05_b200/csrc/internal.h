@@ -87,6 +87,12 @@ cudaError_t launch_decode(const msa_shape& s, const uint16_t* q, const uint16_t*
 msa_status check_decode_static_args(const msa_shape* s, const uint16_t* q, const uint16_t* k,
                                     const uint16_t* v, const int32_t* sel, const uint16_t* o,
                                     const float* lse);
+// The bounded waits' limit of each kernel translation unit, on the current
+// device (msa_set_wait_limit_ns).
+cudaError_t set_wait_limit_decode(uint64_t ns);
+cudaError_t set_wait_limit_dense(uint64_t ns);
+cudaError_t set_wait_limit_index(uint64_t ns);
+cudaError_t set_wait_limit_prefill(uint64_t ns);
 cudaError_t launch_dense_prefill(const msa_shape& s, const uint16_t* q, const uint16_t* k,
                                  const uint16_t* v, uint16_t* o, float* lse, cudaStream_t st);
 

@@ -312,7 +312,7 @@ struct AttnSmem {
   static constexpr uint32_t kOffBar = kOffTrow + kTentWords * 4;
   // barriers: K 2+2, V kNV+kNV, Q kNQ+kNQ, S/P kNS+kNS, O 2+2, row sums 2+2,
   // metadata 2+2; then the TMEM address and the abort flag
-  static constexpr uint32_t kNBars = 4 + 2 * kNV + 2 * kNQ + 2 * kNS + 12;
+  static constexpr uint32_t kNBars = 4 + 2 * kNV + 2 * kNQ + 2 * kNS + 12 + 1;   // + MMA drain
   static constexpr uint32_t kBytes = kOffBar + kNBars * 8 + 8;
   static_assert(kBytes <= 227u * 1024u, "shared memory of one CTA");
 };
@@ -370,9 +370,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   uint64_t* lempty = lfull + 2;         // [2] by tile parity: partial row sums read
   uint64_t* mfull = lempty + 2;         // [2] metadata batch ready
   uint64_t* mempty = mfull + 2;         // [2] metadata batch consumed
+  uint64_t* mma_drain = mempty + 2;     // the MMA thread's last commit before exit
   int4* thdr = reinterpret_cast<int4*>(smem + L::kOffThdr);
   int* trow = reinterpret_cast<int*>(smem + L::kOffTrow);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mempty + 2);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -406,6 +407,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       mbar_init(&qfull[i], 2);           // both gather warps (expect_tx arrivals)
       mbar_init(&qempty[i], 1);
     }
+    mbar_init(mma_drain, 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -441,6 +443,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         uint32_t mph = 0;              // parity of that slot's barriers
         int qb = 0;                    // query buffer
         uint32_t qph = 0;              // its parity
+        long long q_armed = 0;         // query tiles this warp issued loads for (lane 0)
+        int kv_armed = 0;              // K (warp 0) or V (warp 3) columns loaded (lane 0)
         const int nx = (tpt + 63) >> 6;   // this warp's tokens per lane (<= 2)
         for (long long i = 0; i < n; ++i) {
           int ok = 1;
@@ -480,6 +484,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
               // this warp's tokens of the tile's hd.z
               const int mine = (hd.z + 1 - gw) >> 1;
               mbar_arrive_expect_tx(&qfull[qb], static_cast<uint32_t>(mine * p.r * D * 2));
+              ++q_armed;
             }
           }
           ok = __shfl_sync(0xffffffffu, ok, 0);
@@ -510,6 +515,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 const int st = u & 1;
                 ok = mbar_wait(&kempty[st], ((u >> 1) & 1) ^ 1, abort_flag, p.err) ? 1 : 0;
                 if (ok) {
+                  ++kv_armed;
                   mbar_arrive_expect_tx(&kfull[st], L::kKV);
 #pragma unroll
                   for (int c = 0; c < D / 64; ++c)
@@ -520,6 +526,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 const int vs = u % kNV;
                 ok = mbar_wait(&vempty[vs], ((u / kNV) & 1) ^ 1, abort_flag, p.err) ? 1 : 0;
                 if (ok) {
+                  ++kv_armed;
                   mbar_arrive_expect_tx(&vfull[vs], L::kKV);
 #pragma unroll
                   for (int c = 0; c < D / 64; ++c)
@@ -534,6 +541,18 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           if (++qb == kNQ) {
             qb = 0;
             qph ^= 1u;
+          }
+        }
+        // every load this warp issued lands before the CTA may exit
+        if (lane == 0) {
+          for (long long t = q_armed > kNQ ? q_armed - kNQ : 0; t < q_armed; ++t)
+            mbar_drain(&qfull[t % kNQ], (t / kNQ) & 1);
+          if (gw == 0) {
+            for (int c = kv_armed > 2 ? kv_armed - 2 : 0; c < kv_armed; ++c)
+              mbar_drain(&kfull[c & 1], (c >> 1) & 1);
+          } else {
+            for (int c = kv_armed > kNV ? kv_armed - kNV : 0; c < kv_armed; ++c)
+              mbar_drain(&vfull[c % kNV], (c / kNV) & 1);
           }
         }
       }
@@ -674,12 +693,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             break;
           } else if (t_idle == 0) {
             t_idle = globaltimer();
-          } else if (globaltimer() - t_idle > kWaitLimitNs) {
+          } else if (globaltimer() - t_idle > g_wait_limit_ns) {
             atomicOr(p.err, kErrTimeout);
             *abort_flag = 1;
             break;
           }
         }
+        // every MMA issued completes before TMEM is released
+        tc_drain(mma_drain, 0);
       }
       __syncwarp();
     }
@@ -709,6 +730,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       cs_next = *reinterpret_cast<const int2*>(&p.w.tiles[t_begin]);
       e_next = tok < tpt ? p.w.tile_ent[t_begin * tpt + tok] : 0xFFFFFFFFu;
     }
+    // A role that gives up on a wait (an expired bound) must not leave its
+    // partner warpgroup in a named barrier: every exit is decided together,
+    // at the barrier, from this tile's waits and the previous tile's.
+    bool failed = false;
     for (long long i = 0; i < n; ++i) {
       const int2 cs = cs_next;   // column, entry start
       const uint32_t e = e_next;
@@ -721,11 +746,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       const int sb = static_cast<int>(i % kNS);
       const int par = static_cast<int>(i & 1);
       const uint32_t sbuf = sbase + sb * 128;
-      if (!mbar_wait(&sfull[sb], (i / kNS) & 1, abort_flag, p.err)) break;
+      const bool ok = !failed && mbar_wait(&sfull[sb], (i / kNS) & 1, abort_flag, p.err);
       tc_fence_after();
       float sv[64];
-      tmem_ld32(sbuf + wg * 64, sv);
-      tmem_ld32(sbuf + wg * 64 + 32, sv + 32);
+      if (ok) {
+        tmem_ld32(sbuf + wg * 64, sv);
+        tmem_ld32(sbuf + wg * 64 + 32, sv + 32);
+      }
       const int blk = col - (col / p.nb) * p.nb;
       const bool valid = e != 0xFFFFFFFFu;
       int lim = 127;
@@ -735,7 +762,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         const int pos = p.q_off + static_cast<int>(e >> 6);
         if ((pos >> 7) == blk) lim = pos & 127;
       }
-      tc_wait_ld();
+      if (ok) tc_wait_ld();
       // Only rows of the local block need the causal mask; the branch is
       // uniform over the warp in the common case.
       const bool full = __all_sync(0xffffffffu, lim == 127);
@@ -756,7 +783,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       const float mloc = fmaxf(fmax3(m8[0], m8[1], m8[2]),
                                fmax3(fmax3(m8[3], m8[4], m8[5]), m8[6], m8[7]));
       xmax[(par * 2 + wg) * 128 + row] = mloc;
-      named_bar_sync(2, 256);
+      if (named_bar_or(2, 256, !ok)) break;
       const float mx = fmaxf(mloc, xmax[(par * 2 + (wg ^ 1)) * 128 + row]);
       const float mxs = mx * p.scale_log2;
       // P = 2^(s*scale - max) as bf16, written over the S columns (keys
@@ -792,9 +819,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       mbar_arrive(&pfull[sb]);
       if (valid && wg == 0) p.w.part_ml[2 * prow] = mxs;
       // the partial sum for the epilogue of this tile
-      if (!mbar_wait(&lempty[par], ((i >> 1) & 1) ^ 1, abort_flag, p.err)) break;
-      xsum[(par * 2 + wg) * 128 + row] = lpart;
-      mbar_arrive(&lfull[par]);
+      if (mbar_wait(&lempty[par], ((i >> 1) & 1) ^ 1, abort_flag, p.err)) {
+        xsum[(par * 2 + wg) * 128 + row] = lpart;
+        mbar_arrive(&lfull[par]);
+      } else {
+        failed = true;
+      }
     }
   } else {
     // ------------------------------------------------------------- epilogue
@@ -818,8 +848,15 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       if (i + 1 < n) td_next = p.w.tiles[t_begin + i + 1];
       const int ob = static_cast<int>(i % kNO);
       const int par = static_cast<int>(i & 1);
-      if (!mbar_wait(&ofull[ob], (i / kNO) & 1, abort_flag, p.err)) break;
-      if (!mbar_wait(&lfull[par], (i >> 1) & 1, abort_flag, p.err)) break;
+      const bool ok = mbar_wait(&ofull[ob], (i / kNO) & 1, abort_flag, p.err) &&
+                      mbar_wait(&lfull[par], (i >> 1) & 1, abort_flag, p.err);
+      // the staging tile must be free: own stores read out, then everyone's;
+      // and the four warps leave together if a wait gave up
+      if (stored) {
+        bulk_wait_read0();
+        stored = false;
+      }
+      if (named_bar_or(1, 128, !ok)) break;
       tc_fence_after();
       const float l = xsum[(par * 2) * 128 + row] + xsum[(par * 2 + 1) * 128 + row];
       mbar_arrive(&lempty[par]);
@@ -828,12 +865,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       const uint64_t il2 = f2_pack(il, il);
 #pragma unroll
       for (int h = 0; h < D / 64; ++h) {
-        // the staging tile must be free: own stores read out, then everyone's
-        if (stored) {
-          bulk_wait_read0();
-          stored = false;
+        if (h > 0) {
+          // the staging tile must be free: own stores read out, then everyone's
+          if (stored) {
+            bulk_wait_read0();
+            stored = false;
+          }
+          named_bar_sync(1, 128);
         }
-        named_bar_sync(1, 128);
         float ov[64];
         tmem_ld32(tO + ob * D + lane_off + h * 64, ov);
         tmem_ld32(tO + ob * D + lane_off + h * 64 + 32, ov + 32);
@@ -1168,4 +1207,8 @@ cudaError_t launch_sparse_prefill(const msa_shape& s, const uint16_t* q, const u
   return cudaGetLastError();
 }
 
+}  // namespace msa
+
+namespace msa {
+cudaError_t set_wait_limit_prefill(uint64_t ns) { return set_wait_limit_here(ns); }
 }  // namespace msa

@@ -17,8 +17,22 @@ constexpr uint32_t kErrTimeout = 1u;
 constexpr uint32_t kErrBadLength = 2u;   // a ragged-decode cache length outside [1, N]
 constexpr uint32_t kErrBadPage = 4u;     // a page-table entry outside [0, num_pages)
 constexpr uint32_t kErrBadSel = 8u;      // a prefill selection entry past its query's block
-// Bound of every mbarrier wait, in nanoseconds of %globaltimer.
+// Default bound of the bounded waits, in nanoseconds of %globaltimer.
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
+// Fixed bound of the drains a role runs before its CTA exits (loads already
+// in flight landing): independent of the settable limit below, so that a
+// drain still ends cleanly when a small limit made the kernel abort.
+constexpr uint64_t kDrainLimitNs = 2000000000ull;
+
+// The bound the waits use: one copy per translation unit and device, set
+// by msa_set_wait_limit_ns (diagnostics).  0 makes every wait that is not
+// complete at its first probe expire at once.
+static __device__ uint64_t g_wait_limit_ns = kWaitLimitNs;
+
+// Sets this translation unit's copy on the current device.
+static inline cudaError_t set_wait_limit_here(uint64_t ns) {
+  return cudaMemcpyToSymbol(g_wait_limit_ns, &ns, sizeof(ns));
+}
 
 MSA_DEV uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -96,21 +110,31 @@ MSA_DEV bool mbar_test(uint64_t* bar, uint32_t phase) {
 }
 
 // Bounded wait for the completion of phase ``phase`` (parity).  Gives up after
-// kWaitLimitNs or as soon as *abort is set by another role of the CTA; on a
-// timeout it sets the device error word and *abort.  Returns false when the
+// g_wait_limit_ns or as soon as *abort is set by another role of the CTA; on
+// a timeout it sets the device error word and *abort.  Returns false when the
 // caller must stop.
 MSA_DEV bool mbar_wait(uint64_t* bar, uint32_t phase, volatile int* abort, uint32_t* err) {
-  if (mbar_try_wait(bar, phase)) return true;
+  const uint64_t lim = g_wait_limit_ns;
+  if (lim == 0 ? mbar_test(bar, phase) : mbar_try_wait(bar, phase)) return true;
   const uint64_t t0 = globaltimer();
   for (uint32_t it = 0;; ++it) {
-    if (mbar_try_wait(bar, phase)) return true;
-    if (*abort) return false;
-    if ((it & 63u) == 63u && globaltimer() - t0 > kWaitLimitNs) {
+    if (lim == 0 || ((it & 63u) == 63u && globaltimer() - t0 > lim)) {
       atomicOr(err, kErrTimeout);
       *abort = 1;
       return false;
     }
+    if (mbar_try_wait(bar, phase)) return true;
+    if (*abort) return false;
   }
+}
+
+// Waits, bounded by kDrainLimitNs, until phase ``parity`` of *bar has
+// completed: the drain a role runs before its CTA exits, so that no load it
+// issued (or MMA, through a final commit) is still in flight then.
+MSA_DEV void mbar_drain(uint64_t* bar, uint32_t parity) {
+  const uint64_t t0 = globaltimer();
+  while (!mbar_test(bar, parity))
+    if (globaltimer() - t0 > kDrainLimitNs) break;
 }
 
 // ----------------------------------------------------------------------- TMA
@@ -148,22 +172,6 @@ MSA_DEV void bulk_commit_group() { asm volatile("cp.async.bulk.commit_group;" ::
 MSA_DEV void bulk_wait_read0() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
 // Wait until every committed bulk store of this thread has completed.
 MSA_DEV void bulk_wait0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
-
-// ------------------------------------------------------------- cp.async
-// 16-byte copy global -> shared through L2 only (no L1 allocation).
-MSA_DEV void cp_async16(void* smem_dst, const void* gmem_src) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;"
-               ::"r"(smem_u32(smem_dst)), "l"(gmem_src)
-               : "memory");
-}
-// The barrier's current phase cannot complete before every cp.async this
-// thread issued so far has landed (its pending count is raised now and
-// lowered when they land); the thread still makes its own counted arrival.
-MSA_DEV void cp_async_mbar_track(uint64_t* bar) {
-  asm volatile("cp.async.mbarrier.arrive.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
-}
-// Wait until every cp.async of this thread has landed.
-MSA_DEV void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 
 // Named barrier over ``count`` threads (id 0 is __syncthreads).
 MSA_DEV void named_bar_sync(uint32_t id, uint32_t count) {
@@ -273,6 +281,13 @@ MSA_DEV void tc_commit(uint64_t* bar) {
       "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];"
       ::"r"(smem_u32(bar))
       : "memory");
+}
+
+// Every tcgen05 operation this thread issued has completed (bounded): a
+// commit to a barrier used for nothing else, phase ``parity``.
+MSA_DEV void tc_drain(uint64_t* bar, uint32_t parity) {
+  tc_commit(bar);
+  mbar_drain(bar, parity);
 }
 
 MSA_DEV void tc_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }

@@ -74,6 +74,7 @@ _SIGS = {
     "msa_dense_attn_decode": ([ctypes.POINTER(Shape), _vp, _vp, _vp, _vp, _vp, _vp,
                                ctypes.c_size_t, _vp], ctypes.c_int),
     "msa_device_status": ([ctypes.POINTER(ctypes.c_uint32)], ctypes.c_int),
+    "msa_set_wait_limit_ns": ([ctypes.c_uint64], ctypes.c_int),
     "msa_profile_enable": ([ctypes.c_int], ctypes.c_int),
     "msa_profile_read": ([ctypes.c_int, ctypes.POINTER(ctypes.c_char_p),
                           ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_longlong)],
@@ -362,3 +363,10 @@ def device_status() -> int:
     if st not in (0, 7):
         raise MsaError(st, "msa_device_status")
     return int(f.value)
+
+
+def set_wait_limit_ns(ns: int) -> None:
+    """Bound of the kernels' waits on the current device, in nanoseconds
+    (diagnostics; default 2 s; 0 makes every wait that is not already complete
+    expire at once)."""
+    _check(lib().msa_set_wait_limit_ns(int(ns)), "msa_set_wait_limit_ns")

@@ -286,6 +286,18 @@ msa_status msa_sparse_attn_decode_static(const msa_shape* shape, const uint16_t*
  * otherwise; *flags (may be NULL) receives the raw word. */
 msa_status msa_device_status(uint32_t* flags);
 
+/* Sets the bound of the kernels' waits on the current device, in nanoseconds
+ * (diagnostics; no counterpart on the pages; the default is 2 s).  A wait
+ * that runs past it sets bit 0 of the device error word, and its kernel stops
+ * its roles, lets the loads already in flight land and returns.  0 makes every
+ * wait that is not complete at its first probe expire at once, so any call
+ * that has to wait for a load aborts: the way tests exercise the expiry path.
+ * Results of an aborted call are undefined.  Applies to every later launch on
+ * the device from any stream; a process-wide setting, not per call.
+ * Synchronises the device.  Returns MSA_ERR_CUDA if the device cannot be
+ * reached. */
+msa_status msa_set_wait_limit_ns(uint64_t ns);
+
 /* Per-kernel timing with CUDA events (diagnostics; no counterpart on the
  * pages).  msa_profile_enable(1) clears the table and brackets every later
  * kernel launch of the library with a pair of events recorded on the launch
