@@ -84,6 +84,11 @@ size_t forward_pooled_bytes(const msa_shape& s) {
   return !forward_is_decode(s) && index_topk_fusable(s) ? 0 : pooled_bytes(s);
 }
 
+// The same for the paged chunked prefill (always the prefill path).
+size_t paged_prefill_pooled_bytes(const msa_shape& s) {
+  return index_topk_fusable(s, true) ? 0 : pooled_bytes(s);
+}
+
 msa_status from_cuda(cudaError_t e) { return e == cudaSuccess ? MSA_OK : MSA_ERR_CUDA; }
 
 // ------------------------------------------------------------- profiling
@@ -251,6 +256,11 @@ msa_status msa_workspace_size(const msa_shape* s, msa_op op, size_t* bytes) {
       if ((st = check_shape(s, true, true)) != MSA_OK) return st;
       if (!prefill_shape_supported(*s)) return MSA_ERR_UNSUPPORTED;
       *bytes = pooled_bytes(*s) + sel_bytes(*s) + prefill_workspace_bytes(*s);
+      return MSA_OK;
+    case MSA_OP_FORWARD_PREFILL_PAGED:
+      if ((st = check_shape(s, true, true)) != MSA_OK) return st;
+      if (!prefill_shape_supported(*s)) return MSA_ERR_UNSUPPORTED;
+      *bytes = paged_prefill_pooled_bytes(*s) + sel_bytes(*s) + prefill_workspace_bytes(*s);
       return MSA_OK;
   }
   return MSA_ERR_UNSUPPORTED;
@@ -466,6 +476,51 @@ msa_status msa_forward_decode_paged(const msa_shape* s, int num_pages, const int
   pt.num_pages = num_pages;
   return forward_decode_lens(s, seq_lens, pt, q, k, v, q_idx, k_idx, o, lse, sel_out, ws,
                              ws_bytes, stream);
+}
+
+msa_status msa_forward_prefill_paged(const msa_shape* s, int num_pages,
+                                     const int32_t* page_table, const uint16_t* q,
+                                     const uint16_t* k, const uint16_t* v,
+                                     const uint16_t* q_idx, const uint16_t* k_idx, uint16_t* o,
+                                     float* lse, int32_t* sel_out, void* ws, size_t ws_bytes,
+                                     void* stream) {
+  msa_status st = check_shape(s, true, true);
+  if (st != MSA_OK) return st;
+  if (num_pages < 1) return MSA_ERR_INVALID_SHAPE;
+  // 32-bit TMA coordinates (page*G + g) and index-key rows (page*128)
+  if (static_cast<int64_t>(num_pages) * s->n_kv_heads >= (1ll << 31) ||
+      static_cast<int64_t>(num_pages) * 128 >= (1ll << 31))
+    return MSA_ERR_UNSUPPORTED;
+  if ((st = check_attn_ptrs(q, k, v, nullptr, false, o, lse)) != MSA_OK) return st;
+  if (!q_idx || !k_idx || !page_table) return MSA_ERR_NULL_PTR;
+  if (!aligned16(q_idx) || !aligned16(k_idx) || (sel_out && !aligned16(sel_out)) ||
+      (reinterpret_cast<uintptr_t>(page_table) & 3u) != 0)
+    return MSA_ERR_MISALIGNED;
+  size_t need = 0;
+  if ((st = msa_workspace_size(s, MSA_OP_FORWARD_PREFILL_PAGED, &need)) != MSA_OK) return st;
+  if (!ws) return MSA_ERR_NULL_PTR;
+  if (ws_bytes < need) return MSA_ERR_WORKSPACE_TOO_SMALL;
+  if (!aligned16(ws)) return MSA_ERR_MISALIGNED;
+  if (!device_ctx()) return MSA_ERR_CUDA;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  PageTable pt;
+  pt.table = page_table;
+  pt.num_pages = num_pages;
+  char* w = static_cast<char*>(ws);
+  const size_t pb = paged_prefill_pooled_bytes(*s);
+  float* pooled = reinterpret_cast<float*>(w);
+  int32_t* sel = sel_out ? sel_out : reinterpret_cast<int32_t*>(w + pb);
+  void* rest = w + pb + sel_bytes(*s);
+  cudaError_t e;
+  if (pb == 0) {
+    e = launch_index_topk(*s, q_idx, k_idx, sel, cs, pt);
+  } else {
+    e = launch_index_scores(*s, q_idx, k_idx, pooled, false, cs, nullptr, pt);
+    if (e == cudaSuccess) e = launch_block_topk(*s, pooled, sel, cs);
+  }
+  if (e == cudaSuccess)
+    e = launch_sparse_prefill(*s, q, k, v, sel, o, lse, rest, cs, nullptr, nullptr, pt);
+  return from_cuda(e);
 }
 
 msa_status msa_dense_attn_prefill(const msa_shape* s, const uint16_t* q, const uint16_t* k,

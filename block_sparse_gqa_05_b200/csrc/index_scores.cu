@@ -37,6 +37,8 @@ constexpr uint32_t kBarBytes = ((2 * kStages + 4 + 2 * kAcc + 2 * kRing + 1) * 8
 struct IdxParams {
   float* pooled;
   int32_t* sel;  // fused top-k: [B, T, G, k]
+  const int32_t* pages;   // paged index keys: [B, nb] page of each block, or nullptr
+  int num_pages;
   uint32_t* err;
   int T, N, G, q_off, nb, k;
   int rowmajor;  // items are whole row tiles, largest first (fused top-k)
@@ -203,11 +205,33 @@ __global__ void __launch_bounds__(kThreads + (KMAX > 0 ? kTopkThreads : 0), 1)
         mbar_arrive_expect_tx(&qfull[qb], kQTile);
         tma_load_2d(qbuf + qb * kQTile, &tm_q, &qfull[qb], 0, seq * p.T * p.G + m * 128);
         ++q;
+        // paged index keys: a 256-key tile is two 128-row pages; a block past
+        // the sequence's table loads its last page (those scores are unused).
+        // Each tile's page ids are read one tile ahead, so that their latency
+        // overlaps the wait for a free stage.
+        auto page_row = [&](int blk) -> int {
+          const int bb = blk < p.nb ? blk : p.nb - 1;
+          return page_of(p.pages, p.nb, p.num_pages, seq, bb, p.err) * 128;
+        };
+        int pr0 = 0, pr1 = 0;
+        if (p.pages && b0 < b1) {
+          pr0 = page_row(b0);
+          pr1 = page_row(b0 + 1);
+        }
         for (int b = b0; b < b1; b += 2) {
           const int s = static_cast<int>(j % kStages);
           if (!(ok = mbar_wait(&kempty[s], ((j / kStages) & 1) ^ 1, abort_flag, p.err))) break;
           mbar_arrive_expect_tx(&kfull[s], kKTile);
-          tma_load_2d(kbuf + s * kKTile, &tm_k, &kfull[s], 0, seq * p.N + b * 128);
+          if (p.pages) {
+            tma_load_2d(kbuf + s * kKTile, &tm_k, &kfull[s], 0, pr0);
+            tma_load_2d(kbuf + s * kKTile + kKTile / 2, &tm_k, &kfull[s], 0, pr1);
+            if (b + 2 < b1) {
+              pr0 = page_row(b + 2);
+              pr1 = page_row(b + 3);
+            }
+          } else {
+            tma_load_2d(kbuf + s * kKTile, &tm_k, &kfull[s], 0, seq * p.N + b * 128);
+          }
           ++j;
         }
       }
@@ -537,10 +561,13 @@ __global__ void __launch_bounds__(256) index_scores_scan_kernel(const uint16_t* 
 // the selection into ``sel`` (k <= KMAX).
 template <int DI, int KMAX>
 cudaError_t launch_tc(const msa_shape& s, const uint16_t* q_idx, const uint16_t* k_idx,
-                      float* pooled, int32_t* sel, const DevCtx* ctx, cudaStream_t st) {
+                      float* pooled, int32_t* sel, PageTable pages, const DevCtx* ctx,
+                      cudaStream_t st) {
   IdxParams p{};
   p.pooled = pooled;
   p.sel = sel;
+  p.pages = pages.table;
+  p.num_pages = pages.num_pages;
   p.k = s.topk;
   p.rowmajor = KMAX > 0 ? 1 : 0;
   p.err = ctx->err;
@@ -565,10 +592,14 @@ cudaError_t launch_tc(const msa_shape& s, const uint16_t* q_idx, const uint16_t*
   CUtensorMap tq, tk;
   const uint64_t dq[2] = {static_cast<uint64_t>(DI),
                           static_cast<uint64_t>(s.batch) * s.seq_q * s.n_kv_heads};
-  const uint64_t dk[2] = {static_cast<uint64_t>(DI), static_cast<uint64_t>(s.batch) * s.seq_kv};
+  // contiguous keys: [B*N rows][DI], 256-row boxes; paged: [P*128 rows][DI],
+  // one 128-row page per box
+  const uint64_t dk[2] = {static_cast<uint64_t>(DI),
+                          pages.table ? static_cast<uint64_t>(pages.num_pages) * 128
+                                      : static_cast<uint64_t>(s.batch) * s.seq_kv};
   const uint64_t stride[1] = {static_cast<uint64_t>(DI) * 2};
   const uint32_t box[2] = {static_cast<uint32_t>(DI), 128};
-  const uint32_t kbox[2] = {static_cast<uint32_t>(DI), 256};
+  const uint32_t kbox[2] = {static_cast<uint32_t>(DI), pages.table ? 128u : 256u};
   const CUtensorMapSwizzle sw =
       DI == 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
   if (!encode_tmap(&tq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, q_idx, dq, stride, box, sw) ||
@@ -591,11 +622,11 @@ cudaError_t launch_tc(const msa_shape& s, const uint16_t* q_idx, const uint16_t*
   return cudaGetLastError();
 }
 
-// The tensor-core path needs a full 128-row query tile and a 256-key box;
-// ragged and paged decode always scan.
-bool tc_path(const msa_shape& s) {
+// The tensor-core path needs a full 128-row query tile and (contiguous keys)
+// a 256-key box; ragged decode always scans.
+bool tc_path(const msa_shape& s, bool paged) {
   return static_cast<long long>(s.seq_q) * s.n_kv_heads >= 128 &&
-         static_cast<long long>(s.batch) * s.seq_kv >= 256;
+         (paged || static_cast<long long>(s.batch) * s.seq_kv >= 256);
 }
 
 }  // namespace
@@ -608,7 +639,7 @@ cudaError_t launch_index_scores(const msa_shape& s, const uint16_t* q_idx, const
   const int nb = static_cast<int>(ceil_div(s.seq_kv, 128));
   const long long rows = static_cast<long long>(s.batch) * s.seq_q * s.n_kv_heads;
   cudaError_t e;
-  if (lens || pages.table || !tc_path(s)) {
+  if (lens || !tc_path(s, pages.table != nullptr)) {
     const int last_bt = (s.q_offset + s.seq_q - 1) / 128;
     const dim3 grid(static_cast<unsigned>(s.batch * s.seq_q),
                     static_cast<unsigned>(ceil_div(last_bt + 1, 8)));
@@ -624,8 +655,8 @@ cudaError_t launch_index_scores(const msa_shape& s, const uint16_t* q_idx, const
                                                          pages.table, pages.num_pages, ctx->err);
     e = cudaGetLastError();
   } else {
-    e = s.index_dim == 64 ? launch_tc<64, 0>(s, q_idx, k_idx, pooled, nullptr, ctx, st)
-                          : launch_tc<32, 0>(s, q_idx, k_idx, pooled, nullptr, ctx, st);
+    e = s.index_dim == 64 ? launch_tc<64, 0>(s, q_idx, k_idx, pooled, nullptr, pages, ctx, st)
+                          : launch_tc<32, 0>(s, q_idx, k_idx, pooled, nullptr, pages, ctx, st);
   }
   if (e != cudaSuccess || !fill_upper) return e;
   const long long warps_needed = rows;
@@ -645,23 +676,23 @@ cudaError_t launch_index_scores(const msa_shape& s, const uint16_t* q_idx, const
 // standalone top-k is faster; many row tiles, or short rows, balance.  The
 // rule depends on the shape alone, so workspace sizes do not depend on the
 // device.
-bool index_topk_fusable(const msa_shape& s) {
-  if (!tc_path(s) || s.topk > 32) return false;
+bool index_topk_fusable(const msa_shape& s, bool paged) {
+  if (!tc_path(s, paged) || s.topk > 32) return false;
   const long long row_tiles = static_cast<long long>(s.batch) *
                               ceil_div(static_cast<int64_t>(s.seq_q) * s.n_kv_heads, 128);
   return row_tiles >= 1024 || ceil_div(s.seq_kv, 128) <= 1024;
 }
 
 cudaError_t launch_index_topk(const msa_shape& s, const uint16_t* q_idx, const uint16_t* k_idx,
-                              int32_t* sel, cudaStream_t st) {
+                              int32_t* sel, cudaStream_t st, PageTable pages) {
   const DevCtx* ctx = device_ctx();
   if (!ctx) return cudaErrorInitializationError;
-  if (!index_topk_fusable(s)) return cudaErrorNotSupported;
+  if (!index_topk_fusable(s, pages.table != nullptr)) return cudaErrorNotSupported;
   if (s.topk <= 16)
-    return s.index_dim == 64 ? launch_tc<64, 16>(s, q_idx, k_idx, nullptr, sel, ctx, st)
-                             : launch_tc<32, 16>(s, q_idx, k_idx, nullptr, sel, ctx, st);
-  return s.index_dim == 64 ? launch_tc<64, 32>(s, q_idx, k_idx, nullptr, sel, ctx, st)
-                           : launch_tc<32, 32>(s, q_idx, k_idx, nullptr, sel, ctx, st);
+    return s.index_dim == 64 ? launch_tc<64, 16>(s, q_idx, k_idx, nullptr, sel, pages, ctx, st)
+                             : launch_tc<32, 16>(s, q_idx, k_idx, nullptr, sel, pages, ctx, st);
+  return s.index_dim == 64 ? launch_tc<64, 32>(s, q_idx, k_idx, nullptr, sel, pages, ctx, st)
+                           : launch_tc<32, 32>(s, q_idx, k_idx, nullptr, sel, pages, ctx, st);
 }
 
 }  // namespace msa

@@ -64,9 +64,9 @@ cudaError_t launch_index_scores(const msa_shape& s, const uint16_t* q_idx,
                                 PageTable pages = PageTable{});
 // Index scores with the block top-k fused in (prefill shapes on the tensor-core
 // path, k <= 32): writes the selection directly, no pooled scores.
-bool index_topk_fusable(const msa_shape& s);
+bool index_topk_fusable(const msa_shape& s, bool paged = false);
 cudaError_t launch_index_topk(const msa_shape& s, const uint16_t* q_idx, const uint16_t* k_idx,
-                              int32_t* sel, cudaStream_t st);
+                              int32_t* sel, cudaStream_t st, PageTable pages = PageTable{});
 cudaError_t launch_block_topk(const msa_shape& s, const float* pooled, int32_t* sel,
                               cudaStream_t st, const int32_t* lens = nullptr);
 size_t prefill_workspace_bytes(const msa_shape& s);
@@ -75,10 +75,13 @@ size_t prefill_workspace_bytes(const msa_shape& s);
 // entry map (and, with the alignment output, [H] head sums and [G][k] pooled
 // scores).  False when a shape needs more than one CTA can hold.
 bool prefill_shape_supported(const msa_shape& s);
+// Paged caches (chunked prefill): k, v [num_pages, G, 128, d] with the table
+// [B, nb]; the V rows of a sequence's last page past N are zeroed before use.
 cudaError_t launch_sparse_prefill(const msa_shape& s, const uint16_t* q, const uint16_t* k,
                                   const uint16_t* v, const int32_t* sel, uint16_t* o,
                                   float* lse, void* ws, cudaStream_t st,
-                                  const float* pooled = nullptr, float* kl = nullptr);
+                                  const float* pooled = nullptr, float* kl = nullptr,
+                                  PageTable pages = PageTable{});
 size_t decode_workspace_bytes(const msa_shape& s, bool dense);
 cudaError_t launch_decode(const msa_shape& s, const uint16_t* q, const uint16_t* k,
                           const uint16_t* v, const int32_t* sel, uint16_t* o, float* lse,

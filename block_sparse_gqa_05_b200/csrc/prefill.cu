@@ -280,6 +280,8 @@ struct AttnParams {
   uint32_t* err;
   int T, N, H, G, r, k, nb, q_off, tpt;
   int q3d;   // r = 8, d = 128: one 3-D TMA load per token ([half][head][64] in smem)
+  const int32_t* pages;   // paged K/V: [B, nb] page of each block, or nullptr
+  int num_pages;
   float scale_log2;
 };
 
@@ -312,7 +314,8 @@ struct AttnSmem {
   static constexpr uint32_t kOffBar = kOffTrow + kTentWords * 4;
   // barriers: K 2+2, V kNV+kNV, Q kNQ+kNQ, S/P kNS+kNS, O 2+2, row sums 2+2,
   // metadata 2+2; then the TMEM address and the abort flag
-  static constexpr uint32_t kNBars = 4 + 2 * kNV + 2 * kNQ + 2 * kNS + 12 + 1;   // + MMA drain
+  // + MMA drain + one per V stage for the loads of a paged cache's last block
+  static constexpr uint32_t kNBars = 4 + 2 * kNV + 2 * kNQ + 2 * kNS + 12 + 1 + kNV;
   static constexpr uint32_t kBytes = kOffBar + kNBars * 8 + 8;
   static_assert(kBytes <= 227u * 1024u, "shared memory of one CTA");
 };
@@ -371,9 +374,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   uint64_t* mfull = lempty + 2;         // [2] metadata batch ready
   uint64_t* mempty = mfull + 2;         // [2] metadata batch consumed
   uint64_t* mma_drain = mempty + 2;     // the MMA thread's last commit before exit
+  uint64_t* vtail = mma_drain + 1;      // [kNV] V of a paged cache's last block loaded
   int4* thdr = reinterpret_cast<int4*>(smem + L::kOffThdr);
   int* trow = reinterpret_cast<int*>(smem + L::kOffTrow);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_drain + 1);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(vtail + kNV);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -408,6 +412,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       mbar_init(&qempty[i], 1);
     }
     mbar_init(mma_drain, 1);
+    for (int i = 0; i < kNV; ++i) mbar_init(&vtail[i], 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -445,6 +450,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         uint32_t qph = 0;              // its parity
         long long q_armed = 0;         // query tiles this warp issued loads for (lane 0)
         int kv_armed = 0;              // K (warp 0) or V (warp 3) columns loaded (lane 0)
+        uint32_t vtail_ph = 0;         // warp 3: parity of each V stage's tail barrier
         const int nx = (tpt + 63) >> 6;   // this warp's tokens per lane (<= 2)
         for (long long i = 0; i < n; ++i) {
           int ok = 1;
@@ -520,23 +526,53 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 #pragma unroll
                   for (int c = 0; c < D / 64; ++c)
                     tma_load_3d(smem + L::kOffK + st * L::kKV + c * 16384, &tm_k, &kfull[st],
-                                c * 64, hd.y * 128, hd.x);
+                                c * 64, hd.y, hd.x);
                 }
               } else {
                 const int vs = u % kNV;
                 ok = mbar_wait(&vempty[vs], ((u / kNV) & 1) ^ 1, abort_flag, p.err) ? 1 : 0;
                 if (ok) {
+                  // the last block of a paged sequence lands on its own barrier
+                  // and reaches the PV through the zeroing below
+                  uint64_t* vb = (hd.w & 4) ? &vtail[vs] : &vfull[vs];
                   ++kv_armed;
-                  mbar_arrive_expect_tx(&vfull[vs], L::kKV);
+                  mbar_arrive_expect_tx(vb, L::kKV);
 #pragma unroll
                   for (int c = 0; c < D / 64; ++c)
-                    tma_load_3d(smem + L::kOffV + vs * L::kKV + c * 16384, &tm_v, &vfull[vs],
-                                c * 64, hd.y * 128, hd.x);
+                    tma_load_3d(smem + L::kOffV + vs * L::kKV + c * 16384, &tm_v, vb, c * 64,
+                                hd.y, hd.x);
                 }
               }
             }
             ok = __shfl_sync(0xffffffffu, ok, 0);
             if (!ok) break;
+            if (gw == 1 && (hd.w & 4)) {
+              // V rows at or past N: zero them (a weight of 0 times NaN is NaN)
+              const int vs = u % kNV;
+              const uint32_t ph = (vtail_ph >> vs) & 1u;
+              if (lane == 0) ok = mbar_wait(&vtail[vs], ph, abort_flag, p.err) ? 1 : 0;
+              ok = __shfl_sync(0xffffffffu, ok, 0);
+              vtail_ph ^= 1u << vs;
+              if (!ok) {
+                // the load lands before the CTA may exit; the stage's full
+                // barrier completes so that the drain below finds it done
+                if (lane == 0) {
+                  mbar_drain(&vtail[vs], ph);
+                  mbar_arrive(&vfull[vs]);
+                }
+                break;
+              }
+              const int valid = p.N & 127;
+              uint8_t* vt = smem + L::kOffV + vs * L::kKV;
+              for (int x = lane; x < (128 - valid) * (D / 8); x += 32) {
+                const int row = valid + x / (D / 8), unit = x % (D / 8);
+                *reinterpret_cast<uint4*>(vt + (unit >> 3) * 16384 + row * 128 + (unit & 7) * 16) =
+                    make_uint4(0, 0, 0, 0);
+              }
+              fence_proxy_async_smem();
+              __syncwarp();
+              if (lane == 0) mbar_arrive(&vfull[vs]);
+            }
           }
           if (++qb == kNQ) {
             qb = 0;
@@ -580,9 +616,20 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         const int b = bg / p.G, g = bg - b * p.G;
         const int rowbase = b * p.T * p.H + g * p.r;
         if (lane < nt) {
+          const int blk = col - bg * p.nb;
+          // the K/V TMA coordinates of the column's block: (row, matrix) in
+          // [B*G][N][d], or (0, page*G + g) in a paged [P*G][128][d]; flag 4:
+          // the block is the last of a paged sequence, whose rows past N may
+          // hold any bits and are zeroed in V before the PV
+          int z = bg, y = blk * 128, tail = 0;
+          if (p.pages) {
+            z = page_of(p.pages, p.nb, p.num_pages, b, blk, p.err) * p.G + g;
+            y = 0;
+            tail = (blk == p.nb - 1 && (p.N & 127) != 0) ? 4 : 0;
+          }
           const int flags = (col != prvcol ? 1 : 0) |
-                            ((a + lane + 1 >= t_end || nextcol != col) ? 2 : 0);
-          thdr[ms * kMBMax + lane] = make_int4(bg, col - bg * p.nb, td.z, flags);
+                            ((a + lane + 1 >= t_end || nextcol != col) ? 2 : 0) | tail;
+          thdr[ms * kMBMax + lane] = make_int4(z, y, td.z, flags);
         }
         // entries of tiles a .. a+nt-1 are contiguous: nt * tpt words
         const int nent = nt * tpt;
@@ -1055,10 +1102,12 @@ cudaError_t launch_attn(const msa_shape& s, const uint16_t* q, const uint16_t* k
   const uint32_t bq3[3] = {64, 8, 2};
   const uint64_t sq[1] = {static_cast<uint64_t>(D) * 2};
   const uint32_t bq[2] = {64, static_cast<uint32_t>(p.r)};
-  const uint64_t dk[3] = {static_cast<uint64_t>(D), static_cast<uint64_t>(s.seq_kv),
-                          static_cast<uint64_t>(s.batch) * s.n_kv_heads};
-  const uint64_t sk[2] = {static_cast<uint64_t>(D) * 2,
-                          static_cast<uint64_t>(s.seq_kv) * D * 2};
+  // K/V: [B*G][N][d] contiguous, or [P*G][128][d] in pages of one block
+  const uint64_t kv_rows = p.pages ? 128 : static_cast<uint64_t>(s.seq_kv);
+  const uint64_t kv_mats = p.pages ? static_cast<uint64_t>(p.num_pages) * s.n_kv_heads
+                                   : static_cast<uint64_t>(s.batch) * s.n_kv_heads;
+  const uint64_t dk[3] = {static_cast<uint64_t>(D), kv_rows, kv_mats};
+  const uint64_t sk[2] = {static_cast<uint64_t>(D) * 2, kv_rows * D * 2};
   const uint32_t bk[3] = {64, 128, 1};
   // partial rows: (entry, head) with entries in column order
   const uint64_t prow = static_cast<uint64_t>(s.batch) * s.seq_q * s.topk * s.n_q_heads;
@@ -1115,7 +1164,7 @@ bool prefill_shape_supported(const msa_shape& s) {
 cudaError_t launch_sparse_prefill(const msa_shape& s, const uint16_t* q, const uint16_t* k,
                                   const uint16_t* v, const int32_t* sel, uint16_t* o,
                                   float* lse, void* ws, cudaStream_t st, const float* pooled,
-                                  float* kl) {
+                                  float* kl, PageTable pages) {
   const DevCtx* ctx = device_ctx();
   if (!ctx) return cudaErrorInitializationError;
   PrefillWs w = carve(s, ws);
@@ -1170,6 +1219,8 @@ cudaError_t launch_sparse_prefill(const msa_shape& s, const uint16_t* q, const u
   p.q_off = s.q_offset;
   p.tpt = tpt;
   p.q3d = (r == 8 && s.head_dim == 128) ? 1 : 0;
+  p.pages = pages.table;
+  p.num_pages = pages.num_pages;
   p.scale_log2 = kLog2e / sqrtf(static_cast<float>(s.head_dim));
   e = s.head_dim == 128 ? launch_attn<128>(s, q, k, v, p, ctx, st)
                         : launch_attn<64>(s, q, k, v, p, ctx, st);

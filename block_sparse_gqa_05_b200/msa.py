@@ -19,7 +19,7 @@ LIB_PATH = os.path.join(_PKG, "libmsa.so")
 HEADER_PATH = os.path.join(os.path.dirname(_PKG), "include", "msa.h")
 
 OP_INDEX_SCORES, OP_BLOCK_TOPK, OP_SPARSE_PREFILL, OP_SPARSE_DECODE, OP_FORWARD, \
-    OP_DENSE_PREFILL, OP_DENSE_DECODE, OP_FORWARD_ALIGNMENT = range(8)
+    OP_DENSE_PREFILL, OP_DENSE_DECODE, OP_FORWARD_ALIGNMENT, OP_FORWARD_PREFILL_PAGED = range(9)
 
 STATUS = {0: "MSA_OK", 1: "MSA_ERR_INVALID_SHAPE", 2: "MSA_ERR_NULL_PTR", 3: "MSA_ERR_MISALIGNED",
           4: "MSA_ERR_WORKSPACE_TOO_SMALL", 5: "MSA_ERR_UNSUPPORTED", 6: "MSA_ERR_CUDA",
@@ -64,6 +64,8 @@ _SIGS = {
                      ctypes.c_size_t, _vp], ctypes.c_int),
     "msa_forward_alignment": ([ctypes.POINTER(Shape), _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
                                _vp, _vp, ctypes.c_size_t, _vp], ctypes.c_int),
+    "msa_forward_prefill_paged": ([ctypes.POINTER(Shape), ctypes.c_int, _vp, _vp, _vp, _vp, _vp,
+                                   _vp, _vp, _vp, _vp, _vp, ctypes.c_size_t, _vp], ctypes.c_int),
     "msa_forward_decode_paged": ([ctypes.POINTER(Shape), ctypes.c_int, _vp, _vp, _vp, _vp, _vp,
                                   _vp, _vp, _vp, _vp, _vp, _vp, ctypes.c_size_t, _vp],
                                  ctypes.c_int),
@@ -310,6 +312,29 @@ def forward_decode_paged(shape: Shape, q, k_pages, v_pages, q_idx, kidx_pages, s
                                           a["kidx_pages"], a["o"], a["lse"], a["sel"],
                                           *_ws(ws), _stream(stream)),
            "msa_forward_decode_paged")
+    return o, lse, sel
+
+
+def forward_prefill_paged(shape: Shape, q, k_pages, v_pages, q_idx, kidx_pages, page_table,
+                          o=None, lse=None, sel=None, ws=None, want_lse=True, want_sel=True,
+                          stream=None):
+    """msa_forward_prefill_paged: one chunk of query rows (positions
+    shape.q_offset .. + seq_q - 1) over paged caches of seq_kv keys.
+    k_pages / v_pages [P, G, 128, d] bf16, kidx_pages [P, 128, d_i] bf16,
+    page_table int32 [B, ceil(shape.seq_kv / 128)]."""
+    o, lse = _attn_out(shape, q, o, lse, want_lse)
+    if sel is None and want_sel:
+        sel = torch.empty((shape.batch, shape.seq_q, shape.n_kv_heads, shape.topk),
+                          dtype=torch.int32, device=q.device)
+    ws = alloc_workspace(shape, OP_FORWARD_PREFILL_PAGED, q.device) if ws is None else ws
+    P = int(k_pages.shape[0])
+    a = _args(shape, P, page_table=page_table, q=q, k_pages=k_pages, v_pages=v_pages,
+              q_idx=q_idx, kidx_pages=kidx_pages, o=o, lse=lse, sel=sel)
+    _check(lib().msa_forward_prefill_paged(ctypes.byref(shape), P, a["page_table"], a["q"],
+                                           a["k_pages"], a["v_pages"], a["q_idx"],
+                                           a["kidx_pages"], a["o"], a["lse"], a["sel"],
+                                           *_ws(ws), _stream(stream)),
+           "msa_forward_prefill_paged")
     return o, lse, sel
 
 

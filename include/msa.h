@@ -98,7 +98,8 @@ typedef enum msa_op {
   MSA_OP_FORWARD = 4,
   MSA_OP_DENSE_PREFILL = 5,
   MSA_OP_DENSE_DECODE = 6,
-  MSA_OP_FORWARD_ALIGNMENT = 7
+  MSA_OP_FORWARD_ALIGNMENT = 7,
+  MSA_OP_FORWARD_PREFILL_PAGED = 8
 } msa_op;
 
 /* Human-readable name of a status code (static string, never NULL). */
@@ -240,6 +241,32 @@ msa_status msa_forward_decode_paged(const msa_shape* shape, int num_pages,
                                     const uint16_t* q_idx, const uint16_t* k_idx, uint16_t* o,
                                     float* lse, int32_t* sel_out, void* ws, size_t ws_bytes,
                                     void* stream);
+
+/* Whole layer for one chunk of query rows over paged caches (chunked prefill
+ * in a serving loop; no other counterpart on the pages): as msa_forward, for
+ * the T query rows at positions q_offset .. q_offset + T - 1 of B sequences
+ * that each hold N = seq_kv keys, except that the caches are stored as pages
+ * of one 128-row block (the selection unit, so a selected block is one page):
+ *   k, v        [num_pages, G, 128, d]  bf16
+ *   k_idx       [num_pages, 128, d_i]   bf16
+ *   page_table  [B, nb] int32 (device, 4-byte aligned), nb = ceil(N / 128):
+ *               page_table[b, j] holds rows 128j .. 128j+127 of sequence b.
+ * q, q_idx, o, lse, sel_out keep msa_forward's layouts (the chunk's rows
+ * only).  Rows of a sequence's last page at or past N may hold any bits (NaN
+ * and Inf included): they are masked out of the scores and zeroed in V
+ * before the weighted sum.  Several tables may share pages (a common prefix):
+ * the caches are only read.  A page id outside [0, num_pages) is clamped into
+ * it (that block's result is then wrong) and sets bit 2 of the device error
+ * word.  ws >= msa_workspace_size(MSA_OP_FORWARD_PREFILL_PAGED).
+ * Errors: num_pages < 1 -> MSA_ERR_INVALID_SHAPE; num_pages * G or
+ * num_pages * 128 >= 2^31 -> MSA_ERR_UNSUPPORTED; NULL page_table ->
+ * MSA_ERR_NULL_PTR. */
+msa_status msa_forward_prefill_paged(const msa_shape* shape, int num_pages,
+                                     const int32_t* page_table, const uint16_t* q,
+                                     const uint16_t* k, const uint16_t* v,
+                                     const uint16_t* q_idx, const uint16_t* k_idx, uint16_t* o,
+                                     float* lse, int32_t* sel_out, void* ws, size_t ws_bytes,
+                                     void* stream);
 
 /* Dense causal GQA attention (every key x <= p_t), the baseline the pages
  * compare MSA against ([P1] GQA definition; [P2], [P4] speed-ups vs GQA).

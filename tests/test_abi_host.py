@@ -127,6 +127,22 @@ def test_pointer_checks_precede_device_use(L):
                  None) == 4
     assert paged(ctypes.byref(tiny()), 8, ok, ok, ok, ok, ok, ok, ok, ok, None, None, ok, 1 << 40,
                  None) == 1                                # T must be 1
+    # paged chunked prefill: pool size, table pointer and alignment, workspace
+    pp = L.msa_forward_prefill_paged
+    c1 = tiny(seq_q=256, seq_kv=4096, q_offset=3840)
+    assert pp(ctypes.byref(c1), 0, ok, ok, ok, ok, ok, ok, ok, None, None, ok, 1 << 40, None) == 1
+    assert pp(ctypes.byref(c1), 1 << 30, ok, ok, ok, ok, ok, ok, ok, None, None, ok, 1 << 40,
+              None) == 5
+    assert pp(ctypes.byref(c1), 8, None, ok, ok, ok, ok, ok, ok, None, None, ok, 1 << 40,
+              None) == 2
+    assert pp(ctypes.byref(c1), 8, ctypes.c_void_p((1 << 20) + 2), ok, ok, ok, ok, ok, ok, None,
+              None, ok, 1 << 40, None) == 3
+    assert pp(ctypes.byref(c1), 8, ok, ok, ok, ok, ok, ok, ok, None, None, ok, 16, None) == 4
+    assert pp(ctypes.byref(tiny(seq_q=300, seq_kv=200)), 8, ok, ok, ok, ok, ok, ok, ok, None,
+              None, ok, 1 << 40, None) == 1                # q_offset + T > N
+    st, npp = ws(c1, M.OP_FORWARD_PREFILL_PAGED)
+    st2, pre = ws(c1, M.OP_SPARSE_PREFILL)
+    assert st == st2 == 0 and npp > pre                    # + the selection
     dec = tiny(seq_q=1, seq_kv=4096, q_offset=4095)
     assert L.msa_sparse_attn_decode(ctypes.byref(dec), ok, ok, ok, ok, ok, None, ok, 8, None) == 4
     assert L.msa_dense_attn_decode(ctypes.byref(s), ok, ok, ok, ok, None, ok, 1 << 30, None) == 1

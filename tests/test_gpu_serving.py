@@ -137,3 +137,48 @@ def test_forward_many_heads_and_slots(sp):
     O_ref, L_ref = oracle_attention(sp, inp, sref, 0)
     check_attn(o[0], O_ref, "many heads and slots")
     assert np.abs(lse[0].double().cpu().numpy() - L_ref).max() < LSE_ABS
+
+
+@pytest.mark.parametrize("sp,extra", [
+    # fused top-k in the index scores, r = 8, d = 128, last page 80 rows deep
+    (spec(2, 300, 2000, 1700, 16, 2, 128, 64, 16, seed=91, planted=2), 5),
+    # k = 33: index scores then the standalone top-k; d = 64, r = 2
+    (spec(1, 520, 1500, 980, 8, 4, 64, 32, 33, seed=92), 3),
+    # a single 128-row query tile, last page 76 rows deep
+    (spec(2, 64, 1100, 1036, 16, 2, 128, 64, 4, seed=93), 2),
+])
+def test_forward_prefill_paged(sp, extra):
+    """A chunk of query rows over paged caches (shuffled pages; rows past N
+    and unused pages hold NaN): bit-identical to msa_forward on the contiguous
+    caches, and selections and outputs match the oracle."""
+    inp = inputs_cpu(sp)
+    kp, vp, kip, table = _paged_caches(sp, inp, [sp.seq_kv] * sp.batch, extra, seed=sp.seed)
+    sh = M.Shape.of(sp)
+    o, lse, sel = M.forward_prefill_paged(sh, cuda(inp.q), cuda(kp), cuda(vp), cuda(inp.q_idx),
+                                          cuda(kip), cuda(torch.from_numpy(table)))
+    torch.cuda.synchronize()
+    assert M.device_status() == 0
+    o_c, lse_c, sel_c = M.forward(sh, cuda(inp.q), cuda(inp.k), cuda(inp.v), cuda(inp.q_idx),
+                                  cuda(inp.k_idx))
+    torch.cuda.synchronize()
+    assert torch.equal(sel, sel_c), "paged and contiguous selections differ"
+    assert torch.equal(o, o_c) and torch.equal(lse, lse_c), "paged and contiguous outputs differ"
+    o_ref = []
+    for b in range(sp.batch):
+        sref = oracle_sel(sp, oracle_pooled(sp, inp, b))
+        assert np.array_equal(sel[b].cpu().numpy(), sref), f"sel b={b}"
+        o_ref.append(oracle_attention(sp, inp, sref, b)[0])
+    check_attn(o, np.stack(o_ref), "paged chunked prefill")
+
+
+def test_forward_prefill_paged_bad_page_is_flagged():
+    # a page id past the pool is clamped to the last page and flagged (bit 2)
+    sp = spec(1, 256, 1024, 768, 8, 2, 64, 32, 4, seed=94)
+    inp = inputs_cpu(sp)
+    kp, vp, kip, table = _paged_caches(sp, inp, [sp.seq_kv], 2, seed=94)
+    table[0, 1] = kp.shape[0] + 7
+    sh = M.Shape.of(sp)
+    M.forward_prefill_paged(sh, cuda(inp.q), cuda(kp), cuda(vp), cuda(inp.q_idx), cuda(kip),
+                            cuda(torch.from_numpy(table)))
+    torch.cuda.synchronize()
+    assert M.device_status() & 4
