@@ -322,16 +322,16 @@ struct AttnSmem {
 
 // Roles by warpgroup: WG0 = warps 0 and 3 gather the query tiles (TMA) and
 // load K (warp 0) and V (warp 3) at column changes, warp 1 issues the MMAs,
-// warp 2 prepares tile metadata; WG1 and WG2 = softmax of alternate tiles;
-// WG3 = epilogue.  Register budget per thread is moved from WG0/WG3 to the
-// softmax warpgroups so that a softmax thread holds its whole 128-score row.
-// TMEM: each softmax warpgroup owns one S/P buffer of 128 columns (P is
-// written over the first 64 columns of its tile's S as packed bf16 and
-// consumed from there by the PV MMA) and one O buffer of D columns, so a
-// tile's PV never waits for the previous tile's output to be drained: the
-// epilogue has a whole tile of time to read O out.  S(j + 2) reuses tile j's
-// buffer and is issued once PV(j) is (tcgen05 MMAs of one thread run in
-// issue order).
+// warp 2 prepares tile metadata; WG1 and WG2 = softmax, both on every tile
+// (warpgroup wg takes key columns [64 wg, 64 wg + 64) of each row); WG3 =
+// epilogue.  Register budget per thread is moved from WG0/WG3 to the softmax
+// warpgroups so that a softmax thread holds its 64 scores.
+// TMEM: kNS = 2 S/P buffers of 128 columns, by tile parity (P is written over
+// the first 64 columns of its tile's S as packed bf16 and consumed from there
+// by the PV MMA), and kNO = 2 O buffers of D columns, so a tile's PV never
+// waits for the previous tile's output to be drained: the epilogue has a
+// whole tile of time to read O out.  S(j + 2) reuses tile j's buffer and is
+// issued once PV(j) is (tcgen05 MMAs of one thread run in issue order).
 template <int D>
 __global__ void __launch_bounds__(kAttnThreads, 1)
     kvouter_attn_kernel(const __grid_constant__ CUtensorMap tm_q,
@@ -982,9 +982,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 //   P_main(s)  = mean over the group's heads of w_s / sum w
 //   P_index(s) = softmax over the selected slots of pooled[t, g, sel[s]]
 //   kl[t, g]   = sum_s P_main(s) (log P_main(s) - log P_index(s)).
-// Six CTAs per SM (<= 40 registers): the kernel waits on scattered partial
-// reads, and the KL variant at its natural 46 registers fits only five, which
-// cost it a fifth of its speed.
+// Eight CTAs per SM (<= 32 registers, no spills): the kernel waits on
+// scattered partial reads, so resident warps decide its speed (six CTAs at
+// 40 registers ran 13% slower).
 template <int D, bool KL>
 __global__ void __launch_bounds__(256, 8) combine_kernel(const int32_t* __restrict__ sel,
                                                       const PrefillWs w, uint16_t* __restrict__ o,
