@@ -245,6 +245,21 @@ def dense_roofline(sp, ms, peaks):
             "frac": round(a / pk, 4), "algorithmic_per_launch": dense_flops(sp)}
 
 
+def combine_bytes(sp, sel):
+    """The combine's reads and writes: r partial rows of (2*d + 8) bytes per
+    kept (token, group, slot), one bf16 output row per (token, head)."""
+    r = sp.n_q_heads // sp.n_kv_heads
+    kept = float((sel >= 0).sum().item())
+    return kept * r * (2 * sp.head_dim + 8) + float(sp.batch * sp.seq_q * sp.n_q_heads * 2 * sp.head_dim)
+
+
+def l2_note(sp):
+    """How the timed loop relates to the 126 MB L2: its input sizes."""
+    q = sp.batch * sp.seq_q * sp.n_q_heads * sp.head_dim * 2
+    kv = sp.batch * sp.seq_kv * sp.n_kv_heads * sp.head_dim * 2 * 2
+    return f"inputs larger than L2 (Q {q / 2**20:.0f} MiB, K/V {kv / 2**20:.0f} MiB per step)"
+
+
 def decode_kv_bytes(sp):
     return float(sp.batch * sp.n_kv_heads * sp.topk * 128 * sp.head_dim * 2 * 2)
 
@@ -304,8 +319,10 @@ def run_msa(args, world, rank, pg):
     dom = max(kernels, key=lambda k: kernels[k] * prof[k][1])
     work = {
         "kvouter_attn": ("tensor", selected_attention_flops(sp, sel)),
+        "index_topk_tc": ("tensor", index_flops(sp)),     # index GEMM with the top-k fused in
         "index_scores_tc": ("tensor", index_flops(sp)),
         "block_topk": ("hbm", topk_bytes(sp)),
+        "combine": ("hbm", combine_bytes(sp, sel)),
     }
     bound, amount = work.get(dom, ("tensor", selected_attention_flops(sp, sel)))
     dur_s = kernels[dom] / 1e3
@@ -340,6 +357,27 @@ def run_msa(args, world, rank, pg):
                             "frac": round(a / pk, 4)}
     out["stages"] = stages
     out["step_roofline"] = prefill_step_bound(sp, sel, peaks, ms)
+
+    # ---- the same layer with the index-alignment KL (msa_forward_alignment:
+    # pooled scores kept, the combine's KL variant)
+    if args.alignment:
+        ka = torch.empty((sp.batch, sp.seq_q, sp.n_kv_heads), dtype=torch.float32, device="cuda")
+        wsa = M.alloc_workspace(sh, M.OP_FORWARD_ALIGNMENT)
+
+        def astep():
+            M.forward_alignment(sh, inp.q, inp.k, inp.v, inp.q_idx, inp.k_idx, o=o, lse=None,
+                                sel=sel, kl=ka, ws=wsa, want_lse=False)
+        astep()
+        torch.cuda.synchronize()
+        M.profile_enable(True)
+        ams = timed_loop(astep, 2, 1, pg, stream)
+        aprof = M.profile_read()
+        M.profile_enable(False)
+        out["alignment_forward"] = {
+            "ms_per_step": ams,
+            "kernels_ms_per_launch": {k: round(v[0] / v[1], 4) for k, v in aprof.items()}}
+        del ka, wsa
+        torch.cuda.empty_cache()
 
     # ---- the same workload through the dense causal GQA kernel (the baseline
     # the pages compare MSA against)
@@ -686,6 +724,8 @@ def main():
     ap.add_argument("--skip-e2e", action="store_true")
     ap.add_argument("--skip-topk-micro", action="store_true")
     ap.add_argument("--skip-dense", action="store_true")
+    ap.add_argument("--alignment", action="store_true",
+                    help="also time msa_forward_alignment (the KL variant) on the workload")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--ref-step-s", type=float, default=4.0)
     args = ap.parse_args()
@@ -718,12 +758,12 @@ def main():
                            "heads": f"{sp.n_q_heads}q/{sp.n_kv_heads}kv",
                            "head_dim": sp.head_dim, "index_dim": sp.index_dim, "block": sp.block,
                            "topk": sp.topk, "parallelism": parallelism,
-                           "l2": "inputs larger than L2 (Q 2 GiB, K/V 512 MiB per step)"},
+                           "l2": l2_note(sp)},
                 "gpu_launches": res["gpu_launches"], "roofline": res["roofline"],
                 "stages": res["stages"], "kernels_ms_per_launch": res["kernels_ms_per_launch"],
                 "clocks": res["clocks"]}
-        for key in ("step_roofline", "e2e", "dense_gqa_prefill", "topk_microbench", "decode",
-                    "ctx_1m"):
+        for key in ("step_roofline", "e2e", "dense_gqa_prefill", "alignment_forward",
+                    "topk_microbench", "decode", "ctx_1m"):
             if key in res:
                 line[key] = res[key]
         if world == 1 and not args.skip_cpu:

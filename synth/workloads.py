@@ -24,6 +24,9 @@ WORKLOADS = {
     # small cases of the same shapes, sized for profiler captures (a few GB on the device)
     "prefill_16k": WorkloadSpec(1, 16384, 16384, 0, _H, _G, _D, _DI, 128, 16, seed=7, planted=4),
     "decode_16k_b8": WorkloadSpec(8, 1, 16384, 16383, _H, _G, _D, _DI, 128, 16, seed=8, planted=4),
+    # a decode with more than 512 candidate blocks per row and few rows (the
+    # top-k's CTA-per-row kernel), at ~3 GB of caches
+    "decode_80k_b8": WorkloadSpec(8, 1, 81920, 81919, _H, _G, _D, _DI, 128, 16, seed=9, planted=4),
 }
 
 
