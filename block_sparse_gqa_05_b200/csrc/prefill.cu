@@ -198,19 +198,25 @@ __global__ void __launch_bounds__(1024) scan_columns_kernel(PrefillWs w, int tpt
   }
 }
 
-// Tiles of segment s dealt to CTA c: [first(c), first(c + 1)) of its n_s
-// tiles in column order, first(c) = c * n_s / grid, and the CTA holding
-// segment tile x.
-__device__ __forceinline__ long long deal_first(long long c, long long n, int grid) {
-  return c * n / grid;
+// Segment s's n_s tiles, in column order, are cut into grid chunks,
+// chunk j = [first(j), first(j + 1)), first(j) = j * n_s / grid; chunk_of(x)
+// is the chunk holding segment tile x.  Chunk j goes to CTA (j - s * rot)
+// mod grid: the last chunks of a segment (its latest blocks: short columns,
+// so more K/V loads per tile, and causally masked tiles) land on a
+// different CTA for every segment instead of all on the last CTA.
+__device__ __forceinline__ long long deal_first(long long j, long long n, int grid) {
+  return j * n / grid;
 }
-__device__ __forceinline__ int deal_cta(long long x, long long n, int grid) {
+__device__ __forceinline__ int chunk_of(long long x, long long n, int grid) {
   return static_cast<int>(((x + 1) * grid + n - 1) / n - 1);
+}
+__device__ __forceinline__ int chunk_of_cta(int c, long long sg, int rot, int grid) {
+  return static_cast<int>((c + sg * rot) % grid);
 }
 
 // One CTA: per attention CTA c, the tiles it holds in the segments before
 // each segment (seg_prefix) and its first tile in the dealt order (cta_off).
-__global__ void __launch_bounds__(1024) plan_ctas_kernel(PrefillWs w, int nb, int grid) {
+__global__ void __launch_bounds__(1024) plan_ctas_kernel(PrefillWs w, int nb, int grid, int rot) {
   __shared__ uint32_t warp_sum[32];
   const int c = threadIdx.x, lane = c & 31, warp = c >> 5;
   uint32_t acc = 0;
@@ -219,7 +225,8 @@ __global__ void __launch_bounds__(1024) plan_ctas_kernel(PrefillWs w, int nb, in
       const long long lo = w.tile_off[sg * nb];
       const long long n = static_cast<long long>(w.tile_off[(sg + 1) * nb]) - lo;
       w.seg_prefix[sg * grid + c] = acc;
-      acc += static_cast<uint32_t>(deal_first(c + 1, n, grid) - deal_first(c, n, grid));
+      const int j = chunk_of_cta(c, sg, rot, grid);
+      acc += static_cast<uint32_t>(deal_first(j + 1, n, grid) - deal_first(j, n, grid));
     }
   }
   uint32_t incl = acc;
@@ -248,7 +255,7 @@ __global__ void __launch_bounds__(1024) plan_ctas_kernel(PrefillWs w, int nb, in
 // One thread per tile: find its column (upper bound in the tile offsets),
 // write the descriptor and the tile's entries padded to tpt at the tile's
 // place in the dealt order.
-__global__ void make_tiles_kernel(PrefillWs w, int tpt, int nb, int grid) {
+__global__ void make_tiles_kernel(PrefillWs w, int tpt, int nb, int grid, int rot) {
   const long long ntiles = static_cast<long long>(w.tile_off[w.ncol]);
   for (long long ti = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; ti < ntiles;
        ti += static_cast<long long>(gridDim.x) * blockDim.x) {
@@ -265,9 +272,10 @@ __global__ void make_tiles_kernel(PrefillWs w, int tpt, int nb, int grid) {
     const long long slo = w.tile_off[sg * nb];
     const long long n = static_cast<long long>(w.tile_off[(sg + 1) * nb]) - slo;
     const long long x = ti - slo;
-    const int cta = deal_cta(x, n, grid);
+    const int j = chunk_of(x, n, grid);
+    const int cta = static_cast<int>(((j - sg * rot) % grid + grid) % grid);
     const long long dst = static_cast<long long>(w.cta_off[cta]) + w.seg_prefix[sg * grid + cta] +
-                          (x - deal_first(cta, n, grid));
+                          (x - deal_first(j, n, grid));
     w.tiles[dst] = make_int4(static_cast<int>(c), static_cast<int>(start), static_cast<int>(cnt), 0);
     for (int j = 0; j < tpt; ++j)
       w.tile_ent[dst * tpt + j] = j < static_cast<int>(cnt) ? w.entries[start + j] : 0xFFFFFFFFu;
@@ -1195,14 +1203,18 @@ cudaError_t launch_sparse_prefill(const msa_shape& s, const uint16_t* q, const u
     sel_invert_kernel<<<hgrid, 256, hsmem, st>>>(sel, w, s.seq_q, s.n_kv_heads, s.topk, nb,
                                                  s.q_offset, 1, ctx->err);
   }
+  // chunk rotation between consecutive segments: spreads the segments'
+  // last chunks over the grid
+  const int grid = attn_grid(ctx);
+  const int rot = static_cast<int>(std::max<long long>(1, grid / std::max<long long>(1, std::min<long long>(w.nseg, grid))));
   {
     ProfScope ps_("plan_ctas", st);
-    plan_ctas_kernel<<<1, 1024, 0, st>>>(w, nb, attn_grid(ctx));
+    plan_ctas_kernel<<<1, 1024, 0, st>>>(w, nb, grid, rot);
   }
   {
     ProfScope ps_("make_tiles", st);
     make_tiles_kernel<<<static_cast<unsigned>(ceil_div(w.max_tiles, 256)), 256, 0, st>>>(
-        w, tpt, nb, attn_grid(ctx));
+        w, tpt, nb, grid, rot);
   }
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
 
