@@ -31,6 +31,7 @@ constexpr int kConsumerWarps = 8;
 constexpr int kThreads = (kConsumerWarps + 1) * 32;   // 8 consumer warps + 1 TMA warp
 constexpr int kConsumerThreads = kConsumerWarps * 32;
 constexpr int kMaxGrid = 256;
+constexpr int kMergeOnePass = 8;   // most CTAs a (sequence, group) may span for the one-pass merge
 constexpr int kPStride = 136;    // bf16 per row of the P tile: rows 272 B apart, no bank conflicts
 constexpr float kLog2e = 1.4426950408889634f;
 
@@ -497,6 +498,55 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int cf = cta_of(bfirst, n, grid), cl = cta_of(bfirst + p.per_bg - 1, n, grid);
     const int nc = cl - cf + 1;
     const int sf = 2 * cf + (bfirst == cta_first(cf, n, grid) ? 0 : 1);
+    if (nc <= kMergeOnePass) {
+      // one pass: each thread loads every partial's log-sum-exp and its four
+      // output columns together, so the merge costs one round trip
+      for (int e = threadIdx.x; e < r * D / 4; e += kConsumerThreads) {
+        const int row = (e * 4) / D, col = (e * 4) % D;
+        float lj[kMergeOnePass];
+        float4 v4[kMergeOnePass];
+#pragma unroll
+        for (int c = 0; c < kMergeOnePass; ++c) {
+          if (c < nc) {
+            const int sl = c == 0 ? sf : 2 * (cf + c);
+            lj[c] = __ldcg(&p.part_lse[static_cast<long long>(sl) * r + row]);
+            v4[c] = __ldcg(reinterpret_cast<const float4*>(
+                p.part_o + (static_cast<long long>(sl) * r + row) * D + col));
+          }
+        }
+        float M = -INFINITY;
+#pragma unroll
+        for (int c = 0; c < kMergeOnePass; ++c)
+          if (c < nc) M = fmaxf(M, lj[c]);
+        float den = 0.f;
+#pragma unroll
+        for (int c = 0; c < kMergeOnePass; ++c)
+          if (c < nc && lj[c] != -INFINITY) den += exp2f(lj[c] - M);
+        const float rden = den > 0.f ? 1.f / den : 0.f;
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int c = 0; c < kMergeOnePass; ++c) {
+          if (c < nc && lj[c] != -INFINITY) {
+            const float wj = exp2f(lj[c] - M) * rden;
+            acc.x += wj * v4[c].x;
+            acc.y += wj * v4[c].y;
+            acc.z += wj * v4[c].z;
+            acc.w += wj * v4[c].w;
+          }
+        }
+        uint2 pk;
+        pk.x = pack_bf16(acc.x, acc.y);
+        pk.y = pack_bf16(acc.z, acc.w);
+        *reinterpret_cast<uint2*>(p.o + (static_cast<long long>(b) * p.H + g * r + row) * D +
+                                  col) = pk;
+        if (p.lse && col == 0)
+          p.lse[static_cast<long long>(b) * p.H + g * r + row] =
+              den > 0.f ? (M + log2f(den)) / kLog2e : -INFINITY;
+      }
+      if (threadIdx.x == 0) p.counters[bg] = 0u;
+      named_bar_sync(1, kConsumerThreads);
+      continue;
+    }
     for (int e = threadIdx.x; e < nc * r; e += kConsumerThreads) {
       const int c = cf + e / r;
       const int sl = c == cf ? sf : 2 * c;
