@@ -361,10 +361,11 @@ msa_status forward_decode_lens(const msa_shape* s, const int32_t* seq_lens, Page
   float* pooled = reinterpret_cast<float*>(w);
   int32_t* sel = sel_out ? sel_out : reinterpret_cast<int32_t*>(w + pooled_bytes(c));
   void* rest = w + pooled_bytes(c) + sel_bytes(c);
-  cudaError_t e = launch_index_scores(c, q_idx, k_idx, pooled, false, cs, seq_lens, pages);
+  cudaError_t e = prepare_decode(c, rest, cs);
+  if (e == cudaSuccess) e = launch_index_scores(c, q_idx, k_idx, pooled, false, cs, seq_lens, pages);
   if (e == cudaSuccess) e = launch_block_topk(c, pooled, sel, cs, seq_lens);
   if (e == cudaSuccess)
-    e = launch_decode(c, q, k, v, sel, o, lse, rest, false, cs, seq_lens, pages);
+    e = launch_decode(c, q, k, v, sel, o, lse, rest, false, cs, seq_lens, pages, true);
   return from_cuda(e);
 }
 
@@ -410,11 +411,13 @@ msa_status msa_forward(const msa_shape* s, const uint16_t* q, const uint16_t* k,
     if (e == cudaSuccess) e = launch_sparse_prefill(*s, q, k, v, sel, o, lse, rest, cs);
     return from_cuda(e);
   }
-  e = launch_index_scores(*s, q_idx, k_idx, pooled, false, cs);
+  const bool decode = forward_is_decode(*s);
+  e = decode ? prepare_decode(*s, rest, cs) : cudaSuccess;
+  if (e == cudaSuccess) e = launch_index_scores(*s, q_idx, k_idx, pooled, false, cs);
   if (e == cudaSuccess) e = launch_block_topk(*s, pooled, sel, cs);
   if (e == cudaSuccess) {
-    if (forward_is_decode(*s))
-      e = launch_decode(*s, q, k, v, sel, o, lse, rest, false, cs);
+    if (decode)
+      e = launch_decode(*s, q, k, v, sel, o, lse, rest, false, cs, nullptr, PageTable{}, true);
     else
       e = launch_sparse_prefill(*s, q, k, v, sel, o, lse, rest, cs);
   }

@@ -165,6 +165,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     *abort_flag = 0;
     fence_barrier_init();
   }
+  // this kernel may start while the one before it (the top-k) finishes: the
+  // selection is read only after it is complete
+  griddep_wait();
   __syncthreads();
 
   if (warp == kConsumerWarps) {
@@ -615,10 +618,15 @@ size_t decode_workspace_bytes(const msa_shape& s, bool dense) {
          align_up(slots * r * s.head_dim * 4, 256);
 }
 
+cudaError_t prepare_decode(const msa_shape& s, void* ws, cudaStream_t st) {
+  const size_t bg = static_cast<size_t>(s.batch) * s.n_kv_heads;
+  return cudaMemsetAsync(ws, 0, bg * 4, st);   // the counters open the workspace
+}
+
 cudaError_t launch_decode(const msa_shape& s, const uint16_t* q, const uint16_t* k,
                           const uint16_t* v, const int32_t* sel, uint16_t* o, float* lse,
                           void* ws, bool dense, cudaStream_t st, const int32_t* lens,
-                          PageTable pages) {
+                          PageTable pages, bool counters_zeroed) {
   const DevCtx* ctx = device_ctx();
   if (!ctx) return cudaErrorInitializationError;
   const int r = s.n_q_heads / s.n_kv_heads;
@@ -666,7 +674,7 @@ cudaError_t launch_decode(const msa_shape& s, const uint16_t* q, const uint16_t*
                    CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorInvalidValue;
 
-  cudaError_t e = cudaMemsetAsync(p.counters, 0, bg * 4, st);
+  cudaError_t e = counters_zeroed ? cudaSuccess : cudaMemsetAsync(p.counters, 0, bg * 4, st);
   if (e != cudaSuccess) return e;
   const unsigned g = static_cast<unsigned>(grid);
   if (s.head_dim == 128) {
@@ -675,14 +683,16 @@ cudaError_t launch_decode(const msa_shape& s, const uint16_t* q, const uint16_t*
                              static_cast<int>(smem));
     if (e != cudaSuccess) return e;
     ProfScope ps_("decode_attn", st);
-    decode_attn_kernel<128><<<g, kThreads, smem, st>>>(tk, tv, p);
+    e = launch_dependent(decode_attn_kernel<128>, dim3(g), dim3(kThreads), smem, st, tk, tv, p);
+    if (e != cudaSuccess) return e;
   } else {
     const size_t smem = DecLayout<64>::kBytes;
     e = cudaFuncSetAttribute(decode_attn_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(smem));
     if (e != cudaSuccess) return e;
     ProfScope ps_("decode_attn", st);
-    decode_attn_kernel<64><<<g, kThreads, smem, st>>>(tk, tv, p);
+    e = launch_dependent(decode_attn_kernel<64>, dim3(g), dim3(kThreads), smem, st, tk, tv, p);
+    if (e != cudaSuccess) return e;
   }
   return cudaGetLastError();
 }

@@ -470,6 +470,7 @@ __global__ void __launch_bounds__(256) index_scores_scan_kernel(const uint16_t* 
                                                                 int num_pages, uint32_t* err) {
   constexpr int KS = DI / 16;          // k-steps
   constexpr int W = KS * 2;            // 32-bit words per thread per row
+  griddep_launch_dependents();         // the top-k may launch (it waits for this kernel)
   const int row_bt = blockIdx.x;       // seq * T + t
   const int seq = row_bt / T;
   const int t = row_bt - seq * T;

@@ -47,6 +47,26 @@ class ProfScope {
 inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
+// Launches a kernel that may start before the previous kernel on the stream
+// has finished (programmatic dependent launch); the kernel itself waits
+// (griddepcontrol.wait) before reading that kernel's results.  Captured into
+// CUDA graphs as a programmatic edge.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_dependent(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                             cudaStream_t st, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
+
 // ---------------------------------------------------------------- launchers
 // Each returns cudaSuccess or the launch error.  Shapes are already validated.
 // lens (device, [B], may be null): per-sequence cache lengths of ragged decode;
@@ -86,7 +106,13 @@ size_t decode_workspace_bytes(const msa_shape& s, bool dense);
 cudaError_t launch_decode(const msa_shape& s, const uint16_t* q, const uint16_t* k,
                           const uint16_t* v, const int32_t* sel, uint16_t* o, float* lse,
                           void* ws, bool dense, cudaStream_t st,
-                          const int32_t* lens = nullptr, PageTable pages = PageTable{});
+                          const int32_t* lens = nullptr, PageTable pages = PageTable{},
+                          bool counters_zeroed = false);
+// Zeroes the decode workspace's per-(sequence, group) counters ahead of the
+// kernels that precede the attention, so that the attention kernel follows
+// the top-k directly on the stream (and may start while it finishes); then
+// launch_decode(..., counters_zeroed = true).
+cudaError_t prepare_decode(const msa_shape& s, void* ws, cudaStream_t st);
 msa_status check_decode_static_args(const msa_shape* s, const uint16_t* q, const uint16_t* k,
                                     const uint16_t* v, const int32_t* sel, const uint16_t* o,
                                     const float* lse);

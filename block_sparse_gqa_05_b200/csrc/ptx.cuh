@@ -198,6 +198,15 @@ MSA_DEV void regs_dec() { asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"
 template <uint32_t N>
 MSA_DEV void regs_inc() { asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N)); }
 
+// Programmatic dependent launch: a kernel launched with programmatic stream
+// serialization may start while the kernel before it still runs; it waits
+// here for that kernel's completion (and its memory) before reading what it
+// wrote.  Without such a launch the wait returns at once.
+MSA_DEV void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+// Lets the next kernel (launched as above) start once every CTA of this one
+// has run this (it still waits for this kernel's completion before reading).
+MSA_DEV void griddep_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;"); }
+
 // Generic-proxy shared-memory writes -> visible to the async proxy (tensor core).
 MSA_DEV void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");

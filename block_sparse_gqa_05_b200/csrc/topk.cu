@@ -287,6 +287,8 @@ __global__ void __launch_bounds__(kWarps * 32, 3)
   const int warp = threadIdx.x >> 5;
   uint64_t* buf = scratch[warp];
   const long long nwarps = static_cast<long long>(gridDim.x) * kWarps;
+  griddep_launch_dependents();   // the attention may launch (it waits for this kernel)
+  griddep_wait();                // the pooled scores of the kernel before
   const bool vec = (nb & 3) == 0;
   for (long long r = static_cast<long long>(blockIdx.x) * kWarps + warp; r < rows; r += nwarps) {
     // rows < 2^31 (checked by the API): 32-bit index math
@@ -316,6 +318,8 @@ __global__ void __launch_bounds__(kWarps * 32)
   __shared__ uint64_t scratch[kWarps][kScratch];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const long long r = blockIdx.x;
+  griddep_launch_dependents();   // the attention may launch (it waits for this kernel)
+  griddep_wait();                // the pooled scores of the kernel before
   const uint32_t tg = static_cast<uint32_t>(r) / static_cast<uint32_t>(G);
   const int t = static_cast<int>(tg % static_cast<uint32_t>(T));
   const int pos = lens ? ragged_len(lens, static_cast<int>(tg / static_cast<uint32_t>(T)), N, err) - 1
@@ -365,18 +369,23 @@ cudaError_t launch_block_topk(const msa_shape& s, const float* pooled, int32_t* 
   // idle: give each row a CTA instead.
   if (rows <= 4LL * ctx->num_sms && nb > kChunk) {
     ProfScope ps_("block_topk", st);
-    block_topk_row_cta_kernel<<<static_cast<unsigned>(rows), kWarps * 32, 0, st>>>(
-        pooled, sel, s.seq_q, s.n_kv_heads, s.q_offset, nb, s.topk, lens, s.seq_kv, ctx->err);
-    return cudaGetLastError();
+    // may start while the index scan before it finishes (it waits for it)
+    const cudaError_t e = launch_dependent(block_topk_row_cta_kernel,
+                                           dim3(static_cast<unsigned>(rows)), dim3(kWarps * 32), 0,
+                                           st, pooled, sel, s.seq_q, s.n_kv_heads, s.q_offset, nb,
+                                           s.topk, lens, s.seq_kv, ctx->err);
+    return e != cudaSuccess ? e : cudaGetLastError();
   }
   long long blocks = (rows + kWarps - 1) / kWarps;
   const long long cap = static_cast<long long>(ctx->num_sms) * 32;
   if (blocks > cap) blocks = cap;
   {
     ProfScope ps_("block_topk", st);
-    block_topk_kernel<<<static_cast<unsigned>(blocks), kWarps * 32, 0, st>>>(
-      pooled, sel, rows, s.seq_q, s.n_kv_heads, s.q_offset, nb, s.topk, lens, s.seq_kv,
-      ctx->err);
+    const cudaError_t e = launch_dependent(block_topk_kernel, dim3(static_cast<unsigned>(blocks)),
+                                           dim3(kWarps * 32), 0, st, pooled, sel, rows, s.seq_q,
+                                           s.n_kv_heads, s.q_offset, nb, s.topk, lens, s.seq_kv,
+                                           ctx->err);
+    if (e != cudaSuccess) return e;
   }
   return cudaGetLastError();
 }
