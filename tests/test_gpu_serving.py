@@ -182,3 +182,46 @@ def test_forward_prefill_paged_bad_page_is_flagged():
                             cuda(torch.from_numpy(table)))
     torch.cuda.synchronize()
     assert M.device_status() & 4
+
+
+@pytest.mark.parametrize("sp", [
+    spec(4, 1, 70000, 69999, 16, 2, 128, 64, 16, seed=91, planted=4),   # CTA-per-row top-k
+    spec(16, 1, 9000, 8999, 32, 4, 64, 32, 8, seed=92),                  # warp-per-row top-k
+])
+def test_forward_decode_in_cuda_graph(sp):
+    """A decode step captured in a CUDA graph (as a serving loop replays it):
+    the top-k and the decode attention launch as programmatic dependents of
+    the kernel before them, which the graph keeps as programmatic edges.
+    Replays give the eager call's bits, and the eager call matches the
+    oracle."""
+    inp = inputs_cpu(sp)
+    sh = M.Shape.of(sp)
+    q, k, v, qi, ki = (cuda(inp.q), cuda(inp.k), cuda(inp.v), cuda(inp.q_idx), cuda(inp.k_idx))
+    ws = M.alloc_workspace(sh, M.OP_FORWARD)
+    o_e, lse_e, sel_e = M.forward(sh, q, k, v, qi, ki, ws=ws)
+    torch.cuda.synchronize()
+    assert M.device_status() == 0
+    o = torch.full_like(o_e, float("nan"))
+    lse = torch.full_like(lse_e, float("nan"))
+    sel = torch.full_like(sel_e, -7)
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=s):
+            for _ in range(3):
+                M.forward(sh, q, k, v, qi, ki, o=o, lse=lse, sel=sel, ws=ws, stream=s)
+    torch.cuda.current_stream().wait_stream(s)
+    for _ in range(4):
+        g.replay()
+    torch.cuda.synchronize()
+    assert M.device_status() == 0
+    assert torch.equal(sel, sel_e)
+    assert torch.equal(o, o_e)
+    assert torch.equal(lse, lse_e)
+    for b in range(sp.batch):
+        sref = oracle_sel(sp, oracle_pooled(sp, inp, b))
+        assert np.array_equal(sel_e[b].cpu().numpy(), sref)
+        O_ref, _ = oracle_attention(sp, inp, sref, b)
+        check_attn(o_e[b], O_ref, f"graph decode b={b}")
+    del g
