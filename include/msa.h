@@ -43,6 +43,11 @@
  * and the optional workspace.  The library never allocates or frees device
  * memory, never synchronises the stream, and all calls are asynchronous on
  * ``stream`` (a cudaStream_t passed as void*; NULL = legacy default stream).
+ * Per-device state (the SM count and the addresses of the library's device
+ * error word and static decode scratch) is looked up on a device's first
+ * call and kept for the life of the process: after cudaDeviceReset on a
+ * device, the library must not be called on that device again in the same
+ * process.
  *
  * Errors: shape, pointer and alignment checks run before any launch and return
  * a status without touching the device.  Device pointers must be 16-byte
