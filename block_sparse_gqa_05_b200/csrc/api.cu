@@ -268,6 +268,7 @@ msa_status msa_workspace_size(const msa_shape* s, msa_op op, size_t* bytes) {
 
 msa_status msa_index_scores(const msa_shape* s, const uint16_t* q_idx, const uint16_t* k_idx,
                             float* pooled, void* stream) {
+  msa::ApiRange nvtx_("msa_index_scores");
   msa_status st = check_shape(s, false, true);
   if (st != MSA_OK) return st;
   if (!q_idx || !k_idx || !pooled) return MSA_ERR_NULL_PTR;
@@ -278,6 +279,7 @@ msa_status msa_index_scores(const msa_shape* s, const uint16_t* q_idx, const uin
 }
 
 msa_status msa_block_topk(const msa_shape* s, const float* pooled, int32_t* sel, void* stream) {
+  msa::ApiRange nvtx_("msa_block_topk");
   msa_status st = check_shape(s, false, false);
   if (st != MSA_OK) return st;
   if (!pooled || !sel) return MSA_ERR_NULL_PTR;
@@ -299,6 +301,7 @@ static msa_status check_attn_ptrs(const uint16_t* q, const uint16_t* k, const ui
 msa_status msa_sparse_attn_prefill(const msa_shape* s, const uint16_t* q, const uint16_t* k,
                                    const uint16_t* v, const int32_t* sel, uint16_t* o,
                                    float* lse, void* ws, size_t ws_bytes, void* stream) {
+  msa::ApiRange nvtx_("msa_sparse_attn_prefill");
   msa_status st = check_shape(s, true, false);
   if (st != MSA_OK) return st;
   if (!prefill_shape_supported(*s)) return MSA_ERR_UNSUPPORTED;
@@ -315,6 +318,7 @@ msa_status msa_sparse_attn_prefill(const msa_shape* s, const uint16_t* q, const 
 msa_status msa_sparse_attn_decode(const msa_shape* s, const uint16_t* q, const uint16_t* k,
                                   const uint16_t* v, const int32_t* sel, uint16_t* o,
                                   float* lse, void* ws, size_t ws_bytes, void* stream) {
+  msa::ApiRange nvtx_("msa_sparse_attn_decode");
   msa_status st = check_shape(s, true, false);
   if (st != MSA_OK) return st;
   if ((st = check_decode(s)) != MSA_OK) return st;
@@ -386,6 +390,7 @@ msa_status msa_forward(const msa_shape* s, const uint16_t* q, const uint16_t* k,
                        const uint16_t* v, const uint16_t* q_idx, const uint16_t* k_idx,
                        uint16_t* o, float* lse, int32_t* sel_out, void* ws, size_t ws_bytes,
                        void* stream) {
+  msa::ApiRange nvtx_("msa_forward");
   msa_status st = check_shape(s, true, true);
   if (st != MSA_OK) return st;
   if ((st = check_attn_ptrs(q, k, v, nullptr, false, o, lse)) != MSA_OK) return st;
@@ -429,6 +434,7 @@ msa_status msa_forward_alignment(const msa_shape* s, const uint16_t* q, const ui
                                  const uint16_t* k_idx, uint16_t* o, float* lse,
                                  int32_t* sel_out, float* kl, void* ws, size_t ws_bytes,
                                  void* stream) {
+  msa::ApiRange nvtx_("msa_forward_alignment");
   msa_status st = check_shape(s, true, true);
   if (st != MSA_OK) return st;
   if ((st = check_attn_ptrs(q, k, v, nullptr, false, o, lse)) != MSA_OK) return st;
@@ -457,6 +463,7 @@ msa_status msa_forward_decode_ragged(const msa_shape* s, const int32_t* seq_lens
                                      const uint16_t* q_idx, const uint16_t* k_idx, uint16_t* o,
                                      float* lse, int32_t* sel_out, void* ws, size_t ws_bytes,
                                      void* stream) {
+  msa::ApiRange nvtx_("msa_forward_decode_ragged");
   return forward_decode_lens(s, seq_lens, PageTable{}, q, k, v, q_idx, k_idx, o, lse, sel_out,
                              ws, ws_bytes, stream);
 }
@@ -466,6 +473,7 @@ msa_status msa_forward_decode_paged(const msa_shape* s, int num_pages, const int
                                     const uint16_t* k, const uint16_t* v, const uint16_t* q_idx,
                                     const uint16_t* k_idx, uint16_t* o, float* lse,
                                     int32_t* sel_out, void* ws, size_t ws_bytes, void* stream) {
+  msa::ApiRange nvtx_("msa_forward_decode_paged");
   if (!s) return MSA_ERR_NULL_PTR;
   if (num_pages < 1) return MSA_ERR_INVALID_SHAPE;
   // 32-bit TMA coordinates (page*G + g) and index-key row offsets
@@ -487,6 +495,7 @@ msa_status msa_forward_prefill_paged(const msa_shape* s, int num_pages,
                                      const uint16_t* q_idx, const uint16_t* k_idx, uint16_t* o,
                                      float* lse, int32_t* sel_out, void* ws, size_t ws_bytes,
                                      void* stream) {
+  msa::ApiRange nvtx_("msa_forward_prefill_paged");
   msa_status st = check_shape(s, true, true);
   if (st != MSA_OK) return st;
   if (num_pages < 1) return MSA_ERR_INVALID_SHAPE;
@@ -529,6 +538,7 @@ msa_status msa_forward_prefill_paged(const msa_shape* s, int num_pages,
 msa_status msa_dense_attn_prefill(const msa_shape* s, const uint16_t* q, const uint16_t* k,
                                   const uint16_t* v, uint16_t* o, float* lse, void* ws,
                                   size_t ws_bytes, void* stream) {
+  msa::ApiRange nvtx_("msa_dense_attn_prefill");
   (void)ws;
   (void)ws_bytes;
   msa_status st = check_shape(s, true, false);
@@ -541,6 +551,7 @@ msa_status msa_dense_attn_prefill(const msa_shape* s, const uint16_t* q, const u
 msa_status msa_dense_attn_decode(const msa_shape* s, const uint16_t* q, const uint16_t* k,
                                  const uint16_t* v, uint16_t* o, float* lse, void* ws,
                                  size_t ws_bytes, void* stream) {
+  msa::ApiRange nvtx_("msa_dense_attn_decode");
   msa_status st = check_shape(s, true, false);
   if (st != MSA_OK) return st;
   if ((st = check_decode(s)) != MSA_OK) return st;

@@ -732,6 +732,7 @@ extern "C" msa_status msa_sparse_attn_decode_static(const msa_shape* s, const ui
                                                     const uint16_t* k, const uint16_t* v,
                                                     const int32_t* sel, uint16_t* o, float* lse,
                                                     void* stream) {
+  msa::ApiRange nvtx_("msa_sparse_attn_decode_static");
   msa_status st = msa::check_decode_static_args(s, q, k, v, sel, o, lse);
   if (st != MSA_OK) return st;
   if (msa::decode_workspace_bytes(*s, false) > MSA_DECODE_STATIC_SCRATCH_BYTES)

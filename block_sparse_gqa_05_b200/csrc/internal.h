@@ -3,6 +3,7 @@
 
 #include <cuda.h>
 #include <cuda_runtime.h>
+#include <nvtx3/nvToolsExt.h>
 #include <stddef.h>
 #include <stdint.h>
 
@@ -46,6 +47,16 @@ class ProfScope {
 
 inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// An NVTX range around each compute call of the C ABI (a timeline tool shows
+// the call with its kernels under it; without a tool attached it costs a
+// pointer test).
+struct ApiRange {
+  explicit ApiRange(const char* name) { nvtxRangePushA(name); }
+  ~ApiRange() { nvtxRangePop(); }
+  ApiRange(const ApiRange&) = delete;
+  ApiRange& operator=(const ApiRange&) = delete;
+};
 
 // Launches a kernel that may start before the previous kernel on the stream
 // has finished (programmatic dependent launch); the kernel itself waits
