@@ -10,7 +10,8 @@
 //  2. cut every column into tiles of 128/r tokens = 128 (token, head) rows and
 //     deal the tiles of every (sequence, group) segment evenly over the CTAs,
 //     segment after segment, so that every CTA gets the same share of every
-//     group's work;
+//     group's work (one contiguous chunk per CTA and segment, the chunks
+//     rotated from segment to segment: see plan_ctas_kernel);
 //  3. persistent tcgen05 kernel: each selected K/V block is TMA-loaded once per
 //     CTA that works on it and reused by every tile of its column; for a tile,
 //     S = Q K^T (TMEM), softmax over the block (causal mask on the local

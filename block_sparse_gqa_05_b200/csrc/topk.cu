@@ -6,8 +6,8 @@
 // are few long rows (decode).  Candidates are blocks 0..b_t-1;
 // the order is (pooled score descending, block index ascending), encoded as a
 // 64-bit key ((order-preserving score bits) << 32 | ~index) so every compare
-// is exact and ties resolve to the lower block index.  Each chunk of 1024
-// scores is filtered against a threshold that provably keeps the (k-1) best
+// is exact and ties resolve to the lower block index.  Each chunk of 512
+// scores (16 per lane) is filtered against a threshold that provably keeps the (k-1) best
 // (the (k-1)-th largest of the 32 per-lane maxima, or the running (k-1)-th
 // best), and the survivors are merged into the running list with a warp
 // bitonic sort.  No exponentials, no full sort of the row.  Thresholds are
