@@ -207,6 +207,9 @@ MSA_DEV void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory");
 // has run this (it still waits for this kernel's completion before reading).
 MSA_DEV void griddep_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;"); }
 
+// Hint: bring the 128-byte line at p toward L2 (no completion to wait for).
+MSA_DEV void prefetch_l2(const void* p) { asm volatile("prefetch.global.L2 [%0];" ::"l"(p)); }
+
 // Generic-proxy shared-memory writes -> visible to the async proxy (tensor core).
 MSA_DEV void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");

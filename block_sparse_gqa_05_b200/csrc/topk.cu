@@ -278,24 +278,37 @@ MSA_DEV bool write_trivial(int32_t* out, int n, int kk, int bt, int k) {
   return false;
 }
 
-// One warp per row: for many rows (prefill).
-__global__ void __launch_bounds__(kWarps * 32, 3)
+// One warp per row: for many rows (prefill).  Four CTAs per SM (64
+// registers): the kernel waits on its loads, so resident warps matter more
+// than the few registers it spills.
+__global__ void __launch_bounds__(kWarps * 32, 4)
     block_topk_kernel(const float* __restrict__ pooled, int32_t* __restrict__ sel,
                       long long rows, int T, int G, int q_off, int nb, int k,
                       const int32_t* __restrict__ lens, int N, uint32_t* err) {
   __shared__ uint64_t scratch[kWarps][kScratch];
-  const int warp = threadIdx.x >> 5;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   uint64_t* buf = scratch[warp];
   const long long nwarps = static_cast<long long>(gridDim.x) * kWarps;
   griddep_launch_dependents();   // the attention may launch (it waits for this kernel)
   griddep_wait();                // the pooled scores of the kernel before
   const bool vec = (nb & 3) == 0;
-  for (long long r = static_cast<long long>(blockIdx.x) * kWarps + warp; r < rows; r += nwarps) {
-    // rows < 2^31 (checked by the API): 32-bit index math
-    const uint32_t tg = static_cast<uint32_t>(r) / static_cast<uint32_t>(G);
+  // query position of row rr (rows < 2^31, checked by the API: 32-bit index math)
+  auto row_pos = [&](long long rr) {
+    const uint32_t tg = static_cast<uint32_t>(rr) / static_cast<uint32_t>(G);
     const int t = static_cast<int>(tg % static_cast<uint32_t>(T));
-    const int pos = lens ? ragged_len(lens, static_cast<int>(tg / static_cast<uint32_t>(T)), N, err) - 1
-                         : q_off + t;
+    return lens ? ragged_len(lens, static_cast<int>(tg / static_cast<uint32_t>(T)), N, err) - 1
+                : q_off + t;
+  };
+  for (long long r = static_cast<long long>(blockIdx.x) * kWarps + warp; r < rows; r += nwarps) {
+    // the warp's next row: its first two chunks of candidate scores toward
+    // L2 (one 128-byte line per lane) while this row is ranked, so that its
+    // first loads do not wait on DRAM
+    if (r + nwarps < rows) {
+      const float* nsrc = pooled + (r + nwarps) * nb;
+      const int nn = min(row_pos(r + nwarps) >> 7, 2 * kChunk);
+      if (lane * 32 < nn) prefetch_l2(nsrc + lane * 32);
+    }
+    const int pos = row_pos(r);
     const int bt = pos >> 7;
     const int n = bt;                         // candidates 0 .. bt-1
     const int kk = min(k - 1, n);
