@@ -148,6 +148,12 @@ MSA_DEV void scan_chunks(const float* __restrict__ src, int n, int kk, bool vec,
                          uint64_t* buf, uint64_t (&best)[2], int& have) {
   const int lane = threadIdx.x & 31;
   for (int base = c0 * kChunk; base < n; base += cs * kChunk) {
+    // one warp per row: two chunks ahead toward L2 (16 lanes, a 128-byte
+    // line each), so that a long row's loads do not wait on DRAM
+    if (cs == 1) {
+      const int ahead = base + 2 * kChunk + lane * 32;
+      if (lane < kChunk / 32 && ahead < n) prefetch_l2(src + ahead);
+    }
     // this lane's scores: block base + x*128 + lane*4 + e, as order-preserving keys
     uint32_t uk[kPer];
 #pragma unroll
@@ -278,10 +284,10 @@ MSA_DEV bool write_trivial(int32_t* out, int n, int kk, int bt, int k) {
   return false;
 }
 
-// One warp per row: for many rows (prefill).  Four CTAs per SM (64
+// One warp per row: for many rows (prefill).  Five CTAs per SM (48
 // registers): the kernel waits on its loads, so resident warps matter more
 // than the few registers it spills.
-__global__ void __launch_bounds__(kWarps * 32, 4)
+__global__ void __launch_bounds__(kWarps * 32, 5)
     block_topk_kernel(const float* __restrict__ pooled, int32_t* __restrict__ sel,
                       long long rows, int T, int G, int q_off, int nb, int k,
                       const int32_t* __restrict__ lens, int N, uint32_t* err) {
